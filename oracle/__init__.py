@@ -1,0 +1,231 @@
+"""CPU oracle for the causal dynamic short convolution -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline / reference legs of
+``bench.py`` may import this package.  The product library never loads it and shares
+no code with it.
+
+The arithmetic lives in ``dsc_oracle.c`` (plain single-threaded C, double precision),
+written from "Convolucoes Curtas Dinamicas Melhoram Transformers"
+(gist.science/pt/paper/2606.03825), section "Metodologia > Convolucoes Curtas
+Dinamicas" (Mecanismo, Parametrizacao, Posicionamento).  This module only compiles
+that file with gcc, loads it with ctypes and marshals numpy float64 arrays.
+
+Parity pins for every function are in ``tests/test_oracle_pins.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "dsc_oracle.c")
+_LIB = os.path.join(_HERE, "libdsc_oracle.so")
+_lock = threading.Lock()
+_default = None
+
+_GCC_FLAGS = ["gcc", "-O2", "-fno-fast-math", "-ffp-contract=off", "-std=c99", "-shared", "-fPIC"]
+
+
+def build(force: bool = False) -> str:
+    """Compile dsc_oracle.c into libdsc_oracle.so (gcc -O2, strict IEEE double)."""
+    with _lock:
+        if (not force and os.path.exists(_LIB)
+                and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC)):
+            return _LIB
+        tmp = _LIB + ".tmp.%d" % os.getpid()
+        subprocess.run(_GCC_FLAGS + ["-o", tmp, _SRC], check=True)
+        os.replace(tmp, _LIB)
+        return _LIB
+
+
+def source() -> str:
+    with open(_SRC) as f:
+        return f.read()
+
+
+def _bind(lib):
+    dp = ctypes.POINTER(ctypes.c_double)
+    i = ctypes.c_int
+    sig = {
+        "oracle_fwd": (None, [dp, dp, dp, i, i, i, i, i]),
+        "oracle_lowrank_weights": (None, [dp, dp, dp, i, i, i, i, i, i]),
+        "oracle_fwd_lowrank": (i, [dp, dp, dp, dp, i, i, i, i, i, i]),
+        "oracle_bwd": (None, [dp, dp, dp, dp, dp, i, i, i, i, i]),
+        "oracle_bwd_lowrank": (i, [dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, i]),
+        "oracle_static_fwd": (None, [dp, dp, dp, i, i, i, i]),
+        "oracle_static_bwd": (None, [dp, dp, dp, dp, dp, i, i, i, i]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+def _in(a, shape):
+    a = np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+    if tuple(a.shape) != tuple(shape):
+        raise ValueError("oracle: expected shape %s, got %s" % (shape, a.shape))
+    return a
+
+
+def _p(a):
+    return a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _check_dims(B, T, D, G, W, R=1):
+    if min(B, T, D, G, W, R) < 1 or D % G:
+        raise ValueError("oracle: bad sizes B=%d T=%d D=%d G=%d W=%d R=%d" % (B, T, D, G, W, R))
+
+
+class Oracle:
+    """numpy front end over one compiled copy of the oracle source."""
+
+    def __init__(self, lib):
+        self._l = lib
+
+    def fwd(self, x, w, G):
+        """y = x + sum_k w(t)_k * x_{t-k}; x [B,T,D], w [B,T,D/G,W]."""
+        x = np.asarray(x)
+        B, T, D = x.shape
+        W = np.asarray(w).shape[-1]
+        _check_dims(B, T, D, G, W)
+        x = _in(x, (B, T, D))
+        w = _in(w, (B, T, D // G, W))
+        y = np.empty_like(x)
+        self._l.oracle_fwd(_p(x), _p(w), _p(y), B, T, D, G, W)
+        return y
+
+    def lowrank_weights(self, z, U, D, G, W):
+        """w = reshape(z U, [B,T,D/G,W]) by a plain triple loop."""
+        z = np.asarray(z)
+        B, T, R = z.shape
+        _check_dims(B, T, D, G, W, R)
+        z = _in(z, (B, T, R))
+        U = _in(U, (R, (D // G) * W))
+        w = np.empty((B, T, D // G, W), dtype=np.float64)
+        self._l.oracle_lowrank_weights(_p(z), _p(U), _p(w), B, T, D, G, W, R)
+        return w
+
+    def fwd_lowrank(self, x, z, U, G, W):
+        """y = x + dynconv(x; w = z U); x [B,T,D], z [B,T,R], U [R,(D/G)*W]."""
+        x = np.asarray(x)
+        B, T, D = x.shape
+        R = np.asarray(z).shape[-1]
+        _check_dims(B, T, D, G, W, R)
+        x = _in(x, (B, T, D))
+        z = _in(z, (B, T, R))
+        U = _in(U, (R, (D // G) * W))
+        y = np.empty_like(x)
+        if self._l.oracle_fwd_lowrank(_p(x), _p(z), _p(U), _p(y), B, T, D, G, W, R):
+            raise MemoryError("oracle_fwd_lowrank")
+        return y
+
+    def bwd(self, x, w, dy, G):
+        """Backward of fwd: returns (dx [B,T,D], dw [B,T,D/G,W])."""
+        x = np.asarray(x)
+        B, T, D = x.shape
+        W = np.asarray(w).shape[-1]
+        _check_dims(B, T, D, G, W)
+        x = _in(x, (B, T, D))
+        w = _in(w, (B, T, D // G, W))
+        dy = _in(dy, (B, T, D))
+        dx = np.empty_like(x)
+        dw = np.empty_like(w)
+        self._l.oracle_bwd(_p(x), _p(w), _p(dy), _p(dx), _p(dw), B, T, D, G, W)
+        return dx, dw
+
+    def bwd_lowrank(self, x, z, U, dy, G, W):
+        """Backward of fwd_lowrank: returns (dx [B,T,D], dz [B,T,R], dU [R,(D/G)*W])."""
+        x = np.asarray(x)
+        B, T, D = x.shape
+        R = np.asarray(z).shape[-1]
+        _check_dims(B, T, D, G, W, R)
+        N = (D // G) * W
+        x = _in(x, (B, T, D))
+        z = _in(z, (B, T, R))
+        U = _in(U, (R, N))
+        dy = _in(dy, (B, T, D))
+        dx = np.empty_like(x)
+        dz = np.empty_like(z)
+        dU = np.empty_like(U)
+        if self._l.oracle_bwd_lowrank(_p(x), _p(z), _p(U), _p(dy), _p(dx), _p(dz), _p(dU),
+                                      B, T, D, G, W, R):
+            raise MemoryError("oracle_bwd_lowrank")
+        return dx, dz, dU
+
+    def static_fwd(self, x, ws):
+        """y = x + depthwise causal conv with fixed filters ws [D,W]."""
+        x = np.asarray(x)
+        B, T, D = x.shape
+        W = np.asarray(ws).shape[-1]
+        _check_dims(B, T, D, 1, W)
+        x = _in(x, (B, T, D))
+        ws = _in(ws, (D, W))
+        y = np.empty_like(x)
+        self._l.oracle_static_fwd(_p(x), _p(ws), _p(y), B, T, D, W)
+        return y
+
+    def static_bwd(self, x, ws, dy):
+        """Backward of static_fwd: returns (dx [B,T,D], dws [D,W])."""
+        x = np.asarray(x)
+        B, T, D = x.shape
+        W = np.asarray(ws).shape[-1]
+        _check_dims(B, T, D, 1, W)
+        x = _in(x, (B, T, D))
+        ws = _in(ws, (D, W))
+        dy = _in(dy, (B, T, D))
+        dx = np.empty_like(x)
+        dws = np.empty_like(ws)
+        self._l.oracle_static_bwd(_p(x), _p(ws), _p(dy), _p(dx), _p(dws), B, T, D, W)
+        return dx, dws
+
+
+def default() -> Oracle:
+    global _default
+    if _default is None:
+        _default = Oracle(_bind(ctypes.CDLL(build())))
+    return _default
+
+
+def from_source(text: str, workdir: str) -> Oracle:
+    """Compile a variant of the oracle source (used by the pin tests to plant a
+    mistake on the CPU and check that some pin catches it)."""
+    src = os.path.join(workdir, "variant.c")
+    lib = os.path.join(workdir, "libvariant.so")
+    with open(src, "w") as f:
+        f.write(text)
+    subprocess.run(_GCC_FLAGS + ["-o", lib, src], check=True)
+    return Oracle(_bind(ctypes.CDLL(lib)))
+
+
+def fwd(x, w, G):
+    return default().fwd(x, w, G)
+
+
+def lowrank_weights(z, U, D, G, W):
+    return default().lowrank_weights(z, U, D, G, W)
+
+
+def fwd_lowrank(x, z, U, G, W):
+    return default().fwd_lowrank(x, z, U, G, W)
+
+
+def bwd(x, w, dy, G):
+    return default().bwd(x, w, dy, G)
+
+
+def bwd_lowrank(x, z, U, dy, G, W):
+    return default().bwd_lowrank(x, z, U, dy, G, W)
+
+
+def static_fwd(x, ws):
+    return default().static_fwd(x, ws)
+
+
+def static_bwd(x, ws, dy):
+    return default().static_bwd(x, ws, dy)
