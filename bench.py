@@ -1,0 +1,379 @@
+#!/usr/bin/env python
+"""Benchmark: fused low-rank causal dynamic short convolution, forward + backward.
+
+One step = dsc_fwd_lowrank followed by dsc_bwd_lowrank over one batch of the chosen
+workload (default: the stacked-QKV shape x [8,2048,6144], z [8,2048,32],
+U [32,24576], G=1, W=4, dy ~N(0,1)).  Inputs are synthetic and seeded; x alone
+(201 MB) exceeds the 126 MB L2, so no flush is inserted between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+Under torchrun (N > 1) every rank runs the whole workload on its own batch (weak
+scaling) and the per-step weight gradient dU is summed across ranks with NCCL, the
+one exchange a data-parallel training step has for this op.  Time is measured with
+CUDA events on the launching stream, bracketed by a barrier and a synchronize, and
+the maximum over ranks is reported.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import dsc_inputs as di  # noqa: E402
+
+METRIC = "achieved HBM GB/s (% of peak) and tokens/s, fused low-rank dyn-conv fwd+bwd"
+
+
+def algorithmic_bytes(wl):
+    """Bytes that must cross HBM once per call (each tensor counted once)."""
+    e = 2 if wl.dtype == "bf16" else 4
+    x = wl.tokens * wl.D * e
+    z = wl.tokens * wl.R * e
+    U = wl.R * wl.N * e
+    fwd = x + z + U + x                                 # read x, z, U; write y
+    bwd = 3 * x + z + U + wl.tokens * wl.R * 4 + wl.R * wl.N * 4   # dy, x, dx; z, U; dz, dU
+    return fwd, bwd
+
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(prefix="dsc_clocks_", suffix=".csv")
+            os.close(fd)
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.fh, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.fh.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [s.strip() for s in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and args.impl == "ours":
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v, world, device):
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+def oracle_sample_rate(wl, budget_s=15.0):
+    """Time the CPU oracle (fwd + bwd) on a bounded sample of the workload: the first
+    L tokens of one sequence, with L chosen so the run takes about `budget_s`.
+    Returns (tokens/s, description, seconds)."""
+    import numpy as np
+    import oracle
+    t = di.make(di.scaled(wl, B=1, T=min(wl.T, 2048)), "cpu", ("x", "z", "U", "dy"))
+    f = {k: v.to(torch.float64).numpy() for k, v in t.items()}
+
+    def run(L):
+        t0 = time.perf_counter()
+        oracle.fwd_lowrank(f["x"][:, :L], f["z"][:, :L], f["U"], wl.G, wl.W)
+        oracle.bwd_lowrank(f["x"][:, :L], f["z"][:, :L], f["U"], f["dy"][:, :L], wl.G, wl.W)
+        return time.perf_counter() - t0
+
+    L0 = 16
+    dt0 = run(L0)
+    L = int(max(L0, min(f["x"].shape[1], L0 * budget_s / max(dt0, 1e-6))))
+    dt = run(L) if L != L0 else dt0
+    desc = ("oracle fwd+bwd (plain C, fp64, 1 thread) on the first %d tokens of one "
+            "sequence of the %s workload (D=%d, R=%d, G=%d, W=%d)" % (L, wl.name, wl.D, wl.R, wl.G, wl.W))
+    return L / dt, desc, dt
+
+
+def run_reference(args, wl, world, rank):
+    """The reference arm: the CPU oracle as it stands, on host cores."""
+    if rank != 0:
+        return 0
+    rates = []
+    desc = ""
+    for i in range(args.warmup + args.steps):
+        rate, desc, _ = oracle_sample_rate(wl, budget_s=args.ref_budget)
+        if i >= args.warmup:
+            rates.append(rate)
+    v = statistics.median(rates)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * wl.tokens / v, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,s^2))",
+        "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "D": wl.D, "G": wl.G, "W": wl.W,
+                   "R": wl.R, "tokens_per_step": wl.tokens},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, wl, world, rank, local):
+    import dynamic_short_convolutions_causal_b200 as dsc
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    wl_rank = di.scaled(wl, seed=wl.seed + 1000 * rank)
+    t = di.make(wl_rank, dev, ("x", "z", "U", "dy"))
+    x, z, U, dy = t["x"], t["z"], t["U"], t["dy"]
+    G, W, R = wl.G, wl.W, wl.R
+    y = torch.empty_like(x)
+    dx = torch.empty_like(x)
+    dz = torch.empty((wl.B, wl.T, R), dtype=torch.float32, device=dev)
+    dU = torch.empty((R, wl.N), dtype=torch.float32, device=dev)
+    ws = dsc.workspace(dsc.dsc_bwd_lowrank_workspace_bytes(wl.B, wl.T, wl.D, G, W, R, x.dtype), dev)
+    path = dsc.dsc_lowrank_path(wl.B, wl.T, wl.D, G, W, R, x.dtype)
+    stream = torch.cuda.current_stream(dev)
+    if world > 1:
+        import torch.distributed as dist
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        dsc.dsc_fwd_lowrank(x, z, U, y, G, W)
+        if ev is not None:
+            ev[1].record(stream)
+        dsc.dsc_bwd_lowrank(x, z, U, dy, dx, dz, dU, ws, G, W)
+        if ev is not None:
+            ev[2].record(stream)
+        if world > 1:
+            dist.all_reduce(dU)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks = Clocks(local)
+    clocks.start()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ck = clocks.stop()
+    ms = start.elapsed_time(end)
+    ms = max_over_ranks(ms, world, dev)
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    ms_step = ms / args.steps
+    tokens_s = wl.tokens * world / (ms_step * 1e-3)
+    fwd_b, bwd_b = algorithmic_bytes(wl)
+    peak, peak_kind = read_peaks()
+    gbs_step = (fwd_b + bwd_b) / (ms_step * 1e-3) / 1e9
+    dom = ("dsc_bwd_lowrank", bwd_b, bwd_ms) if bwd_ms >= fwd_ms else ("dsc_fwd_lowrank", fwd_b, fwd_ms)
+    achieved = dom[1] / (dom[2] * 1e-3) / 1e9
+    launches_fwd = 1 if path == 1 else 1
+    launches_bwd = 2 if path == 1 else 5
+    traffic = load_traffic(dom[0], wl)
+
+    # end to end through the public API with host buffers (pinned), copies inside the region
+    e2e = None
+    if not args.no_e2e:
+        e2e = measure_e2e(dsc, t, y, dx, dz, dU, ws, wl, world, dev, args)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, desc, _ = oracle_sample_rate(wl, budget_s=args.cpu_budget)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": tokens_s, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": wl.dtype,
+            "data": "synthetic (seeded N(0,s^2); no dataset)",
+            "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "D": wl.D, "G": G, "W": W, "R": R,
+                       "tokens_per_step_per_gpu": wl.tokens, "parallelism": "dp%d" % world,
+                       "l2": "inputs larger than L2 (x is %.0f MB), no flush" % (wl.tokens * wl.D * 2 / 1e6),
+                       "path": "tcgen05" if path == 1 else "cuda-cores"},
+            "hbm_gbs_step": gbs_step, "hbm_pct_of_peak_step": 100.0 * gbs_step / peak,
+            "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+            "fwd_gbs": fwd_b / (fwd_ms * 1e-3) / 1e9, "bwd_gbs": bwd_b / (bwd_ms * 1e-3) / 1e9,
+            "roofline": {"bound": "hbm", "kernel": dom[0], "achieved": achieved, "peak": peak,
+                         "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": traffic, "algorithmic_bytes": dom[1]},
+            "gpu_launches": (launches_fwd + launches_bwd) * args.steps,
+            "e2e": e2e, "cpu_baseline": cpu, "clocks": ck,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def load_traffic(kernel, wl):
+    """Per-launch DRAM bytes from a committed ncu summary, if one matches the current
+    kernel build (profiles/traffic.json); null otherwise."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        ent = d.get(wl.name, {}).get(kernel)
+        return ent["bytes_per_launch"] if ent else None
+    except Exception:
+        return None
+
+
+def measure_e2e(dsc, t, y, dx, dz, dU, ws, wl, world, dev, args):
+    G, W = wl.G, wl.W
+    hx = t["x"].cpu().pin_memory()
+    hz = t["z"].cpu().pin_memory()
+    hU = t["U"].cpu().pin_memory()
+    hdy = t["dy"].cpu().pin_memory()
+    hy = torch.empty_like(hx).pin_memory()
+    hdx = torch.empty_like(hx).pin_memory()
+    hdz = torch.empty(dz.shape, dtype=dz.dtype).pin_memory()
+    hdU = torch.empty(dU.shape, dtype=dU.dtype).pin_memory()
+    x = torch.empty_like(t["x"])
+    z = torch.empty_like(t["z"])
+    U = torch.empty_like(t["U"])
+    dy = torch.empty_like(t["dy"])
+    stream = torch.cuda.current_stream(dev)
+    h2d = sum(a.numel() * a.element_size() for a in (hx, hz, hU, hdy))
+    d2h = sum(a.numel() * a.element_size() for a in (hy, hdx, hdz, hdU))
+    if world > 1:
+        import torch.distributed as dist
+
+    def step():
+        x.copy_(hx, non_blocking=True)
+        z.copy_(hz, non_blocking=True)
+        U.copy_(hU, non_blocking=True)
+        dy.copy_(hdy, non_blocking=True)
+        dsc.dsc_fwd_lowrank(x, z, U, y, G, W)
+        dsc.dsc_bwd_lowrank(x, z, U, dy, dx, dz, dU, ws, G, W)
+        if world > 1:
+            dist.all_reduce(dU)
+        hy.copy_(y, non_blocking=True)
+        hdx.copy_(dx, non_blocking=True)
+        hdz.copy_(dz, non_blocking=True)
+        hdU.copy_(dU, non_blocking=True)
+
+    for _ in range(max(1, args.warmup // 2)):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    steps = max(2, min(args.steps, 10))
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        step()
+    e.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(s.elapsed_time(e) / steps, world, dev)
+    return {"value": wl.tokens * world / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="lowrank_qkv", choices=["lowrank_qkv", "lowrank_mlp"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--ref-budget", type=float, default=8.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    wl = di.WORKLOADS[args.workload]
+    world, rank, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            return run_reference(args, wl, world, rank)
+        return run_ours(args, wl, world, rank, local)
+    finally:
+        if world > 1 and args.impl == "ours":
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,193 @@
+"""Python binding of libdsc.so, the B200 (sm_100a) causal dynamic short convolution.
+
+Argument marshalling only: every function here derives the sizes from torch tensor
+shapes, checks devices and dtypes, and calls the C entry point of the same name on the
+current CUDA stream.  All arithmetic runs in the library's CUDA kernels; there is no
+CPU or PyTorch fallback.  Importing this module fails loudly when libdsc.so is
+missing (build it with ``python -m dynamic_short_convolutions_causal_b200.build``).
+
+Operation ("Convolucoes Curtas Dinamicas Melhoram Transformers", Metodologia >
+Convolucoes Curtas Dinamicas): y_t = x_t + sum_{k<W} w(t)_k * x_{t-k}, with explicit,
+low-rank (w = z U, formed on chip) or static filters; see include/dsc.h.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "DscError", "lib", "lib_path", "dsc_fwd", "dsc_fwd_lowrank", "dsc_bwd_lowrank",
+    "dsc_bwd_lowrank_workspace_bytes", "dsc_bwd", "dsc_static_fwd", "dsc_static_bwd",
+    "dsc_static_bwd_workspace_bytes", "dsc_lowrank_path", "DSC_F32", "DSC_BF16",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_HERE, "libdsc.so")
+
+DSC_OK, DSC_ERR_INVALID_ARG, DSC_ERR_UNSUPPORTED, DSC_ERR_CUDA = 0, 1, 2, 3
+DSC_F32, DSC_BF16 = 0, 1
+
+
+class DscError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__("%s (status %d)" % (detail, status))
+        self.status = status
+
+
+def _load():
+    if not os.path.exists(lib_path):
+        raise ImportError(
+            "libdsc.so not found at %s: build it with "
+            "`python -m dynamic_short_convolutions_causal_b200.build`" % lib_path)
+    L = ctypes.CDLL(lib_path)
+    vp, i, sz, fp = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
+    sigs = {
+        "dsc_fwd": (i, [vp, vp, vp, i, i, i, i, i, i, vp]),
+        "dsc_fwd_lowrank": (i, [vp, vp, vp, vp, i, i, i, i, i, i, i, vp]),
+        "dsc_bwd_lowrank_workspace_bytes": (sz, [i, i, i, i, i, i, i]),
+        "dsc_bwd_lowrank": (i, [vp, vp, vp, vp, vp, fp, fp, vp, sz, i, i, i, i, i, i, i, vp]),
+        "dsc_bwd": (i, [vp, vp, vp, vp, fp, i, i, i, i, i, i, vp]),
+        "dsc_static_fwd": (i, [vp, vp, vp, i, i, i, i, i, vp]),
+        "dsc_static_bwd_workspace_bytes": (sz, [i, i, i, i, i]),
+        "dsc_static_bwd": (i, [vp, vp, vp, vp, fp, vp, sz, i, i, i, i, i, vp]),
+        "dsc_lowrank_path": (i, [i, i, i, i, i, i, i]),
+        "dsc_status_string": (ctypes.c_char_p, [i]),
+        "dsc_last_error": (ctypes.c_char_p, []),
+    }
+    for name, (res, args) in sigs.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    return L
+
+
+lib = _load()
+
+
+def _check(status: int):
+    if status != DSC_OK:
+        raise DscError(status, (lib.dsc_last_error() or b"").decode() or
+                       lib.dsc_status_string(status).decode())
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return DSC_BF16
+    if t.dtype == torch.float32:
+        return DSC_F32
+    raise TypeError("dsc: unsupported dtype %s (bf16 or fp32)" % t.dtype)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("dsc: tensors must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("dsc: tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(t: torch.Tensor):
+    return ctypes.c_void_p(torch.cuda.current_stream(t.device).cuda_stream)
+
+
+def _same(ref, *ts):
+    for t in ts:
+        if t.device != ref.device:
+            raise ValueError("dsc: all tensors must be on %s" % ref.device)
+
+
+def dsc_fwd(x, w, y, G: int):
+    """y = x + dynconv(x; w); x, y [B,T,D], w [B,T,D/G,W] (same dtype)."""
+    B, T, D = x.shape
+    W = w.shape[-1]
+    _same(x, w, y)
+    with torch.cuda.device(x.device):
+        _check(lib.dsc_fwd(_ptr(x), _ptr(w), _ptr(y), B, T, D, G, W, _dt(x), _stream(x)))
+    return y
+
+
+def dsc_fwd_lowrank(x, z, U, y, G: int, W: int):
+    """y = x + dynconv(x; w = z U formed on chip); z [B,T,R], U [R,(D/G)*W]."""
+    B, T, D = x.shape
+    R = z.shape[-1]
+    _same(x, z, U, y)
+    with torch.cuda.device(x.device):
+        _check(lib.dsc_fwd_lowrank(_ptr(x), _ptr(z), _ptr(U), _ptr(y), B, T, D, G, W, R, _dt(x),
+                                   _stream(x)))
+    return y
+
+
+def dsc_bwd_lowrank_workspace_bytes(B, T, D, G, W, R, dtype=torch.bfloat16) -> int:
+    dt = DSC_BF16 if dtype == torch.bfloat16 else DSC_F32
+    return int(lib.dsc_bwd_lowrank_workspace_bytes(B, T, D, G, W, R, dt))
+
+
+def dsc_bwd_lowrank(x, z, U, dy, dx, dz, dU, workspace, G: int, W: int):
+    """dx [B,T,D] (x's dtype), dz [B,T,R] fp32, dU [R,(D/G)*W] fp32 (overwritten).
+    ``workspace`` is a device tensor of at least dsc_bwd_lowrank_workspace_bytes()."""
+    B, T, D = x.shape
+    R = z.shape[-1]
+    _same(x, z, U, dy, dx, dz, dU)
+    if dz.dtype != torch.float32 or dU.dtype != torch.float32:
+        raise TypeError("dsc_bwd_lowrank: dz and dU must be fp32")
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    with torch.cuda.device(x.device):
+        _check(lib.dsc_bwd_lowrank(_ptr(x), _ptr(z), _ptr(U), _ptr(dy), _ptr(dx), _ptr(dz),
+                                   _ptr(dU), _ptr(workspace), ws_bytes, B, T, D, G, W, R, _dt(x),
+                                   _stream(x)))
+    return dx, dz, dU
+
+
+def dsc_bwd(x, w, dy, dx, dw, G: int):
+    """Explicit-filter backward: dx [B,T,D] (x's dtype), dw [B,T,D/G,W] fp32."""
+    B, T, D = x.shape
+    W = w.shape[-1]
+    _same(x, w, dy, dx, dw)
+    if dw.dtype != torch.float32:
+        raise TypeError("dsc_bwd: dw must be fp32")
+    with torch.cuda.device(x.device):
+        _check(lib.dsc_bwd(_ptr(x), _ptr(w), _ptr(dy), _ptr(dx), _ptr(dw), B, T, D, G, W, _dt(x),
+                           _stream(x)))
+    return dx, dw
+
+
+def dsc_static_fwd(x, w, y):
+    """y = x + depthwise causal conv with fixed filters w [D,W]."""
+    B, T, D = x.shape
+    W = w.shape[-1]
+    _same(x, w, y)
+    with torch.cuda.device(x.device):
+        _check(lib.dsc_static_fwd(_ptr(x), _ptr(w), _ptr(y), B, T, D, W, _dt(x), _stream(x)))
+    return y
+
+
+def dsc_static_bwd_workspace_bytes(B, T, D, W, dtype=torch.bfloat16) -> int:
+    dt = DSC_BF16 if dtype == torch.bfloat16 else DSC_F32
+    return int(lib.dsc_static_bwd_workspace_bytes(B, T, D, W, dt))
+
+
+def dsc_static_bwd(x, w, dy, dx, dw, workspace):
+    """dx [B,T,D] (x's dtype) and dw [D,W] fp32 summed over all tokens."""
+    B, T, D = x.shape
+    W = w.shape[-1]
+    _same(x, w, dy, dx, dw, workspace)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    with torch.cuda.device(x.device):
+        _check(lib.dsc_static_bwd(_ptr(x), _ptr(w), _ptr(dy), _ptr(dx), _ptr(dw), _ptr(workspace),
+                                  ws_bytes, B, T, D, W, _dt(x), _stream(x)))
+    return dx, dw
+
+
+def dsc_lowrank_path(B, T, D, G, W, R, dtype=torch.bfloat16) -> int:
+    """1: tensor-core kernels, 0: CUDA-core kernels, -1: invalid sizes."""
+    dt = DSC_BF16 if dtype == torch.bfloat16 else DSC_F32
+    return int(lib.dsc_lowrank_path(B, T, D, G, W, R, dt))
+
+
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """A 256-byte aligned device scratch buffer of at least ``nbytes`` bytes."""
+    return torch.empty(max(int(nbytes), 16), dtype=torch.uint8, device=device)

@@ -1,0 +1,36 @@
+// Internal launcher declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <algorithm>
+
+namespace dsc {
+
+// CUDA-core kernels (simt.cu)
+void launch_conv_fwd(const void *x, const void *w, void *y, int B, int T, int D, int G, int W,
+                     bool bf16, bool is_static, cudaStream_t s);
+void launch_conv_dx(const void *w, bool w_is_f32, const void *dy, void *dx, int B, int T, int D,
+                    int G, int W, bool bf16, bool is_static, cudaStream_t s);
+int static_dw_partials(int B, int T);
+void launch_static_dw(const void *x, const void *dy, float *part, float *dw, int B, int T, int D,
+                      int W, bool bf16, cudaStream_t s);
+void launch_dyn_dw(const void *x, const void *dy, float *dw, int B, int T, int D, int G, int W,
+                   bool bf16, cudaStream_t s);
+void launch_lowrank_fwd_simt(const void *x, const void *z, const void *U, void *y, int B, int T,
+                             int D, int G, int W, int R, bool bf16, cudaStream_t s);
+size_t lowrank_bwd_simt_workspace(int B, int T, int D, int G, int W);
+void launch_lowrank_bwd_simt(const void *x, const void *z, const void *U, const void *dy, void *dx,
+                             float *dz, float *dU, void *ws, int B, int T, int D, int G, int W,
+                             int R, bool bf16, cudaStream_t s);
+
+// Tensor-core (tcgen05) low-rank kernels (tc_fwd.cu, tc_bwd.cu)
+bool tc_lowrank_supported(int B, int T, int D, int G, int W, int R, bool bf16);
+cudaError_t launch_tc_lowrank_fwd(const void *x, const void *z, const void *U, void *y, int B,
+                                  int T, int D, int G, int W, int R, cudaStream_t s);
+size_t tc_lowrank_bwd_workspace(int B, int T, int D, int G, int W, int R);
+cudaError_t launch_tc_lowrank_bwd(const void *x, const void *z, const void *U, const void *dy,
+                                  void *dx, float *dz, float *dU, void *ws, int B, int T, int D,
+                                  int G, int W, int R, cudaStream_t s);
+
+}  // namespace dsc

@@ -1,0 +1,540 @@
+// CUDA-core kernels: the HBM-streaming explicit and static convolutions (forward and
+// backward), and the general-shape low-rank path used where the tensor-core kernels
+// do not apply (fp32, or R / G / W outside the tensor-core shapes).
+//
+// The operation is the causal dynamic short convolution of "Convolucoes Curtas
+// Dinamicas Melhoram Transformers" (Metodologia > Convolucoes Curtas Dinamicas):
+//   y_t[c] = x_t[c] + sum_{k<W} f_t[c,k] x_{t-k}[c],   x_{t'} = 0 for t' < 0,
+// and its chain-rule backward.
+//
+// Streaming layout: one thread owns one 16-byte vector of channels (8 bf16 or 4 fp32)
+// and walks a chunk of tokens of one sequence, keeping the W-1 previous rows of x in
+// registers, so x and y each cross HBM once (the W-1 halo rows at a chunk start are
+// re-read, mostly from L2).
+#include "common.cuh"
+#include "internal.h"
+
+namespace dsc {
+
+// Filter taps for the thread's V channels at token row `bt` (flattened b*T+t).
+//   STATIC:  ws[c,k]                  (loaded once by the caller)
+//   G == 1:  w[bt, c, k] contiguous   (V*W elements, 16-byte vectors)
+//   G % V == 0: one group for all V channels (W elements)
+//   else:    per channel
+template <typename T, typename TW, int W>
+__device__ __forceinline__ void load_taps(const TW *__restrict__ w, size_t bt, int c0, int D,
+                                          int G, float (&f)[W][Vec<T>::N]) {
+    constexpr int V = Vec<T>::N;
+    const int NG = D / G;
+    if (G == 1 && sizeof(TW) == sizeof(T)) {
+        // V*W contiguous elements; (bt*D + c0)*W*sizeof(TW) is a multiple of 16.
+        const TW *p = w + (bt * (size_t)D + c0) * W;
+        float tmp[V * W];
+#pragma unroll
+        for (int q = 0; q < W; ++q) {
+            float v[V];
+            Vec<T>::load(reinterpret_cast<const T *>(p) + q * V, v);
+#pragma unroll
+            for (int e = 0; e < V; ++e) tmp[q * V + e] = v[e];
+        }
+#pragma unroll
+        for (int i = 0; i < V; ++i)
+#pragma unroll
+            for (int k = 0; k < W; ++k) f[k][i] = tmp[i * W + k];
+    } else if (G % V == 0) {
+        const TW *p = w + (bt * NG + c0 / G) * W;
+        float t[W];
+#pragma unroll
+        for (int k = 0; k < W; ++k) t[k] = to_f(p[k]);
+#pragma unroll
+        for (int i = 0; i < V; ++i)
+#pragma unroll
+            for (int k = 0; k < W; ++k) f[k][i] = t[k];
+    } else {
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            const TW *p = w + (bt * NG + (c0 + i) / G) * W;
+#pragma unroll
+            for (int k = 0; k < W; ++k) f[k][i] = to_f(p[k]);
+        }
+    }
+}
+
+// ------------------------------------------------------------------ forward
+template <typename T, int W, bool STATIC>
+__global__ void __launch_bounds__(128)
+k_conv_fwd(const T *__restrict__ x, const T *__restrict__ w, T *__restrict__ y,
+           int B, int T_, int D, int G, int chunk) {
+    constexpr int V = Vec<T>::N;
+    const int v = blockIdx.x * blockDim.x + threadIdx.x;
+    if (v >= D / V) return;
+    const int nchunks = cdiv(T_, chunk);
+    const int b = blockIdx.y / nchunks;
+    const int t0 = (blockIdx.y % nchunks) * chunk;
+    const int t1 = min(t0 + chunk, T_);
+    const int c0 = v * V;
+    const size_t row0 = (size_t)b * T_;
+
+    float win[W][V];   // win[k] = x_{t-k}; win[0] is filled each step
+#pragma unroll
+    for (int k = 1; k < W; ++k) {
+        const int t = t0 - k;
+        if (t >= 0) {
+            Vec<T>::load(x + (row0 + t) * D + c0, win[k]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < V; ++i) win[k][i] = 0.f;
+        }
+    }
+    float f[W][V];
+    if (STATIC) {
+#pragma unroll
+        for (int i = 0; i < V; ++i)
+#pragma unroll
+            for (int k = 0; k < W; ++k) f[k][i] = to_f(w[(size_t)(c0 + i) * W + k]);
+    }
+    for (int t = t0; t < t1; ++t) {
+        const size_t bt = row0 + t;
+        Vec<T>::load(x + bt * D + c0, win[0]);
+        if (!STATIC) load_taps<T, T, W>(w, bt, c0, D, G, f);
+        float out[V];
+#pragma unroll
+        for (int i = 0; i < V; ++i) {
+            float acc = win[0][i];
+#pragma unroll
+            for (int k = 0; k < W; ++k) acc = fmaf(f[k][i], win[k][i], acc);
+            out[i] = acc;
+        }
+        Vec<T>::store(y + bt * D + c0, out);
+#pragma unroll
+        for (int k = W - 1; k >= 1; --k)
+#pragma unroll
+            for (int i = 0; i < V; ++i) win[k][i] = win[k - 1][i];
+    }
+}
+
+// ------------------------------------------------------------------ dx (scatter form)
+// Walks t upward through [t0, t1 + W - 1): at token t the products w_t[.,k] * dy_t are
+// added into the open rows t-k; row t-W+1 is complete after token t.  Rows outside
+// [t0, t1) belong to neighbouring chunks and are not stored.
+//   STATIC: taps ws[c,k]; otherwise per-token taps w (type TW, G-tied).
+template <typename T, typename TW, int W, bool STATIC>
+__global__ void __launch_bounds__(128)
+k_conv_bwd_dx(const TW *__restrict__ w, const T *__restrict__ dy, T *__restrict__ dx,
+              int B, int T_, int D, int G, int chunk) {
+    constexpr int V = Vec<T>::N;
+    const int v = blockIdx.x * blockDim.x + threadIdx.x;
+    if (v >= D / V) return;
+    const int nchunks = cdiv(T_, chunk);
+    const int b = blockIdx.y / nchunks;
+    const int t0 = (blockIdx.y % nchunks) * chunk;
+    const int t1 = min(t0 + chunk, T_);
+    const int tend = min(t1 + W - 1, T_);
+    const int c0 = v * V;
+    const size_t row0 = (size_t)b * T_;
+
+    float acc[W][V];   // acc[k] = partial dx of row t-k
+#pragma unroll
+    for (int k = 0; k < W; ++k)
+#pragma unroll
+        for (int i = 0; i < V; ++i) acc[k][i] = 0.f;
+    float f[W][V];
+    if (STATIC) {
+#pragma unroll
+        for (int i = 0; i < V; ++i)
+#pragma unroll
+            for (int k = 0; k < W; ++k) f[k][i] = to_f(w[(size_t)(c0 + i) * W + k]);
+    }
+    for (int t = t0; t < tend; ++t) {
+        const size_t bt = row0 + t;
+        float g[V];
+        Vec<T>::load(dy + bt * D + c0, g);
+        if (!STATIC) load_taps<T, TW, W>(w, bt, c0, D, G, f);
+#pragma unroll
+        for (int i = 0; i < V; ++i) acc[0][i] = (t < t1) ? g[i] : 0.f;   // residual
+#pragma unroll
+        for (int k = 0; k < W; ++k)
+#pragma unroll
+            for (int i = 0; i < V; ++i) acc[k][i] = fmaf(f[k][i], g[i], acc[k][i]);
+        const int done = t - (W - 1);
+        if (done >= t0 && done < t1) Vec<T>::store(dx + (row0 + done) * D + c0, acc[W - 1]);
+#pragma unroll
+        for (int k = W - 1; k >= 1; --k)
+#pragma unroll
+            for (int i = 0; i < V; ++i) acc[k][i] = acc[k - 1][i];
+    }
+    // Sequence end: the still-open rows received all their contributions.
+    // After the shift, acc[k] holds row (tend - k) for k = 1..W-1.
+#pragma unroll
+    for (int k = 1; k < W; ++k) {
+        const int row = tend - k;
+        if (tend == T_ && row >= t0 && row < t1 && row > tend - W)
+            Vec<T>::store(dx + (row0 + row) * D + c0, acc[k]);
+    }
+}
+
+// ------------------------------------------------------------------ static dw partials
+// Thread (vector v, token sub-chunk ty) accumulates dw[c,k] += dy_t[c] x_{t-k}[c] over its
+// tokens; the block sums its sub-chunks in a fixed order and writes one partial row
+// part[p, c, k] (p = blockIdx.y).
+template <typename T, int W>
+__global__ void __launch_bounds__(256)
+k_static_dw_partial(const T *__restrict__ x, const T *__restrict__ dy, float *__restrict__ part,
+                    int B, int T_, int D, int sub) {
+    constexpr int V = Vec<T>::N;
+    constexpr int BX = 32, BY = 8;
+    __shared__ float red[BY][BX][V];
+    const int v = blockIdx.x * BX + threadIdx.x;
+    const int per_block = BY * sub;
+    const int nblk = cdiv(T_, per_block);
+    const int b = blockIdx.y / nblk;
+    const int t0 = (blockIdx.y % nblk) * per_block + threadIdx.y * sub;
+    const int t1 = min(t0 + sub, T_);
+    const int c0 = v * V;
+    const bool active = v < D / V;
+    const size_t row0 = (size_t)b * T_;
+
+    float acc[W][V];
+#pragma unroll
+    for (int k = 0; k < W; ++k)
+#pragma unroll
+        for (int i = 0; i < V; ++i) acc[k][i] = 0.f;
+    if (active && t0 < t1) {
+        float win[W][V];
+#pragma unroll
+        for (int k = 1; k < W; ++k) {
+            const int t = t0 - k;
+            if (t >= 0) {
+                Vec<T>::load(x + (row0 + t) * D + c0, win[k]);
+            } else {
+#pragma unroll
+                for (int i = 0; i < V; ++i) win[k][i] = 0.f;
+            }
+        }
+        for (int t = t0; t < t1; ++t) {
+            const size_t bt = row0 + t;
+            float g[V];
+            Vec<T>::load(x + bt * D + c0, win[0]);
+            Vec<T>::load(dy + bt * D + c0, g);
+#pragma unroll
+            for (int k = 0; k < W; ++k)
+#pragma unroll
+                for (int i = 0; i < V; ++i) acc[k][i] = fmaf(g[i], win[k][i], acc[k][i]);
+#pragma unroll
+            for (int k = W - 1; k >= 1; --k)
+#pragma unroll
+                for (int i = 0; i < V; ++i) win[k][i] = win[k - 1][i];
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < W; ++k) {
+#pragma unroll
+        for (int i = 0; i < V; ++i) red[threadIdx.y][threadIdx.x][i] = acc[k][i];
+        __syncthreads();
+        if (threadIdx.y == 0 && active) {
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                float s = 0.f;
+                for (int y = 0; y < BY; ++y) s += red[y][threadIdx.x][i];
+                part[((size_t)blockIdx.y * D + c0 + i) * W + k] = s;
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// out[e] = sum_{p < P} part[p * n + e], in order of p.
+__global__ void k_sum_partials(const float *__restrict__ part, float *__restrict__ out,
+                               int P, size_t n) {
+    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n;
+         e += (size_t)gridDim.x * blockDim.x) {
+        float s = 0.f;
+        for (int p = 0; p < P; ++p) s += part[(size_t)p * n + e];
+        out[e] = s;
+    }
+}
+
+// ------------------------------------------------------------------ explicit dw
+// dw[bt,g,k] = sum_{c in g, t-k >= 0} dy[bt,c] x[bt-k,c]; one thread per (bt, g).
+template <typename T>
+__global__ void k_dyn_dw(const T *__restrict__ x, const T *__restrict__ dy, float *__restrict__ dw,
+                         int B, int T_, int D, int G, int W) {
+    const int NG = D / G;
+    const size_t n = (size_t)B * T_ * NG;
+    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n;
+         e += (size_t)gridDim.x * blockDim.x) {
+        const size_t bt = e / NG;
+        const int g = (int)(e % NG);
+        const int t = (int)(bt % T_);
+        for (int k = 0; k < W; ++k) {
+            float s = 0.f;
+            if (t - k >= 0) {
+                const T *pg = dy + bt * D + (size_t)g * G;
+                const T *px = x + (bt - k) * D + (size_t)g * G;
+                for (int c = 0; c < G; ++c) s = fmaf(to_f(pg[c]), to_f(px[c]), s);
+            }
+            dw[e * W + k] = s;
+        }
+    }
+}
+
+// ------------------------------------------------------------------ low-rank, CUDA cores
+// Fused forward for general shapes.  Block = TT tokens of one sequence x 64 channels.
+// Phase 1 forms the filter tile wt[t][j] = sum_r z[t,r] U[r, jbase + j] in shared memory
+// (fp32), phase 2 applies the causal convolution with the residual.
+constexpr int kLrTT = 16;
+constexpr int kLrCS = 64;
+constexpr int kLrMaxCols = (kLrCS + 2) * 8;   // groups touched by 64 channels, W <= 8
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+k_lowrank_fwd_simt(const T *__restrict__ x, const T *__restrict__ z, const T *__restrict__ U,
+                   T *__restrict__ y, int B, int T_, int D, int G, int W, int R) {
+    __shared__ float wt[kLrTT][kLrMaxCols];
+    extern __shared__ float zs[];   // [kLrTT][R]
+    const int NG = D / G;
+    const int N = NG * W;
+    const int c0 = blockIdx.x * kLrCS;
+    const int c1 = min(c0 + kLrCS, D);
+    const int ntile = cdiv(T_, kLrTT);
+    const int b = blockIdx.y / ntile;
+    const int t0 = (blockIdx.y % ntile) * kLrTT;
+    const int nt = min(kLrTT, T_ - t0);
+    const int g_lo = c0 / G, g_hi = (c1 - 1) / G;
+    const int ncols = (g_hi - g_lo + 1) * W;
+    const size_t row0 = (size_t)b * T_ + t0;
+
+    for (int e = threadIdx.x; e < kLrTT * R; e += blockDim.x) {
+        const int t = e / R, r = e % R;
+        zs[e] = (t < nt) ? to_f(z[(row0 + t) * R + r]) : 0.f;
+    }
+    __syncthreads();
+    for (int j = threadIdx.x; j < ncols; j += blockDim.x) {
+        float acc[kLrTT];
+#pragma unroll
+        for (int t = 0; t < kLrTT; ++t) acc[t] = 0.f;
+        const int col = g_lo * W + j;
+        if (col < N) {
+            for (int r = 0; r < R; ++r) {
+                const float u = to_f(U[(size_t)r * N + col]);
+#pragma unroll
+                for (int t = 0; t < kLrTT; ++t) acc[t] = fmaf(zs[t * R + r], u, acc[t]);
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < kLrTT; ++t) wt[t][j] = acc[t];
+    }
+    __syncthreads();
+    const int width = c1 - c0;
+    for (int e = threadIdx.x; e < nt * width; e += blockDim.x) {
+        const int t = e / width, c = c0 + e % width;
+        const int gt = t0 + t;
+        const int jb = (c / G - g_lo) * W;
+        const size_t bt = row0 + t;
+        float acc = to_f(x[bt * D + c]);
+        for (int k = 0; k < W && gt - k >= 0; ++k)
+            acc = fmaf(wt[t][jb + k], to_f(x[(bt - k) * D + c]), acc);
+        y[bt * D + c] = from_f<T>(acc);
+    }
+}
+
+// wm[bt, j] = sum_r z[bt, r] U[r, j] in fp32 (materialised filters for the CUDA-core
+// backward).  Block = kLrTT tokens x 256 columns.
+template <typename T>
+__global__ void __launch_bounds__(256)
+k_lowrank_weights(const T *__restrict__ z, const T *__restrict__ U, float *__restrict__ wm,
+                  int BT, int N, int R) {
+    extern __shared__ float zs[];   // [kLrTT][R]
+    const int bt0 = blockIdx.y * kLrTT;
+    const int nt = min(kLrTT, BT - bt0);
+    for (int e = threadIdx.x; e < kLrTT * R; e += blockDim.x) {
+        const int t = e / R, r = e % R;
+        zs[e] = (t < nt) ? to_f(z[(size_t)(bt0 + t) * R + r]) : 0.f;
+    }
+    __syncthreads();
+    const int j = blockIdx.x * blockDim.x + threadIdx.x;
+    if (j >= N) return;
+    float acc[kLrTT];
+#pragma unroll
+    for (int t = 0; t < kLrTT; ++t) acc[t] = 0.f;
+    for (int r = 0; r < R; ++r) {
+        const float u = to_f(U[(size_t)r * N + j]);
+#pragma unroll
+        for (int t = 0; t < kLrTT; ++t) acc[t] = fmaf(zs[t * R + r], u, acc[t]);
+    }
+    for (int t = 0; t < nt; ++t) wm[(size_t)(bt0 + t) * N + j] = acc[t];
+}
+
+// dz[bt, r] = sum_j dw[bt, j] U[r, j]; one warp per token, lanes over j.
+template <typename T>
+__global__ void __launch_bounds__(256)
+k_lowrank_dz(const float *__restrict__ dw, const T *__restrict__ U, float *__restrict__ dz,
+             int BT, int N, int R) {
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (warp >= BT) return;
+    const float *row = dw + (size_t)warp * N;
+    for (int r = 0; r < R; ++r) {
+        const T *u = U + (size_t)r * N;
+        float s = 0.f;
+        for (int j = lane; j < N; j += 32) s = fmaf(row[j], to_f(u[j]), s);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == 0) dz[(size_t)warp * R + r] = s;
+    }
+}
+
+// dU[r, j] = sum_bt z[bt, r] dw[bt, j], summed over bt in order.
+template <typename T>
+__global__ void __launch_bounds__(256)
+k_lowrank_dU(const T *__restrict__ z, const float *__restrict__ dw, float *__restrict__ dU,
+             int BT, int N, int R) {
+    const int j = blockIdx.x * blockDim.x + threadIdx.x;
+    const int r = blockIdx.y;
+    if (j >= N) return;
+    float s = 0.f;
+    for (int bt = 0; bt < BT; ++bt) s = fmaf(to_f(z[(size_t)bt * R + r]), dw[(size_t)bt * N + j], s);
+    dU[(size_t)r * N + j] = s;
+}
+
+// ------------------------------------------------------------------ launchers
+constexpr int kChunk = 32;
+
+template <typename T, bool STATIC>
+static void launch_fwd_T(const void *x, const void *w, void *y, int B, int T_, int D, int G, int W,
+                         cudaStream_t s) {
+    constexpr int V = Vec<T>::N;
+    const dim3 block(128);
+    const dim3 grid(cdiv(D / V, 128), B * cdiv(T_, kChunk));
+    const T *xp = (const T *)x;
+    const T *wp = (const T *)w;
+    T *yp = (T *)y;
+    switch (W) {
+#define DSC_CASE(WW) \
+    case WW: k_conv_fwd<T, WW, STATIC><<<grid, block, 0, s>>>(xp, wp, yp, B, T_, D, G, kChunk); break;
+        DSC_CASE(1) DSC_CASE(2) DSC_CASE(3) DSC_CASE(4) DSC_CASE(5) DSC_CASE(6) DSC_CASE(7) DSC_CASE(8)
+#undef DSC_CASE
+    }
+}
+
+void launch_conv_fwd(const void *x, const void *w, void *y, int B, int T, int D, int G, int W,
+                     bool bf16_, bool is_static, cudaStream_t s) {
+    if (bf16_) {
+        if (is_static) launch_fwd_T<bf16, true>(x, w, y, B, T, D, 1, W, s);
+        else launch_fwd_T<bf16, false>(x, w, y, B, T, D, G, W, s);
+    } else {
+        if (is_static) launch_fwd_T<float, true>(x, w, y, B, T, D, 1, W, s);
+        else launch_fwd_T<float, false>(x, w, y, B, T, D, G, W, s);
+    }
+}
+
+template <typename T, typename TW, bool STATIC>
+static void launch_dx_T(const void *w, const void *dy, void *dx, int B, int T_, int D, int G, int W,
+                        cudaStream_t s) {
+    constexpr int V = Vec<T>::N;
+    const dim3 block(128);
+    const dim3 grid(cdiv(D / V, 128), B * cdiv(T_, kChunk));
+    const TW *wp = (const TW *)w;
+    const T *gp = (const T *)dy;
+    T *op = (T *)dx;
+    switch (W) {
+#define DSC_CASE(WW) \
+    case WW: k_conv_bwd_dx<T, TW, WW, STATIC><<<grid, block, 0, s>>>(wp, gp, op, B, T_, D, G, kChunk); break;
+        DSC_CASE(1) DSC_CASE(2) DSC_CASE(3) DSC_CASE(4) DSC_CASE(5) DSC_CASE(6) DSC_CASE(7) DSC_CASE(8)
+#undef DSC_CASE
+    }
+}
+
+void launch_conv_dx(const void *w, bool w_is_f32, const void *dy, void *dx, int B, int T, int D,
+                    int G, int W, bool bf16_, bool is_static, cudaStream_t s) {
+    if (bf16_) {
+        if (is_static) launch_dx_T<bf16, bf16, true>(w, dy, dx, B, T, D, 1, W, s);
+        else if (w_is_f32) launch_dx_T<bf16, float, false>(w, dy, dx, B, T, D, G, W, s);
+        else launch_dx_T<bf16, bf16, false>(w, dy, dx, B, T, D, G, W, s);
+    } else {
+        if (is_static) launch_dx_T<float, float, true>(w, dy, dx, B, T, D, 1, W, s);
+        else launch_dx_T<float, float, false>(w, dy, dx, B, T, D, G, W, s);
+    }
+}
+
+constexpr int kStaticSub = 32;   // tokens per thread in the static dw partials
+constexpr int kStaticBY = 8;
+
+int static_dw_partials(int B, int T) { return B * cdiv(T, kStaticBY * kStaticSub); }
+
+template <typename T>
+static void launch_static_dw_T(const void *x, const void *dy, float *part, float *dw, int B, int T_,
+                               int D, int W, cudaStream_t s) {
+    constexpr int V = Vec<T>::N;
+    const dim3 block(32, kStaticBY);
+    const int P = static_dw_partials(B, T_);
+    const dim3 grid(cdiv(D / V, 32), P);
+    const T *xp = (const T *)x;
+    const T *gp = (const T *)dy;
+    switch (W) {
+#define DSC_CASE(WW) \
+    case WW: k_static_dw_partial<T, WW><<<grid, block, 0, s>>>(xp, gp, part, B, T_, D, kStaticSub); break;
+        DSC_CASE(1) DSC_CASE(2) DSC_CASE(3) DSC_CASE(4) DSC_CASE(5) DSC_CASE(6) DSC_CASE(7) DSC_CASE(8)
+#undef DSC_CASE
+    }
+    const size_t n = (size_t)D * W;
+    k_sum_partials<<<(unsigned)std::min<size_t>(cdiv((int)std::min<size_t>(n, 1u << 30), 256), 4096), 256, 0, s>>>(
+        part, dw, P, n);
+}
+
+void launch_static_dw(const void *x, const void *dy, float *part, float *dw, int B, int T, int D,
+                      int W, bool bf16_, cudaStream_t s) {
+    if (bf16_) launch_static_dw_T<bf16>(x, dy, part, dw, B, T, D, W, s);
+    else launch_static_dw_T<float>(x, dy, part, dw, B, T, D, W, s);
+}
+
+void launch_dyn_dw(const void *x, const void *dy, float *dw, int B, int T, int D, int G, int W,
+                   bool bf16_, cudaStream_t s) {
+    const size_t n = (size_t)B * T * (D / G);
+    const unsigned grid = (unsigned)std::min<size_t>((n + 255) / 256, 65535u * 8);
+    if (bf16_) k_dyn_dw<bf16><<<grid, 256, 0, s>>>((const bf16 *)x, (const bf16 *)dy, dw, B, T, D, G, W);
+    else k_dyn_dw<float><<<grid, 256, 0, s>>>((const float *)x, (const float *)dy, dw, B, T, D, G, W);
+}
+
+void launch_lowrank_fwd_simt(const void *x, const void *z, const void *U, void *y, int B, int T,
+                             int D, int G, int W, int R, bool bf16_, cudaStream_t s) {
+    const dim3 grid(cdiv(D, kLrCS), B * cdiv(T, kLrTT));
+    const size_t smem = sizeof(float) * kLrTT * R;
+    if (bf16_)
+        k_lowrank_fwd_simt<bf16><<<grid, 256, smem, s>>>((const bf16 *)x, (const bf16 *)z,
+                                                         (const bf16 *)U, (bf16 *)y, B, T, D, G, W, R);
+    else
+        k_lowrank_fwd_simt<float><<<grid, 256, smem, s>>>((const float *)x, (const float *)z,
+                                                          (const float *)U, (float *)y, B, T, D, G, W, R);
+}
+
+size_t lowrank_bwd_simt_workspace(int B, int T, int D, int G, int W) {
+    const size_t n = (size_t)B * T * (D / G) * W;
+    return 2 * n * sizeof(float);
+}
+
+void launch_lowrank_bwd_simt(const void *x, const void *z, const void *U, const void *dy, void *dx,
+                             float *dz, float *dU, void *ws, int B, int T, int D, int G, int W,
+                             int R, bool bf16_, cudaStream_t s) {
+    const int BT = B * T;
+    const int N = (D / G) * W;
+    float *wm = (float *)ws;
+    float *dwm = wm + (size_t)BT * N;
+    const dim3 gw(cdiv(N, 256), cdiv(BT, kLrTT));
+    const size_t smem = sizeof(float) * kLrTT * R;
+    if (bf16_) k_lowrank_weights<bf16><<<gw, 256, smem, s>>>((const bf16 *)z, (const bf16 *)U, wm, BT, N, R);
+    else k_lowrank_weights<float><<<gw, 256, smem, s>>>((const float *)z, (const float *)U, wm, BT, N, R);
+    launch_conv_dx(wm, true, dy, dx, B, T, D, G, W, bf16_, false, s);
+    launch_dyn_dw(x, dy, dwm, B, T, D, G, W, bf16_, s);
+    const unsigned gz = (unsigned)cdiv(BT, 8);
+    const dim3 gU(cdiv(N, 256), R);
+    if (bf16_) {
+        k_lowrank_dz<bf16><<<gz, 256, 0, s>>>(dwm, (const bf16 *)U, dz, BT, N, R);
+        k_lowrank_dU<bf16><<<gU, 256, 0, s>>>((const bf16 *)z, dwm, dU, BT, N, R);
+    } else {
+        k_lowrank_dz<float><<<gz, 256, 0, s>>>(dwm, (const float *)U, dz, BT, N, R);
+        k_lowrank_dU<float><<<gU, 256, 0, s>>>((const float *)z, dwm, dU, BT, N, R);
+    }
+}
+
+}  // namespace dsc

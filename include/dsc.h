@@ -1,0 +1,151 @@
+/*
+ * dsc.h -- C ABI of libdsc.so: the causal dynamic short convolution on NVIDIA B200
+ * (sm_100a).
+ *
+ * The operation ("Convolucoes Curtas Dinamicas Melhoram Transformers",
+ * gist.science/pt/paper/2606.03825, section "Metodologia > Convolucoes Curtas
+ * Dinamicas"):
+ *
+ *   Mecanismo:       y_t = sum_{k=0}^{W-1} w(t)_k (.) x_{t-k}     (elementwise per channel)
+ *   Posicionamento:  applied with a residual, X = X + dynamicShortConv(X)
+ *   Parametrizacao:  w(t) is produced by a learned linear map of the hidden state;
+ *                    (1) low-rank factorisation of rank R: w(t) = z_t U, whose second
+ *                        factor the fused kernel applies on chip ("Implementacao de
+ *                        Treinamento Eficiente", fused low-rank kernel), and
+ *                    (2) head-wise tying: one filter is shared by G consecutive channels.
+ *
+ * Every entry point computes, for each sequence b, token t and channel c,
+ *
+ *   y[b,t,c] = x[b,t,c] + sum_{k=0}^{W-1} f(b,t,c,k) * x[b,t-k,c],   x[b,t',c] = 0 for t' < 0,
+ *
+ * where the tap k = 0 multiplies the current token, g(c) = floor(c / G) is the
+ * filter group of channel c, and f is
+ *   dsc_fwd:          w[b,t,g(c),k]                        (explicit dynamic filters)
+ *   dsc_fwd_lowrank:  sum_r z[b,t,r] U[r, g(c)*W + k]      (filters formed on chip)
+ *   dsc_static_fwd:   w[c,k]                               (static depthwise filters)
+ * Sequences are independent: nothing crosses from one b to another.
+ *
+ * Conventions shared by all entry points
+ *   - Layouts are dense and row-major, last index fastest:
+ *       x, y, dy, dx [B,T,D];  w, dw [B,T,D/G,W];  z, dz [B,T,R];
+ *       U, dU [R,(D/G)*W] with column j = g*W + k;  static w, dw [D,W].
+ *   - Pointers are device memory owned by the caller; the library allocates
+ *     nothing and keeps no pointer after the call returns.  Inputs are read-only.
+ *     Outputs must not overlap inputs.
+ *   - x, w, z, U, y, dy and dx share the element type `dt`; dz, dU and the weight
+ *     gradients dw are always fp32.  Arithmetic is fp32 (fp32 accumulation); bf16
+ *     outputs are rounded once, to nearest even.
+ *   - Calls are asynchronous on `stream` (NULL = the legacy default stream) and
+ *     enqueue work on the current CUDA device.
+ *   - Requirements: B, T, D, G, W >= 1, D % G == 0, 1 <= W <= 8, 1 <= R <= 256;
+ *     D a multiple of 8 (bf16) or 4 (fp32); every pointer 16-byte aligned;
+ *     B*T < 2^31.
+ *   - Errors are reported by the return value; no exception crosses the ABI and
+ *     nothing is launched when validation fails:
+ *       DSC_ERR_INVALID_ARG  null pointer, non-positive size, D % G != 0;
+ *       DSC_ERR_UNSUPPORTED  W or R out of range, D not a multiple of the vector
+ *                            width, misaligned pointer, workspace too small;
+ *       DSC_ERR_CUDA         a CUDA launch error (read from cudaGetLastError).
+ *     dsc_last_error() returns a human-readable detail for the calling thread.
+ *   - Results are deterministic: repeated calls on the same inputs produce
+ *     bitwise-identical outputs (reductions run in a fixed order, no float atomics).
+ */
+#ifndef DSC_H
+#define DSC_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define DSC_API __attribute__((visibility("default")))
+#else
+#define DSC_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DSC_OK = 0,
+    DSC_ERR_INVALID_ARG = 1,
+    DSC_ERR_UNSUPPORTED = 2,
+    DSC_ERR_CUDA = 3
+} dsc_status_t;
+
+typedef enum { DSC_F32 = 0, DSC_BF16 = 1 } dsc_dtype_t;
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *dsc_stream_t;
+
+/* Forward with explicit dynamic filters (Mecanismo + Posicionamento, head-wise
+ * tying by G).  x, y [B,T,D]; w [B,T,D/G,W], element (b,t,g,k) multiplies
+ * x[b,t-k,c] for every channel c of group g. */
+DSC_API dsc_status_t dsc_fwd(const void *x, const void *w, void *y,
+                     int B, int T, int D, int G, int W,
+                     dsc_dtype_t dt, dsc_stream_t stream);
+
+/* Fused low-rank forward ("Implementacao de Treinamento Eficiente", fused low-rank
+ * kernel): the filters w(t) = z_t U are formed on chip, tile by tile, and never
+ * written to memory.  x, y [B,T,D]; z [B,T,R]; U [R,(D/G)*W]. */
+DSC_API dsc_status_t dsc_fwd_lowrank(const void *x, const void *z, const void *U, void *y,
+                             int B, int T, int D, int G, int W, int R,
+                             dsc_dtype_t dt, dsc_stream_t stream);
+
+/* Bytes of device workspace dsc_bwd_lowrank needs for these sizes (0 if none). */
+DSC_API size_t dsc_bwd_lowrank_workspace_bytes(int B, int T, int D, int G, int W, int R,
+                                       dsc_dtype_t dt);
+
+/* Backward of dsc_fwd_lowrank (chain rule through Mecanismo and Parametrizacao 1):
+ *   dx[b,s,c] = dy[b,s,c] + sum_{k, s+k<T} w[b,s+k,g(c),k] dy[b,s+k,c]
+ *   dw[b,t,g,k] = sum_{c in g, t-k>=0} dy[b,t,c] x[b,t-k,c]      (on chip only)
+ *   dz[b,t,r] = sum_j dw[b,t,j] U[r,j]
+ *   dU[r,j]   = sum_{b,t} z[b,t,r] dw[b,t,j]                    (over all B*T tokens)
+ * dx [B,T,D] has type dt; dz [B,T,R] and dU [R,(D/G)*W] are fp32 and are
+ * overwritten, not accumulated.  `workspace` is caller-owned device scratch of at
+ * least dsc_bwd_lowrank_workspace_bytes() bytes (may be NULL when that is 0); its
+ * contents on entry do not matter. */
+DSC_API dsc_status_t dsc_bwd_lowrank(const void *x, const void *z, const void *U, const void *dy,
+                             void *dx, float *dz, float *dU,
+                             void *workspace, size_t workspace_bytes,
+                             int B, int T, int D, int G, int W, int R,
+                             dsc_dtype_t dt, dsc_stream_t stream);
+
+/* Backward of dsc_fwd (explicit filters): dx [B,T,D] of type dt and the per-token
+ * filter gradient dw [B,T,D/G,W] in fp32 (overwritten). */
+DSC_API dsc_status_t dsc_bwd(const void *x, const void *w, const void *dy,
+                     void *dx, float *dw,
+                     int B, int T, int D, int G, int W,
+                     dsc_dtype_t dt, dsc_stream_t stream);
+
+/* Static depthwise causal convolution, the primitive the method generalises
+ * ("Declaracao do Problema"): y = x + conv(x; w), w [D,W] fixed over t. */
+DSC_API dsc_status_t dsc_static_fwd(const void *x, const void *w, void *y,
+                            int B, int T, int D, int W,
+                            dsc_dtype_t dt, dsc_stream_t stream);
+
+/* Bytes of device workspace dsc_static_bwd needs for these sizes. */
+DSC_API size_t dsc_static_bwd_workspace_bytes(int B, int T, int D, int W, dsc_dtype_t dt);
+
+/* Backward of dsc_static_fwd: dx [B,T,D] of type dt, and dw [D,W] fp32 summed over
+ * all B*T tokens in a fixed order (overwritten). */
+DSC_API dsc_status_t dsc_static_bwd(const void *x, const void *w, const void *dy,
+                            void *dx, float *dw,
+                            void *workspace, size_t workspace_bytes,
+                            int B, int T, int D, int W,
+                            dsc_dtype_t dt, dsc_stream_t stream);
+
+/* Which implementation dsc_fwd_lowrank / dsc_bwd_lowrank use for these sizes:
+ * 1 = tensor-core (tcgen05) kernels, 0 = CUDA-core kernels, -1 = invalid sizes. */
+DSC_API int dsc_lowrank_path(int B, int T, int D, int G, int W, int R, dsc_dtype_t dt);
+
+/* Static description of a status code. */
+DSC_API const char *dsc_status_string(dsc_status_t status);
+
+/* Detail of the last failed call on this host thread ("" if none). */
+DSC_API const char *dsc_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSC_H */

@@ -1,0 +1,279 @@
+"""GPU parity: every entry point of libdsc.so against the CPU oracle, element by
+element, on seeded inputs (sizes that span several tiles, ragged tails, edge cases),
+plus sampled outputs at the full workload sizes.
+
+All calls go through the C ABI (the binding only marshals arguments)."""
+import numpy as np
+import pytest
+import torch
+
+import dsc_inputs as di
+import oracle
+from parity import assert_close, f64, future, window
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dsc():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import dynamic_short_convolutions_causal_b200 as m
+    return m
+
+
+DEV = "cuda"
+
+
+def _guarded(shape, dtype, fill=float("nan"), guard=256):
+    """An output tensor inside a larger buffer whose guard bands hold a canary."""
+    n = int(np.prod(shape))
+    buf = torch.full((n + 2 * guard,), fill, dtype=dtype, device=DEV)
+    buf[:guard] = 4096.0
+    buf[-guard:] = 4096.0
+    return buf, buf[guard:guard + n].view(*shape)
+
+
+def _check_guard(buf, guard=256):
+    assert torch.all(buf[:guard] == 4096.0) and torch.all(buf[-guard:] == 4096.0), \
+        "a kernel wrote outside its output"
+
+
+def _gen(wl, parts):
+    return {k: v.to(DEV) for k, v in di.make(wl, "cpu", parts).items()}
+
+
+# ------------------------------------------------------------------ explicit filters
+EXPLICIT = [
+    # B, T, D, G, W, dtype
+    (1, 64, 64, 8, 4, "f32"),          # the small fp32 workload's shape
+    (2, 300, 192, 1, 4, "bf16"),
+    (3, 77, 256, 64, 3, "bf16"),
+    (1, 5, 64, 8, 8, "bf16"),
+    (2, 1, 16, 2, 1, "bf16"),
+    (2, 45, 24, 3, 5, "bf16"),
+    (2, 33, 96, 96, 2, "f32"),
+    (1, 130, 40, 5, 7, "f32"),
+]
+
+
+@pytest.mark.parametrize("B,T,D,G,W,dt", EXPLICIT)
+def test_explicit_fwd_bwd(dsc, B, T, D, G, W, dt):
+    wl = di.small(B, T, D, G, W, 0, dt, seed=B * 1000 + T)
+    t = _gen(wl, ("x", "w", "dy"))
+    buf, y = _guarded((B, T, D), t["x"].dtype)
+    dsc.dsc_fwd(t["x"], t["w"], y, G)
+    torch.cuda.synchronize()
+    _check_guard(buf)
+    assert_close(y, oracle.fwd(f64(t["x"]), f64(t["w"]), G), dt, "y")
+    bdx, dx = _guarded((B, T, D), t["x"].dtype)
+    bdw, dw = _guarded((B, T, D // G, W), torch.float32)
+    dsc.dsc_bwd(t["x"], t["w"], t["dy"], dx, dw, G)
+    torch.cuda.synchronize()
+    _check_guard(bdx)
+    _check_guard(bdw)
+    rdx, rdw = oracle.bwd(f64(t["x"]), f64(t["w"]), f64(t["dy"]), G)
+    assert_close(dx, rdx, dt, "dx")
+    assert_close(dw, rdw, dt, "dw", reduction=True)
+
+
+def test_small_fp32_workload_exact_bound(dsc):
+    """The fp32 explicit workload (seed 0) at its full size: max|err| <= 1e-5."""
+    wl = di.WORKLOADS["explicit_fp32_small"]
+    t = _gen(wl, ("x", "w"))
+    y = torch.empty_like(t["x"])
+    dsc.dsc_fwd(t["x"], t["w"], y, wl.G)
+    ref = oracle.fwd(f64(t["x"]), f64(t["w"]), wl.G)
+    assert np.max(np.abs(f64(y) - ref)) <= 1e-5
+
+
+# ------------------------------------------------------------------ static filters
+STATIC = [
+    (2, 300, 192, 4, "bf16"), (1, 1000, 64, 8, "bf16"), (2, 3, 16, 5, "bf16"),
+    (3, 70, 32, 1, "f32"), (2, 257, 128, 3, "f32"),
+]
+
+
+@pytest.mark.parametrize("B,T,D,W,dt", STATIC)
+def test_static_fwd_bwd(dsc, B, T, D, W, dt):
+    wl = di.small(B, T, D, 1, W, 0, dt, seed=7 + T)
+    t = _gen(wl, ("x", "dy", "ws"))
+    buf, y = _guarded((B, T, D), t["x"].dtype)
+    dsc.dsc_static_fwd(t["x"], t["ws"], y)
+    torch.cuda.synchronize()
+    _check_guard(buf)
+    assert_close(y, oracle.static_fwd(f64(t["x"]), f64(t["ws"])), dt, "y")
+    dx = torch.full_like(t["x"], float("nan"))
+    dw = torch.full((D, W), float("nan"), dtype=torch.float32, device=DEV)
+    ws = dsc.workspace(dsc.dsc_static_bwd_workspace_bytes(B, T, D, W, t["x"].dtype), DEV)
+    dsc.dsc_static_bwd(t["x"], t["ws"], t["dy"], dx, dw, ws)
+    rdx, rdw = oracle.static_bwd(f64(t["x"]), f64(t["ws"]), f64(t["dy"]))
+    assert_close(dx, rdx, dt, "dx")
+    assert_close(dw, rdw, dt, "dw", reduction=True)
+
+
+# ------------------------------------------------------------------ low-rank
+LOWRANK = [
+    # B, T, D, G, W, R, dtype
+    (2, 300, 192, 1, 4, 32, "bf16"),
+    (2, 257, 256, 4, 8, 64, "bf16"),
+    (1, 130, 128, 2, 3, 16, "bf16"),
+    (3, 50, 64, 64, 2, 16, "bf16"),
+    (2, 200, 128, 1, 4, 1, "bf16"),
+    (1, 9, 64, 1, 5, 3, "bf16"),
+    (2, 3, 64, 1, 4, 32, "bf16"),
+    (1, 1, 64, 2, 6, 32, "bf16"),
+    (2, 140, 320, 8, 7, 48, "bf16"),
+    (2, 70, 64, 1, 4, 32, "f32"),
+    (1, 100, 48, 3, 3, 8, "f32"),
+]
+
+
+@pytest.mark.parametrize("B,T,D,G,W,R,dt", LOWRANK)
+def test_lowrank_fwd_bwd(dsc, B, T, D, G, W, R, dt):
+    wl = di.small(B, T, D, G, W, R, dt, seed=R * 100 + T)
+    t = _gen(wl, ("x", "z", "U", "dy"))
+    x, z, U, dy = t["x"], t["z"], t["U"], t["dy"]
+    buf, y = _guarded((B, T, D), x.dtype)
+    dsc.dsc_fwd_lowrank(x, z, U, y, G, W)
+    torch.cuda.synchronize()
+    _check_guard(buf)
+    assert_close(y, oracle.fwd_lowrank(f64(x), f64(z), f64(U), G, W), dt, "y")
+
+    ws = dsc.workspace(dsc.dsc_bwd_lowrank_workspace_bytes(B, T, D, G, W, R, x.dtype), DEV)
+    bdx, dx = _guarded((B, T, D), x.dtype)
+    bdz, dz = _guarded((B, T, R), torch.float32)
+    bdU, dU = _guarded((R, (D // G) * W), torch.float32)
+    dsc.dsc_bwd_lowrank(x, z, U, dy, dx, dz, dU, ws, G, W)
+    torch.cuda.synchronize()
+    for b in (bdx, bdz, bdU):
+        _check_guard(b)
+    rdx, rdz, rdU = oracle.bwd_lowrank(f64(x), f64(z), f64(U), f64(dy), G, W)
+    assert_close(dx, rdx, dt, "dx")
+    assert_close(dz, rdz, dt, "dz", reduction=True)
+    assert_close(dU, rdU, dt, "dU", reduction=True)
+
+
+def test_lowrank_deterministic(dsc):
+    B, T, D, G, W, R = 2, 300, 192, 1, 4, 32
+    t = _gen(di.small(B, T, D, G, W, R, "bf16", seed=3), ("x", "z", "U", "dy"))
+    ws = dsc.workspace(dsc.dsc_bwd_lowrank_workspace_bytes(B, T, D, G, W, R), DEV)
+    outs = []
+    for _ in range(2):
+        y = torch.empty_like(t["x"])
+        dx = torch.empty_like(t["x"])
+        dz = torch.empty((B, T, R), dtype=torch.float32, device=DEV)
+        dU = torch.empty((R, D * W), dtype=torch.float32, device=DEV)
+        dsc.dsc_fwd_lowrank(t["x"], t["z"], t["U"], y, G, W)
+        dsc.dsc_bwd_lowrank(t["x"], t["z"], t["U"], t["dy"], dx, dz, dU, ws, G, W)
+        outs.append((y, dx, dz, dU))
+    for a, b in zip(*outs):
+        assert torch.equal(a, b), "repeated call differs bitwise"
+
+
+def test_failed_call_launches_nothing(dsc):
+    x = torch.randn(2, 8, 64, device=DEV, dtype=torch.bfloat16)
+    w = torch.randn(2, 8, 64, 9, device=DEV, dtype=torch.bfloat16)   # W = 9: unsupported
+    y = torch.full_like(x, float("nan"))
+    with pytest.raises(dsc.DscError):
+        dsc.dsc_fwd(x, w, y, 1)
+    torch.cuda.synchronize()
+    assert torch.isnan(y).all()
+
+
+# ------------------------------------------------------------------ full sizes, sampled
+def _sample_rows(B, T, n, seed):
+    r = np.random.default_rng(seed)
+    rows = {(0, 0), (B - 1, T - 1), (0, 1), (B - 1, 2)}
+    while len(rows) < n:
+        rows.add((int(r.integers(B)), int(r.integers(T))))
+    return sorted(rows)
+
+
+def _full(wl, parts):
+    return di.make(wl, DEV, parts)
+
+
+@pytest.mark.parametrize("name", ["tied_qkv"])
+def test_full_size_explicit_fwd_sampled(dsc, name):
+    wl = di.WORKLOADS[name]
+    t = _full(wl, ("x", "w"))
+    y = torch.empty_like(t["x"])
+    dsc.dsc_fwd(t["x"], t["w"], y, wl.G)
+    for (b, tt) in _sample_rows(wl.B, wl.T, 24, 1):
+        t0, t1 = window(wl.T, tt, wl.W)
+        ref = oracle.fwd(f64(t["x"][b:b + 1, t0:t1]), f64(t["w"][b:b + 1, t0:t1]), wl.G)[0, -1]
+        assert_close(y[b, tt], ref, wl.dtype, "y[%d,%d]" % (b, tt))
+    del t, y
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.parametrize("name", ["lowrank_qkv", "lowrank_mlp"])
+def test_full_size_lowrank_sampled(dsc, name):
+    wl = di.WORKLOADS[name]
+    G, W, R = wl.G, wl.W, wl.R
+    t = _full(wl, ("x", "z", "U", "dy"))
+    x, z, U, dy = t["x"], t["z"], t["U"], t["dy"]
+    y = torch.empty_like(x)
+    dsc.dsc_fwd_lowrank(x, z, U, y, G, W)
+    ws = dsc.workspace(dsc.dsc_bwd_lowrank_workspace_bytes(wl.B, wl.T, wl.D, G, W, R), DEV)
+    dx = torch.empty_like(x)
+    dz = torch.empty((wl.B, wl.T, R), dtype=torch.float32, device=DEV)
+    dU = torch.empty((R, wl.N), dtype=torch.float32, device=DEV)
+    dsc.dsc_bwd_lowrank(x, z, U, dy, dx, dz, dU, ws, G, W)
+    torch.cuda.synchronize()
+    del ws
+    Uh = f64(U)
+    for (b, tt) in _sample_rows(wl.B, wl.T, 12, 2):
+        t0, t1 = window(wl.T, tt, W)
+        ry = oracle.fwd_lowrank(f64(x[b:b + 1, t0:t1]), f64(z[b:b + 1, t0:t1]), Uh, G, W)[0, -1]
+        assert_close(y[b, tt], ry, wl.dtype, "y[%d,%d]" % (b, tt))
+        _, rdz, _ = oracle.bwd_lowrank(f64(x[b:b + 1, t0:t1]), f64(z[b:b + 1, t0:t1]), Uh,
+                                       f64(dy[b:b + 1, t0:t1]), G, W)
+        assert_close(dz[b, tt], rdz[0, -1], wl.dtype, "dz[%d,%d]" % (b, tt), reduction=True)
+        s0, s1 = future(wl.T, tt, W)
+        rdx, _, _ = oracle.bwd_lowrank(f64(x[b:b + 1, s0:s1]), f64(z[b:b + 1, s0:s1]), Uh,
+                                       f64(dy[b:b + 1, s0:s1]), G, W)
+        assert_close(dx[b, tt], rdx[0, 0], wl.dtype, "dx[%d,%d]" % (b, tt))
+    # dU columns of a few filter groups: the sub-problem restricted to that group's
+    # channels (every token) gives those columns exactly.
+    r = np.random.default_rng(3)
+    zh = f64(z)
+    for g in sorted(set([0, wl.NG - 1] + [int(v) for v in r.integers(wl.NG, size=2)])):
+        c0, c1 = g * G, (g + 1) * G
+        _, _, rdU = oracle.bwd_lowrank(f64(x[:, :, c0:c1]), zh, Uh[:, g * W:(g + 1) * W],
+                                       f64(dy[:, :, c0:c1]), G, W)
+        assert_close(dU[:, g * W:(g + 1) * W], rdU, wl.dtype, "dU group %d" % g, reduction=True)
+    # invariant at full size: sum(dU * U) == sum(dz * z)
+    pu = dU.double() * U.double()
+    pz = dz.double() * z.double()
+    a, bsum = float(pu.sum()), float(pz.sum())
+    scale = float(pu.abs().sum()) + float(pz.abs().sum())
+    assert abs(a - bsum) <= 1e-3 * scale, (a, bsum, scale)
+    del t, x, z, U, dy, y, dx, dz, dU
+    torch.cuda.empty_cache()
+
+
+def test_full_size_static_sampled(dsc):
+    wl = di.WORKLOADS["lowrank_mlp"]
+    t = _full(wl, ("x", "dy", "ws"))
+    x, dy, w = t["x"], t["dy"], t["ws"]
+    y = torch.empty_like(x)
+    dsc.dsc_static_fwd(x, w, y)
+    dx = torch.empty_like(x)
+    dw = torch.empty((wl.D, wl.W), dtype=torch.float32, device=DEV)
+    ws = dsc.workspace(dsc.dsc_static_bwd_workspace_bytes(wl.B, wl.T, wl.D, wl.W), DEV)
+    dsc.dsc_static_bwd(x, w, dy, dx, dw, ws)
+    torch.cuda.synchronize()
+    wh = f64(w)
+    for (b, tt) in _sample_rows(wl.B, wl.T, 12, 4):
+        t0, t1 = window(wl.T, tt, wl.W)
+        assert_close(y[b, tt], oracle.static_fwd(f64(x[b:b + 1, t0:t1]), wh)[0, -1], wl.dtype, "y")
+        s0, s1 = future(wl.T, tt, wl.W)
+        rdx, _ = oracle.static_bwd(f64(x[b:b + 1, s0:s1]), wh, f64(dy[b:b + 1, s0:s1]))
+        assert_close(dx[b, tt], rdx[0, 0], wl.dtype, "dx")
+    for c0 in (0, 4096, wl.D - 8):
+        _, rdw = oracle.static_bwd(f64(x[:, :, c0:c0 + 8]), wh[c0:c0 + 8], f64(dy[:, :, c0:c0 + 8]))
+        assert_close(dw[c0:c0 + 8], rdw, wl.dtype, "dw[%d:]" % c0, reduction=True)
+    del t, x, dy, y, dx, dw, ws
+    torch.cuda.empty_cache()
