@@ -4,7 +4,7 @@ Argument marshalling only: every function here derives the sizes from torch tens
 shapes, checks devices and dtypes, and calls the C entry point of the same name on the
 current CUDA stream.  All arithmetic runs in the library's CUDA kernels; there is no
 CPU or PyTorch fallback.  Importing this module fails loudly when libdsc.so is
-missing (build it with ``python -m dynamic_short_convolutions_causal_b200.build``).
+missing (build it with ``python dynamic_short_convolutions_causal_b200/build.py``).
 
 Operation ("Convolucoes Curtas Dinamicas Melhoram Transformers", Metodologia >
 Convolucoes Curtas Dinamicas): y_t = x_t + sum_{k<W} w(t)_k * x_{t-k}, with explicit,
@@ -20,7 +20,8 @@ import torch
 __all__ = [
     "DscError", "lib", "lib_path", "dsc_fwd", "dsc_fwd_lowrank", "dsc_bwd_lowrank",
     "dsc_bwd_lowrank_workspace_bytes", "dsc_bwd", "dsc_static_fwd", "dsc_static_bwd",
-    "dsc_static_bwd_workspace_bytes", "dsc_lowrank_path", "DSC_F32", "DSC_BF16",
+    "dsc_static_bwd_workspace_bytes", "dsc_static_bwd_noalloc", "dsc_lowrank_path",
+    "DSC_F32", "DSC_BF16",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -40,7 +41,7 @@ def _load():
     if not os.path.exists(lib_path):
         raise ImportError(
             "libdsc.so not found at %s: build it with "
-            "`python -m dynamic_short_convolutions_causal_b200.build`" % lib_path)
+            "`python dynamic_short_convolutions_causal_b200/build.py`" % lib_path)
     L = ctypes.CDLL(lib_path)
     vp, i, sz, fp = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p
     sigs = {
@@ -52,6 +53,8 @@ def _load():
         "dsc_static_fwd": (i, [vp, vp, vp, i, i, i, i, i, vp]),
         "dsc_static_bwd_workspace_bytes": (sz, [i, i, i, i, i]),
         "dsc_static_bwd": (i, [vp, vp, vp, vp, fp, vp, sz, i, i, i, i, i, vp]),
+        "dsc_static_bwd_noalloc": (i, [vp, vp, vp, vp, fp, i, i, i, i, i, vp]),
+        "dsc_static_bwd_noalloc_max_scratch_bytes": (sz, []),
         "dsc_lowrank_path": (i, [i, i, i, i, i, i, i]),
         "dsc_status_string": (ctypes.c_char_p, [i]),
         "dsc_last_error": (ctypes.c_char_p, []),
@@ -179,6 +182,18 @@ def dsc_static_bwd(x, w, dy, dx, dw, workspace):
     with torch.cuda.device(x.device):
         _check(lib.dsc_static_bwd(_ptr(x), _ptr(w), _ptr(dy), _ptr(dx), _ptr(dw), _ptr(workspace),
                                   ws_bytes, B, T, D, W, _dt(x), _stream(x)))
+    return dx, dw
+
+
+def dsc_static_bwd_noalloc(x, w, dy, dx, dw):
+    """dsc_static_bwd with the library's fixed scratch array instead of a workspace
+    (for callers that cannot allocate device memory; see include/dsc.h)."""
+    B, T, D = x.shape
+    W = w.shape[-1]
+    _same(x, w, dy, dx, dw)
+    with torch.cuda.device(x.device):
+        _check(lib.dsc_static_bwd_noalloc(_ptr(x), _ptr(w), _ptr(dy), _ptr(dx), _ptr(dw), B, T, D,
+                                          W, _dt(x), _stream(x)))
     return dx, dw
 
 

@@ -1,6 +1,8 @@
 """Build libdsc.so in-tree with nvcc for sm_100a (B200).
 
-    python -m dynamic_short_convolutions_causal_b200.build [--force] [--verbose]
+    python dynamic_short_convolutions_causal_b200/build.py [--force] [--verbose]
+
+(run as a script: importing the package itself needs the built library)
 
 Each .cu under csrc/ is compiled to an object in csrc/_build/ (rebuilt when it or any
 header is newer), then linked into libdsc.so next to this file.

@@ -78,6 +78,10 @@ size_t lowrank_ws(const Dims &d, bool bf16) {
 
 }  // namespace
 
+namespace dsc {
+void set_last_error(const char *msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+}  // namespace dsc
+
 extern "C" {
 
 DSC_API dsc_status_t dsc_fwd(const void *x, const void *w, void *y, int B, int T, int D, int G, int W,

@@ -7,6 +7,9 @@
 
 namespace dsc {
 
+// Records the detail string that dsc_last_error() returns on this host thread.
+void set_last_error(const char *msg);
+
 // CUDA-core kernels (simt.cu)
 void launch_conv_fwd(const void *x, const void *w, void *y, int B, int T, int D, int G, int W,
                      bool bf16, bool is_static, cudaStream_t s);

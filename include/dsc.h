@@ -134,6 +134,30 @@ DSC_API dsc_status_t dsc_static_bwd(const void *x, const void *w, const void *dy
                             int B, int T, int D, int W,
                             dsc_dtype_t dt, dsc_stream_t stream);
 
+/* dsc_static_bwd without a caller-provided workspace.  The paper has no counterpart:
+ * this entry point exists for callers that cannot allocate device memory, such as a
+ * plug-in that a host framework hands only its input and output buffers, or a
+ * latency-critical loop that must not call cudaMalloc (which can synchronise the
+ * device).  It computes exactly what dsc_static_bwd computes, with the same arguments
+ * minus the workspace, and allocates nothing.
+ *   - Scratch comes from one fixed array of dsc_static_bwd_noalloc_max_scratch_bytes()
+ *     (16 MiB) compiled into the library; every GPU that loads the library holds it
+ *     until the process exits.  Sizes whose dsc_static_bwd_workspace_bytes() exceed it
+ *     are rejected with DSC_ERR_UNSUPPORTED and a message naming both sizes.
+ *   - The first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call before
+ *     any stream capture.
+ *   - All calls on a device share the array, which keeps the last call's contents.
+ *     Calls that can overlap on the GPU (other streams, other host threads) race on
+ *     it; the caller must order them.  No part of it needs to start at zero. */
+DSC_API dsc_status_t dsc_static_bwd_noalloc(const void *x, const void *w, const void *dy,
+                                            void *dx, float *dw,
+                                            int B, int T, int D, int W,
+                                            dsc_dtype_t dt, dsc_stream_t stream);
+
+/* Size in bytes of the fixed scratch array dsc_static_bwd_noalloc uses. */
+DSC_API size_t dsc_static_bwd_noalloc_max_scratch_bytes(void);
+
 /* Which implementation dsc_fwd_lowrank / dsc_bwd_lowrank use for these sizes:
  * 1 = tensor-core (tcgen05) kernels, 0 = CUDA-core kernels, -1 = invalid sizes. */
 DSC_API int dsc_lowrank_path(int B, int T, int D, int G, int W, int R, dsc_dtype_t dt);
