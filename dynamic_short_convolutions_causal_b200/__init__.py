@@ -56,6 +56,7 @@ def _load():
         "dsc_static_bwd_noalloc": (i, [vp, vp, vp, vp, fp, i, i, i, i, i, vp]),
         "dsc_static_bwd_noalloc_max_scratch_bytes": (sz, []),
         "dsc_lowrank_path": (i, [i, i, i, i, i, i, i]),
+        "dsc_device_fault": (ctypes.c_uint, [i]),
         "dsc_status_string": (ctypes.c_char_p, [i]),
         "dsc_last_error": (ctypes.c_char_p, []),
     }
@@ -197,8 +198,13 @@ def dsc_static_bwd_noalloc(x, w, dy, dx, dw):
     return dx, dw
 
 
+def dsc_device_fault(reset: bool = False) -> int:
+    """Fault word of the current device (nonzero: a kernel gave up on a wait)."""
+    return int(lib.dsc_device_fault(1 if reset else 0))
+
+
 def dsc_lowrank_path(B, T, D, G, W, R, dtype=torch.bfloat16) -> int:
-    """1: tensor-core kernels, 0: CUDA-core kernels, -1: invalid sizes."""
+    """Bit 0: forward on tensor cores, bit 1: backward on tensor cores; -1: invalid."""
     dt = DSC_BF16 if dtype == torch.bfloat16 else DSC_F32
     return int(lib.dsc_lowrank_path(B, T, D, G, W, R, dt))
 

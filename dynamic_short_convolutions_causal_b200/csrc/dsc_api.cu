@@ -71,7 +71,7 @@ dsc_status_t check_ptrs(const char *fn, const void *const *ptrs, const char *con
 }
 
 size_t lowrank_ws(const Dims &d, bool bf16) {
-    if (dsc::tc_lowrank_supported(d.B, d.T, d.D, d.G, d.W, d.R, bf16))
+    if (dsc::tc_lowrank_bwd_supported(d.B, d.T, d.D, d.G, d.W, d.R, bf16))
         return dsc::tc_lowrank_bwd_workspace(d.B, d.T, d.D, d.G, d.W, d.R);
     return dsc::lowrank_bwd_simt_workspace(d.B, d.T, d.D, d.G, d.W);
 }
@@ -105,7 +105,7 @@ DSC_API dsc_status_t dsc_fwd_lowrank(const void *x, const void *z, const void *U
     const char *n[] = {"x", "z", "U", "y"};
     if ((st = check_ptrs(fn, p, n, 4)) != DSC_OK) return st;
     const bool bf16 = dt == DSC_BF16;
-    if (dsc::tc_lowrank_supported(B, T, D, G, W, R, bf16))
+    if (dsc::tc_lowrank_fwd_supported(B, T, D, G, W, R, bf16))
         return check_launch(fn, dsc::launch_tc_lowrank_fwd(x, z, U, y, B, T, D, G, W, R, (cudaStream_t)stream));
     dsc::launch_lowrank_fwd_simt(x, z, U, y, B, T, D, G, W, R, bf16, (cudaStream_t)stream);
     return check_launch(fn);
@@ -137,7 +137,7 @@ DSC_API dsc_status_t dsc_bwd_lowrank(const void *x, const void *z, const void *U
         const char *wn[] = {"workspace"};
         if ((st = check_ptrs(fn, wp, wn, 1)) != DSC_OK) return st;
     }
-    if (dsc::tc_lowrank_supported(B, T, D, G, W, R, bf16))
+    if (dsc::tc_lowrank_bwd_supported(B, T, D, G, W, R, bf16))
         return check_launch(fn, dsc::launch_tc_lowrank_bwd(x, z, U, dy, dx, dz, dU, workspace, B, T, D,
                                                            G, W, R, (cudaStream_t)stream));
     dsc::launch_lowrank_bwd_simt(x, z, U, dy, dx, dz, dU, workspace, B, T, D, G, W, R, bf16,
@@ -197,8 +197,12 @@ DSC_API dsc_status_t dsc_static_bwd(const void *x, const void *w, const void *dy
 
 DSC_API int dsc_lowrank_path(int B, int T, int D, int G, int W, int R, dsc_dtype_t dt) {
     if (check_dims("dsc_lowrank_path", Dims{B, T, D, G, W, R}, dt) != DSC_OK) return -1;
-    return dsc::tc_lowrank_supported(B, T, D, G, W, R, dt == DSC_BF16) ? 1 : 0;
+    const bool bf16 = dt == DSC_BF16;
+    return (dsc::tc_lowrank_fwd_supported(B, T, D, G, W, R, bf16) ? 1 : 0) |
+           (dsc::tc_lowrank_bwd_supported(B, T, D, G, W, R, bf16) ? 2 : 0);
 }
+
+DSC_API unsigned dsc_device_fault(int reset) { return dsc::read_device_fault(reset != 0); }
 
 DSC_API const char *dsc_status_string(dsc_status_t s) {
     switch (s) {

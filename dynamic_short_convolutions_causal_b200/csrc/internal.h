@@ -27,8 +27,10 @@ void launch_lowrank_bwd_simt(const void *x, const void *z, const void *U, const 
                              float *dz, float *dU, void *ws, int B, int T, int D, int G, int W,
                              int R, bool bf16, cudaStream_t s);
 
-// Tensor-core (tcgen05) low-rank kernels (tc_fwd.cu, tc_bwd.cu)
-bool tc_lowrank_supported(int B, int T, int D, int G, int W, int R, bool bf16);
+// Tensor-core (tcgen05) low-rank kernels (tc_lowrank.cu)
+bool tc_lowrank_fwd_supported(int B, int T, int D, int G, int W, int R, bool bf16);
+bool tc_lowrank_bwd_supported(int B, int T, int D, int G, int W, int R, bool bf16);
+unsigned read_device_fault(bool reset);
 cudaError_t launch_tc_lowrank_fwd(const void *x, const void *z, const void *U, void *y, int B,
                                   int T, int D, int G, int W, int R, cudaStream_t s);
 size_t tc_lowrank_bwd_workspace(int B, int T, int D, int G, int W, int R);

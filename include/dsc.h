@@ -158,9 +158,18 @@ DSC_API dsc_status_t dsc_static_bwd_noalloc(const void *x, const void *w, const 
 /* Size in bytes of the fixed scratch array dsc_static_bwd_noalloc uses. */
 DSC_API size_t dsc_static_bwd_noalloc_max_scratch_bytes(void);
 
-/* Which implementation dsc_fwd_lowrank / dsc_bwd_lowrank use for these sizes:
- * 1 = tensor-core (tcgen05) kernels, 0 = CUDA-core kernels, -1 = invalid sizes. */
+/* Which implementations the low-rank entry points use for these sizes: bit 0 set when
+ * dsc_fwd_lowrank runs on the tensor-core (tcgen05) kernel, bit 1 when
+ * dsc_bwd_lowrank does; 0 = both on CUDA cores; -1 = invalid sizes.  The tensor-core
+ * kernels take bf16 with R in {16, 32, 64}, D a multiple of 64, G a power of two
+ * <= 64 and (64/G)*W a multiple of 8; other valid sizes run on CUDA cores. */
 DSC_API int dsc_lowrank_path(int B, int T, int D, int G, int W, int R, dsc_dtype_t dt);
+
+/* Diagnostic: the current device's fault word.  A tensor-core kernel that waited past
+ * its time limit (one second per wait) records a nonzero code here and returns early,
+ * leaving its outputs undefined.  Synchronous (copies from the device); reset != 0
+ * clears the word afterwards. */
+DSC_API unsigned dsc_device_fault(int reset);
 
 /* Static description of a status code. */
 DSC_API const char *dsc_status_string(dsc_status_t status);

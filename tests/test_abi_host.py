@@ -111,4 +111,4 @@ def test_lowrank_path_query(dsc):
     assert L.dsc_lowrank_path(0, 8, 64, 1, 4, 32, 1) == -1
     assert L.dsc_lowrank_path(2, 8, 64, 1, 4, 32, 0) == 0      # fp32: CUDA cores
     assert L.dsc_lowrank_path(2, 8, 64, 1, 4, 3, 1) == 0       # R=3: CUDA cores
-    assert L.dsc_lowrank_path(2, 8, 64, 1, 4, 32, 1) in (0, 1)
+    assert L.dsc_lowrank_path(2, 8, 64, 1, 4, 32, 1) in (0, 1, 2, 3)

@@ -126,6 +126,14 @@ LOWRANK = [
     (2, 140, 320, 8, 7, 48, "bf16"),
     (2, 70, 64, 1, 4, 32, "f32"),
     (1, 100, 48, 3, 3, 8, "f32"),
+    # shapes aimed at the tensor-core kernels
+    (1, 4096, 2048, 1, 4, 16, "bf16"),   # many tiles per CTA: ring wrap-around, slice changes
+    (2, 1000, 512, 1, 8, 64, "bf16"),    # 512 filter columns: two MMA N-chunks, one accumulator
+    (2, 300, 256, 16, 2, 32, "bf16"),    # G = 16
+    (2, 129, 128, 32, 4, 64, "bf16"),    # G = 32
+    (1, 200, 128, 64, 8, 32, "bf16"),    # G = 64
+    (2, 77, 128, 8, 1, 16, "bf16"),      # W = 1
+    (3, 2048, 384, 2, 3, 32, "bf16"),    # G = 2, W = 3
 ]
 
 
@@ -152,6 +160,17 @@ def test_lowrank_fwd_bwd(dsc, B, T, D, G, W, R, dt):
     assert_close(dx, rdx, dt, "dx")
     assert_close(dz, rdz, dt, "dz", reduction=True)
     assert_close(dU, rdU, dt, "dU", reduction=True)
+
+
+def test_tensor_core_path_is_selected(dsc):
+    """The bf16 workloads of the benchmark run on the tcgen05 forward kernel."""
+    for name in ("lowrank_qkv", "lowrank_mlp"):
+        wl = di.WORKLOADS[name]
+        assert dsc.dsc_lowrank_path(wl.B, wl.T, wl.D, wl.G, wl.W, wl.R) & 1, name
+
+
+def test_no_device_fault_recorded(dsc):
+    assert dsc.dsc_device_fault() == 0
 
 
 def test_lowrank_deterministic(dsc):
