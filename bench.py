@@ -247,8 +247,10 @@ def run_ours(args, wl, world, rank, local):
     gbs_step = (fwd_b + bwd_b) / (ms_step * 1e-3) / 1e9
     dom = ("dsc_bwd_lowrank", bwd_b, bwd_ms) if bwd_ms >= fwd_ms else ("dsc_fwd_lowrank", fwd_b, fwd_ms)
     achieved = dom[1] / (dom[2] * 1e-3) / 1e9
-    launches_fwd = 1 if path == 1 else 1
-    launches_bwd = 2 if path == 1 else 5
+    # kernels per call: tcgen05 forward 1; tcgen05 backward 4 (U reorder, main, dz and dU
+    # reductions); CUDA-core forward 1, backward 5
+    launches_fwd = 1
+    launches_bwd = 4 if path & 2 else 5
     traffic = load_traffic(dom[0], wl)
 
     # end to end through the public API with host buffers (pinned), copies inside the region
@@ -270,7 +272,8 @@ def run_ours(args, wl, world, rank, local):
             "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "D": wl.D, "G": G, "W": W, "R": R,
                        "tokens_per_step_per_gpu": wl.tokens, "parallelism": "dp%d" % world,
                        "l2": "inputs larger than L2 (x is %.0f MB), no flush" % (wl.tokens * wl.D * 2 / 1e6),
-                       "path": "tcgen05" if path == 1 else "cuda-cores"},
+                       "path": {"fwd": "tcgen05" if path & 1 else "cuda-cores",
+                                "bwd": "tcgen05" if path & 2 else "cuda-cores"}},
             "hbm_gbs_step": gbs_step, "hbm_pct_of_peak_step": 100.0 * gbs_step / peak,
             "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
             "fwd_gbs": fwd_b / (fwd_ms * 1e-3) / 1e9, "bwd_gbs": bwd_b / (bwd_ms * 1e-3) / 1e9,

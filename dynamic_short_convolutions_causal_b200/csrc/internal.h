@@ -31,6 +31,7 @@ void launch_lowrank_bwd_simt(const void *x, const void *z, const void *U, const 
 bool tc_lowrank_fwd_supported(int B, int T, int D, int G, int W, int R, bool bf16);
 bool tc_lowrank_bwd_supported(int B, int T, int D, int G, int W, int R, bool bf16);
 unsigned read_device_fault(bool reset);
+unsigned read_device_fault_bwd(bool reset);
 cudaError_t launch_tc_lowrank_fwd(const void *x, const void *z, const void *U, void *y, int B,
                                   int T, int D, int G, int W, int R, cudaStream_t s);
 size_t tc_lowrank_bwd_workspace(int B, int T, int D, int G, int W, int R);

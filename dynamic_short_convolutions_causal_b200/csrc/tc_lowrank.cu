@@ -33,40 +33,46 @@ namespace tc {
 
 __device__ unsigned int g_fault = 0;
 
+// Build-time tuning constants of the forward kernel.
+#ifndef DSC_FWD_SETS
+#define DSC_FWD_SETS 2         // epilogue warp sets working on alternating tiles (1 or 2)
+#endif
+#ifndef DSC_FWD_F32X2
+#define DSC_FWD_F32X2 0        // pair taps with packed fp32x2 FMAs (1) or use scalar FMAs (0)
+#endif
+#ifndef DSC_X_L2_PROMO
+#define DSC_X_L2_PROMO 128     // L2 promotion of the x tile loads (128 or 256 bytes)
+#endif
+
 constexpr int kTt = 128;          // tokens per tile (MMA M)
 constexpr int kDt = 64;           // channels per slice
-constexpr int kEpiWarps = 8;
-constexpr int kThreads = 32 * (2 + kEpiWarps);
-constexpr int kYBuf = 32 * 64;    // one warp's y staging: 32 rows x 32 bf16 channels
 
 struct FwdParams {
     int B, T, D, G, R;
-    int per_slice;            // B * tiles_per_seq
+    int n_slices;             // D / 64
     int tiles_per_seq;
-    int n_tiles;
+    int n_tiles;              // tiles in token-major order: i = token_tile * n_slices + slice
     int slice_cols;           // (64/G)*W
     int n_pad;                // slice_cols rounded up to 16
     int u_boxes;              // ceil(n_pad / 64) TMA boxes of 64 columns
     int bufcols, nbuf, tmem_cols;
-    int stages, nU;
-    uint32_t x_stage_tx, x_stage_bytes, z_stage_bytes, u_bytes;
-    uint32_t off_x, off_z, off_u, off_y, off_bar;
+    int stages, nwg;          // nwg: epilogue warp sets (1 or 2)
+    uint32_t x_stage_tx, x_stage_bytes, z_stage_bytes, u_bytes, y_buf_bytes;
+    uint32_t stage_bytes;     // one ring stage: x tile, z tile and the U slice
+    uint32_t off_x, off_z, off_u, off_y, off_bar;   // off_x/z/u within a stage
     uint32_t z_layout;        // swizzle of the z tile (32/64/128-byte rows)
 };
 
-// Barrier slots in shared memory (in units of 8 bytes) for a ring of `S` stages.
+// Barrier slots in shared memory (8 bytes each).
 struct Bars {
     uint32_t base;
-    int S;
     __device__ uint32_t full(int s) const { return base + 8 * s; }
     __device__ uint32_t empty(int s) const { return base + 8 * (4 + s); }
     __device__ uint32_t accf(int a) const { return base + 8 * (8 + a); }
     __device__ uint32_t acce(int a) const { return base + 8 * (10 + a); }
-    __device__ uint32_t uf(int u) const { return base + 8 * (12 + u); }
-    __device__ uint32_t ue(int u) const { return base + 8 * (14 + u); }
-    __device__ uint32_t done() const { return base + 8 * 16; }
+    __device__ uint32_t done() const { return base + 8 * 12; }
 };
-constexpr uint32_t kBarBytes = 8 * 17;
+constexpr uint32_t kBarBytes = 8 * 13;
 
 __device__ __forceinline__ void unpack8(const uint4 &u, float (&v)[8]) {
     v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x);
@@ -75,40 +81,89 @@ __device__ __forceinline__ void unpack8(const uint4 &u, float (&v)[8]) {
     v[6] = bf16_lo(u.w); v[7] = bf16_hi(u.w);
 }
 
-// Columns of the chunk's filter taps, read from TMEM into wr[]:
-//   GC <= 8: 8/GC groups x W taps, group-major (column gl*W + k), loaded as W pieces of
-//            8/GC columns, each piece aligned to its width;
-//   GC == 16 (any G >= 16): one group, W columns, loaded one by one.
+__host__ __device__ constexpr int pow2_divisor(int n, int cap) {
+    int p = 1;
+    while (p * 2 <= cap && n % (p * 2) == 0) p *= 2;
+    return p;
+}
+
+// Filter taps of one 8-channel chunk, read from TMEM:
+//   GC <= 8: 8/GC groups x W taps in U's column order (column gl*W + k), a contiguous
+//            block of NCOL columns loaded in aligned pieces of PIECE columns;
+//   GC == 16 (any G >= 16): one group, W columns.
 template <int W, int GC>
 struct Taps {
-    static constexpr int PIECE = GC <= 8 ? 8 / GC : 1;
-    static constexpr int NCOL = PIECE * W;
+    static constexpr int NCOL = GC <= 8 ? (8 / GC) * W : W;
+    static constexpr int PIECE = GC <= 8 ? pow2_divisor(NCOL, 64) : 1;
 };
 
+// Epilogue: each set of 8 warps covers one whole tile (warp = 32 token rows x 32
+// channels); with two sets, consecutive tiles (the two TMEM accumulator buffers) are
+// processed concurrently.  Two sets need the chunk's taps to fit in 32 registers.
 template <int W, int GC>
-__global__ void __launch_bounds__(kThreads, 1)
+struct EpiShape {
+    static constexpr int SETS = (Taps<W, GC>::NCOL <= 32 && DSC_FWD_SETS >= 2) ? 2 : 1;
+    static constexpr int WARPS = 8 * SETS;
+    static constexpr int THREADS = 32 * (2 + WARPS);
+    static constexpr int CPW = 32;                 // channels per epilogue warp
+    static constexpr int CHUNKS = CPW / 8;
+    static constexpr int YBUF = 32 * CPW * 2;      // one warp's y staging: 32 rows x 32 bf16
+};
+
+// y[t,c] = x[t,c] + sum_k w[t, g(c), k] x[t-k, c] for the 8 channels of one chunk.
+template <int W, int GC>
+__device__ __forceinline__ void conv_chunk(const uint32_t *wr, const uint4 (&xu)[W], float (&out)[8]) {
+    float xv[W][8];
+#pragma unroll
+    for (int k = 0; k < W; ++k) unpack8(xu[k], xv[k]);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        const int gl = GC <= 8 ? e / GC : 0;
+        const uint32_t *wg = wr + gl * W;
+#if DSC_FWD_F32X2
+        // taps in pairs with packed fp32x2 FMAs (two partial sums, added at the end)
+        uint64_t acc = f2pack(xv[0][e], 0.f);
+#pragma unroll
+        for (int k = 0; k + 1 < W; k += 2)
+            acc = f2fma(f2pack(__uint_as_float(wg[k]), __uint_as_float(wg[k + 1])),
+                        f2pack(xv[k][e], xv[k + 1][e]), acc);
+        float a0, a1;
+        f2unpack(acc, a0, a1);
+        if (W & 1) a0 = fmaf(__uint_as_float(wg[W - 1]), xv[W - 1][e], a0);
+        out[e] = a0 + a1;
+#else
+        float acc = xv[0][e];
+#pragma unroll
+        for (int k = 0; k < W; ++k) acc = fmaf(__uint_as_float(wg[k]), xv[k][e], acc);
+        out[e] = acc;
+#endif
+    }
+}
+
+template <int W, int GC>
+__global__ void __launch_bounds__(EpiShape<W, GC>::THREADS, 1)
 k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z,
                  const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_y,
                  const FwdParams p) {
+    using ES = EpiShape<W, GC>;
+    using TP = Taps<W, GC>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sb = smem_u32(smem);
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const Bars bar{sb + p.off_bar, p.stages};
+    const Bars bar{sb + p.off_bar};
     uint32_t *tmem_holder = (uint32_t *)(smem + p.off_bar + kBarBytes);
     volatile int *abort = (volatile int *)(smem + p.off_bar + kBarBytes + 8);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < p.stages; ++s) {
             mbar_init(bar.full(s), 1);
-            mbar_init(bar.empty(s), kEpiWarps);
+            mbar_init(bar.empty(s), 8);
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(bar.accf(a), 1);
-            mbar_init(bar.acce(a), kEpiWarps);
-            mbar_init(bar.uf(a), 1);
-            mbar_init(bar.ue(a), 1);
+            mbar_init(bar.acce(a), 8);
         }
         mbar_init(bar.done(), 1);
         *abort = 0;
@@ -129,38 +184,27 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
-    const int tbeg = (int)((long long)blockIdx.x * p.n_tiles / gridDim.x);
-    const int tend = (int)((long long)(blockIdx.x + 1) * p.n_tiles / gridDim.x);
     const int S = p.stages;
 
     if (warp == 0) {
         // ---------------------------------------------------------- TMA producer
         if (lane == 0) {
-            int prev = -1, v = -1;
-            for (int i = tbeg; i < tend; ++i) {
-                const int it = i - tbeg;
-                const int slice = i / p.per_slice, rem = i % p.per_slice;
-                const int b = rem / p.tiles_per_seq, t0 = (rem % p.tiles_per_seq) * kTt;
-                if (slice != prev) {
-                    prev = slice;
-                    ++v;
-                    const int ub = v % p.nU, un = v / p.nU;
-                    if (!mbar_wait(bar.ue(ub), (un & 1) ^ 1, abort, 1u, &g_fault)) break;
-                    mbar_arrive_expect_tx(bar.uf(ub), p.u_bytes);
-                    const uint32_t ud = sb + p.off_u + ub * p.u_bytes;
-                    for (int bx = 0; bx < p.u_boxes; ++bx)
-                        tma_load_2d(ud + bx * (uint32_t)(p.R * 128), &tm_u, bar.uf(ub),
-                                    slice * p.slice_cols + 64 * bx, 0);
-                }
+            int it = 0;
+            for (int i = blockIdx.x; i < p.n_tiles; i += gridDim.x, ++it) {
+                const int slice = i % p.n_slices, tl_ = i / p.n_slices;
+                const int b = tl_ / p.tiles_per_seq, t0 = (tl_ % p.tiles_per_seq) * kTt;
                 const int s = it % S, n = it / S;
                 if (!mbar_wait(bar.empty(s), (n & 1) ^ 1, abort, 2u, &g_fault)) break;
-                mbar_arrive_expect_tx(bar.full(s), p.x_stage_tx + p.z_stage_bytes);
-                tma_load_3d(sb + p.off_x + s * p.x_stage_bytes, &tm_x, bar.full(s), slice * kDt,
-                            t0 - (W - 1), b);
-                tma_load_3d(sb + p.off_z + s * p.z_stage_bytes, &tm_z, bar.full(s), 0, t0, b);
+                mbar_arrive_expect_tx(bar.full(s), p.x_stage_tx + p.z_stage_bytes + p.u_bytes);
+                const uint32_t st = sb + s * p.stage_bytes;
+                tma_load_3d(st + p.off_x, &tm_x, bar.full(s), slice * kDt, t0 - (W - 1), b);
+                tma_load_3d(st + p.off_z, &tm_z, bar.full(s), 0, t0, b);
+                for (int bx = 0; bx < p.u_boxes; ++bx)
+                    tma_load_2d(st + p.off_u + bx * (uint32_t)(p.R * 128), &tm_u, bar.full(s),
+                                slice * p.slice_cols + 64 * bx, 0);
             }
             // Let every load this warp issued land before the CTA can exit.
-            const int issued = tend - tbeg;
+            const int issued = it;
             for (int s = 0; s < S && s < issued; ++s) {
                 const int last = issued - 1 - ((issued - 1 - s) % S);   // last tile using stage s
                 mbar_wait(bar.full(s), (last / S) & 1, abort, 0u, &g_fault);
@@ -172,24 +216,16 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
         if (lane == 0) {
             const int nchunks = (p.n_pad + 255) / 256;
             const uint32_t zsbo = 8u * p.R * 2u;
-            int prev = -1, v = -1, ub = 0;
-            for (int i = tbeg; i < tend; ++i) {
-                const int it = i - tbeg;
-                const int slice = i / p.per_slice;
-                if (slice != prev) {
-                    prev = slice;
-                    ++v;
-                    ub = v % p.nU;
-                    if (!mbar_wait(bar.uf(ub), (v / p.nU) & 1, abort, 4u, &g_fault)) break;
-                }
+            int it = 0;
+            for (int i = blockIdx.x; i < p.n_tiles; i += gridDim.x, ++it) {
                 const int s = it % S, n = it / S;
                 const int a = it % p.nbuf, m = it / p.nbuf;
                 if (!mbar_wait(bar.full(s), n & 1, abort, 8u, &g_fault)) break;
                 if (!mbar_wait(bar.acce(a), (m & 1) ^ 1, abort, 16u, &g_fault)) break;
                 tc_fence_after();
                 const uint32_t d = tmem + a * p.bufcols;
-                const uint32_t za = sb + p.off_z + s * p.z_stage_bytes;
-                const uint32_t ua = sb + p.off_u + ub * p.u_bytes;
+                const uint32_t za = sb + s * p.stage_bytes + p.off_z;
+                const uint32_t ua = sb + s * p.stage_bytes + p.off_u;
                 for (int nc = 0; nc < nchunks; ++nc) {
                     const int ncols = min(256, p.n_pad - 256 * nc);
                     const uint32_t idesc = idesc_bf16(128, ncols, false, true);
@@ -201,73 +237,78 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
                     }
                 }
                 mma_commit(bar.accf(a));
-                const bool last_of_slice = (i + 1 == tend) || ((i + 1) / p.per_slice != slice);
-                if (last_of_slice) mma_commit(bar.ue(ub));
             }
             mma_commit(bar.done());
         }
         __syncwarp();
     } else {
         // ---------------------------------------------------------- epilogue
-        using TP = Taps<W, GC>;
+        const int ew = warp - 2;
+        const int set = ew >> 3;             // tiles it with it % SETS == set
         const int q = warp & 3;              // TMEM lane quarter == token rows 32q..32q+31
-        const int h = (warp - 2) >> 2;       // channel half of the slice
+        const int h = (ew >> 2) & 1;         // channel half of the slice
         const int row = 32 * q + lane;       // token row in the tile
-        const uint32_t ybase = sb + p.off_y + (uint32_t)(warp - 2) * 2 * kYBuf;
-        uint8_t *ygen = smem + p.off_y + (warp - 2) * 2 * kYBuf;
+        // y staging: row `lane` of this warp's buffer, 64-byte swizzle (16-byte chunk ^ (lane/2)%4)
+        const uint32_t ystage = sb + p.off_y + (uint32_t)ew * 2 * ES::YBUF;
+        const uint32_t yrow = (ystage + lane * 64) ^ ((uint32_t)((lane >> 1) & 3) << 4);
+        // x stage: the thread's rows r_k = row + W-1-k; a row is 128 bytes with 128-byte
+        // swizzle (16-byte chunk ^ r%8).  Rows are 128-byte aligned, so the swizzled address
+        // of chunk c is (row address ^ ((r%8) << 4)) ^ (c << 4).
+        uint32_t xrow[W];
+#pragma unroll
+        for (int k = 0; k < W; ++k) {
+            const uint32_t r = (uint32_t)(row + (W - 1) - k);
+            xrow[k] = (r * 128u) ^ ((r & 7u) << 4) ^ ((uint32_t)(4 * h) << 4);
+        }
         int yc = 0;
-        for (int i = tbeg; i < tend; ++i) {
-            const int it = i - tbeg;
-            const int slice = i / p.per_slice, rem = i % p.per_slice;
-            const int b = rem / p.tiles_per_seq, t0 = (rem % p.tiles_per_seq) * kTt;
+        int it = set;
+        int i = blockIdx.x + set * gridDim.x;
+        int slice = i % p.n_slices, tlin = i / p.n_slices;
+        const int step = ES::SETS * gridDim.x;
+        const int dslice = step % p.n_slices, dtl = step / p.n_slices;
+        for (; i < p.n_tiles; it += ES::SETS, i += step) {
+            const int b = tlin / p.tiles_per_seq, t0 = (tlin - b * p.tiles_per_seq) * kTt;
             const int s = it % S, n = it / S;
             const int a = it % p.nbuf, m = it / p.nbuf;
-            if (!mbar_wait(bar.full(s), n & 1, abort, 32u, &g_fault)) break;
-            if (!mbar_wait(bar.accf(a), m & 1, abort, 64u, &g_fault)) break;
+            if (!warp_wait(bar.full(s), n & 1, abort, 32u, &g_fault)) break;
+            if (!warp_wait(bar.accf(a), m & 1, abort, 64u, &g_fault)) break;
             tc_fence_after();
             const int yb = yc & 1;
             if (lane == 0) bulk_wait_read<1>();
             __syncwarp();
-            const uint8_t *xs = smem + p.off_x + s * p.x_stage_bytes;
+            const uint32_t xs = sb + s * p.stage_bytes + p.off_x;
             const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16) + a * p.bufcols;
-#pragma unroll
-            for (int cq = 0; cq < 4; ++cq) {
-                const int c8 = 32 * h + 8 * cq;          // first channel of the chunk in the slice
-                uint32_t wr[TP::NCOL];
+            const uint32_t yw = yrow + yb * ES::YBUF;
+            uint32_t wr[2][TP::NCOL];
+            auto issue_taps = [&](int cq, uint32_t *dst) {
+                const int c8 = ES::CPW * h + 8 * cq;
                 if (GC <= 8) {
                     const uint32_t col = (uint32_t)((c8 / GC) * W);
 #pragma unroll
-                    for (int m2 = 0; m2 < W; ++m2) tmem_ld<TP::PIECE>(tl + col + m2 * TP::PIECE, &wr[m2 * TP::PIECE]);
+                    for (int m2 = 0; m2 < TP::NCOL / TP::PIECE; ++m2)
+                        tmem_ld<TP::PIECE>(tl + col + m2 * TP::PIECE, dst + m2 * TP::PIECE);
                 } else {
                     const uint32_t col = (uint32_t)((c8 / p.G) * W);
 #pragma unroll
-                    for (int k = 0; k < W; ++k) tmem_ld<1>(tl + col + k, &wr[k]);
+                    for (int k = 0; k < W; ++k) tmem_ld<1>(tl + col + k, dst + k);
                 }
-                float xv[W][8];
+            };
+            issue_taps(0, wr[0]);
 #pragma unroll
-                for (int k = 0; k < W; ++k) {
-                    const int rw = row + (W - 1) - k;
-                    const int ch = (4 * h + cq) ^ (rw & 7);
-                    const uint4 u = *reinterpret_cast<const uint4 *>(xs + rw * 128 + ch * 16);
-                    unpack8(u, xv[k]);
-                }
-                tmem_wait_ld_regs(wr);
+            for (int cq = 0; cq < ES::CHUNKS; ++cq) {
+                uint4 xu[W];
+#pragma unroll
+                for (int k = 0; k < W; ++k) xu[k] = lds128(xs + (xrow[k] ^ ((uint32_t)cq << 4)));
+                tmem_wait_ld_regs(wr[cq & 1]);
+                if (cq + 1 < ES::CHUNKS) issue_taps(cq + 1, wr[(cq + 1) & 1]);   // overlaps the math below
                 float out[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int gl = GC <= 8 ? e / GC : 0;
-                    float acc = xv[0][e];
-#pragma unroll
-                    for (int k = 0; k < W; ++k) acc = fmaf(__uint_as_float(wr[gl * W + k]), xv[k][e], acc);
-                    out[e] = acc;
-                }
+                conv_chunk<W, GC>(wr[cq & 1], xu, out);
                 uint4 o;
                 o.x = pack_bf16x2(out[0], out[1]);
                 o.y = pack_bf16x2(out[2], out[3]);
                 o.z = pack_bf16x2(out[4], out[5]);
                 o.w = pack_bf16x2(out[6], out[7]);
-                const int pc = cq ^ ((lane >> 1) & 3);   // 64-byte swizzle of the staging rows
-                *reinterpret_cast<uint4 *>(ygen + yb * kYBuf + lane * 64 + pc * 16) = o;
+                sts128(yw ^ ((uint32_t)cq << 4), o);
             }
             tc_fence_before();
             fence_proxy_async_smem();
@@ -275,10 +316,16 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
             if (lane == 0) {
                 mbar_arrive(bar.acce(a));
                 mbar_arrive(bar.empty(s));
-                tma_store_3d(&tm_y, ybase + yb * kYBuf, slice * kDt + 32 * h, t0 + 32 * q, b);
+                tma_store_3d(&tm_y, ystage + yb * ES::YBUF, slice * kDt + ES::CPW * h, t0 + 32 * q, b);
                 bulk_commit();
             }
             ++yc;
+            slice += dslice;
+            tlin += dtl;
+            if (slice >= p.n_slices) {
+                slice -= p.n_slices;
+                ++tlin;
+            }
         }
         if (lane == 0) bulk_wait_all();
         __syncwarp();
@@ -313,7 +360,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encoder() {
 
 // Row-major bf16 tensor map; dims[0] is the contiguous dimension.
 bool make_map(CUtensorMap *m, const void *ptr, int rank, const uint64_t *dims, const uint32_t *box,
-              CUtensorMapSwizzle sw) {
+              CUtensorMapSwizzle sw, CUtensorMapL2promotion promo = CU_TENSOR_MAP_L2_PROMOTION_L2_128B) {
     auto enc = encoder();
     if (!enc) return false;
     cuuint64_t gdim[3], gstride[2];
@@ -326,7 +373,7 @@ bool make_map(CUtensorMap *m, const void *ptr, int rank, const uint64_t *dims, c
         stride *= dims[i];
     }
     const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void *>(ptr), gdim, gstride,
-                           bdim, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           bdim, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, promo,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
@@ -353,8 +400,8 @@ bool plan_fwd(int B, int T, int D, int G, int W, int R, FwdParams &p) {
     p.n_pad = (p.slice_cols + 15) / 16 * 16;
     p.u_boxes = (p.n_pad + 63) / 64;
     p.tiles_per_seq = (T + kTt - 1) / kTt;
-    p.per_slice = B * p.tiles_per_seq;
-    const long long nt = (long long)(D / kDt) * p.per_slice;
+    p.n_slices = D / kDt;
+    const long long nt = (long long)p.n_slices * B * p.tiles_per_seq;
     if (nt >= (1ll << 31)) return false;
     p.n_tiles = (int)nt;
     p.bufcols = p.n_pad;
@@ -367,18 +414,22 @@ bool plan_fwd(int B, int T, int D, int G, int W, int R, FwdParams &p) {
     p.z_stage_bytes = (uint32_t)(kTt * R * 2);
     p.u_bytes = (uint32_t)(p.u_boxes * R * 128);
     p.z_layout = R == 16 ? kSw32 : (R == 32 ? kSw64 : kSw128);
-    const int options[5][2] = {{4, 2}, {3, 2}, {4, 1}, {3, 1}, {2, 1}};
-    for (auto &o : options) {
-        const uint32_t off_x = 0;
-        const uint32_t off_z = off_x + o[0] * p.x_stage_bytes;
-        const uint32_t off_u = off_z + o[0] * p.z_stage_bytes;
-        const uint32_t off_y = off_u + o[1] * p.u_bytes;
-        const uint32_t off_bar = off_y + kEpiWarps * 2 * kYBuf;
+    const int ncol = G <= 8 ? (8 / G) * W : W;      // must match EpiShape / Taps
+    p.nwg = (ncol <= 32 && DSC_FWD_SETS >= 2) ? 2 : 1;   // epilogue warp sets
+    if (p.nbuf < p.nwg) p.nwg = p.nbuf;
+    p.y_buf_bytes = (uint32_t)(32 * 32 * 2);
+    p.off_x = 0;
+    p.off_z = p.x_stage_bytes;
+    p.off_u = p.off_z + p.z_stage_bytes;
+    p.stage_bytes = (p.off_u + p.u_bytes + 1023) / 1024 * 1024;
+    for (int st = 4; st >= 2; --st) {
+        const uint32_t off_y = st * p.stage_bytes;
+        const uint32_t off_bar = off_y + 8 * p.nwg * 2 * p.y_buf_bytes;
         const uint32_t total = off_bar + kBarBytes + 16 + 1024;
         if (total <= kSmemLimit) {
-            p.stages = o[0];
-            p.nU = o[1];
-            p.off_x = off_x; p.off_z = off_z; p.off_u = off_u; p.off_y = off_y; p.off_bar = off_bar;
+            p.stages = st;
+            p.off_y = off_y;
+            p.off_bar = off_bar;
             return true;
         }
     }
@@ -391,11 +442,13 @@ template <int W, int GC>
 cudaError_t launch_fwd_t(const CUtensorMap &mx, const CUtensorMap &mz, const CUtensorMap &mu,
                          const CUtensorMap &my, const FwdParams &p, cudaStream_t s) {
     auto kern = k_tc_lowrank_fwd<W, GC>;
+    using ES = EpiShape<W, GC>;
+    if (p.nwg != ES::SETS || p.y_buf_bytes != (uint32_t)ES::YBUF) return cudaErrorInvalidConfiguration;
     const uint32_t smem = smem_bytes(p);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int grid = std::min(p.n_tiles, num_sms());
-    kern<<<grid, kThreads, smem, s>>>(mx, mz, mu, my, p);
+    kern<<<grid, ES::THREADS, smem, s>>>(mx, mz, mu, my, p);
     return cudaGetLastError();
 }
 
@@ -434,8 +487,11 @@ cudaError_t launch_tc_lowrank_fwd(const void *x, const void *z, const void *U, v
     const uint32_t by[3] = {32, 32, 1};
     const CUtensorMapSwizzle zsw = R == 16 ? CU_TENSOR_MAP_SWIZZLE_32B
                                            : (R == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
-    if (!make_map(&mx, x, 3, dx, bx, CU_TENSOR_MAP_SWIZZLE_128B) || !make_map(&mz, z, 3, dz, bz, zsw) ||
-        !make_map(&mu, U, 2, du, bu, CU_TENSOR_MAP_SWIZZLE_128B) ||
+    const CUtensorMapL2promotion xpromo =
+        DSC_X_L2_PROMO == 256 ? CU_TENSOR_MAP_L2_PROMOTION_L2_256B : CU_TENSOR_MAP_L2_PROMOTION_L2_128B;
+    if (!make_map(&mx, x, 3, dx, bx, CU_TENSOR_MAP_SWIZZLE_128B, xpromo) ||
+        !make_map(&mz, z, 3, dz, bz, zsw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
+        !make_map(&mu, U, 2, du, bu, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
         !make_map(&my, y, 3, dx, by, CU_TENSOR_MAP_SWIZZLE_64B)) {
         set_last_error("dsc_fwd_lowrank: cuTensorMapEncodeTiled failed");
         return cudaErrorInvalidValue;
@@ -452,15 +508,6 @@ cudaError_t launch_tc_lowrank_fwd(const void *x, const void *z, const void *U, v
     }
 }
 
-bool tc_lowrank_bwd_supported(int, int, int, int, int, int, bool) { return false; }
-
-size_t tc_lowrank_bwd_workspace(int, int, int, int, int, int) { return 0; }
-
-cudaError_t launch_tc_lowrank_bwd(const void *, const void *, const void *, const void *, void *, float *,
-                                  float *, void *, int, int, int, int, int, int, cudaStream_t) {
-    return cudaErrorNotSupported;
-}
-
 unsigned read_device_fault(bool reset) {
     unsigned v = 0;
     if (cudaMemcpyFromSymbol(&v, tc::g_fault, sizeof(v)) != cudaSuccess) return 0xffffffffu;
@@ -468,7 +515,7 @@ unsigned read_device_fault(bool reset) {
         const unsigned z = 0;
         cudaMemcpyToSymbol(tc::g_fault, &z, sizeof(z));
     }
-    return v;
+    return v | (read_device_fault_bwd(reset) << 16);
 }
 
 }  // namespace dsc

@@ -134,6 +134,9 @@ LOWRANK = [
     (1, 200, 128, 64, 8, 32, "bf16"),    # G = 64
     (2, 77, 128, 8, 1, 16, "bf16"),      # W = 1
     (3, 2048, 384, 2, 3, 32, "bf16"),    # G = 2, W = 3
+    (2, 500, 256, 4, 4, 16, "bf16"),     # backward: 64 filter columns, padded dU^T block
+    (2, 260, 128, 1, 3, 32, "bf16"),     # backward: 192 filter columns, padded dU^T block
+    (1, 300, 128, 2, 8, 32, "bf16"),     # backward: G = 2, W = 8
 ]
 
 
@@ -163,10 +166,11 @@ def test_lowrank_fwd_bwd(dsc, B, T, D, G, W, R, dt):
 
 
 def test_tensor_core_path_is_selected(dsc):
-    """The bf16 workloads of the benchmark run on the tcgen05 forward kernel."""
+    """The bf16 workloads of the benchmark run on the tcgen05 kernels (forward: bit 0,
+    backward: bit 1)."""
     for name in ("lowrank_qkv", "lowrank_mlp"):
         wl = di.WORKLOADS[name]
-        assert dsc.dsc_lowrank_path(wl.B, wl.T, wl.D, wl.G, wl.W, wl.R) & 1, name
+        assert dsc.dsc_lowrank_path(wl.B, wl.T, wl.D, wl.G, wl.W, wl.R) == 3, name
 
 
 def test_no_device_fault_recorded(dsc):
