@@ -43,7 +43,6 @@ constexpr int kTt = 128;
 constexpr int kDt = 64;
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 32 * (2 + kEpiWarps);
-constexpr int kStages = 2;
 
 struct BwdParams {
     int B, T, D, G, W, R;
@@ -53,7 +52,7 @@ struct BwdParams {
     int SCp;                  // SC rounded up to 128 (dU^T M-blocks)
     int n_slices, tiles_per_seq, per_slice, n_tiles, maxseg;
     int u_boxes;              // TMA boxes of 64 Up columns per slice
-    int nU;
+    int nU, stages;
     uint32_t rows;            // tile rows incl. halo: 128 + W - 1
     uint32_t xy_tile_bytes;   // one dy or x tile (rows x 128 B), 1024-aligned
     uint32_t z_slab;          // stride of the 8-wide z slabs (rows x 16 B, rounded up to 128:
@@ -70,16 +69,16 @@ struct BwdParams {
 struct Bars {
     uint32_t base;
     __device__ uint32_t full(int s) const { return base + 8 * s; }
-    __device__ uint32_t empty(int s) const { return base + 8 * (2 + s); }
-    __device__ uint32_t uf(int u) const { return base + 8 * (4 + u); }
-    __device__ uint32_t ue(int u) const { return base + 8 * (6 + u); }
-    __device__ uint32_t wfull() const { return base + 8 * 8; }
-    __device__ uint32_t wempty() const { return base + 8 * 9; }
-    __device__ uint32_t dwready() const { return base + 8 * 10; }
-    __device__ uint32_t mm2() const { return base + 8 * 11; }
-    __device__ uint32_t done() const { return base + 8 * 12; }
+    __device__ uint32_t empty(int s) const { return base + 8 * (3 + s); }
+    __device__ uint32_t uf(int u) const { return base + 8 * (6 + u); }
+    __device__ uint32_t ue(int u) const { return base + 8 * (8 + u); }
+    __device__ uint32_t wfull() const { return base + 8 * 10; }
+    __device__ uint32_t wempty() const { return base + 8 * 11; }
+    __device__ uint32_t dwready() const { return base + 8 * 12; }
+    __device__ uint32_t mm2() const { return base + 8 * 13; }
+    __device__ uint32_t done() const { return base + 8 * 14; }
 };
-constexpr uint32_t kBarBytes = 8 * 13;
+constexpr uint32_t kBarBytes = 8 * 15;
 
 __device__ __forceinline__ void unpack8(const uint4 &u, float (&v)[8]) {
     v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x);
@@ -140,7 +139,7 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
     volatile int *abort = (volatile int *)(smem + p.off_bar + kBarBytes + 8);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < p.stages; ++s) {
             mbar_init(bar.full(s), 1);
             mbar_init(bar.empty(s), kEpiWarps);
         }
@@ -202,7 +201,7 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
                         tma_load_2d(ud + bx * (uint32_t)(p.R * 128), &tm_u, bar.uf(ub),
                                     id.slice * p.SC + 64 * bx, 0);
                 }
-                const int s = it % kStages, n = it / kStages;
+                const int s = it % p.stages, n = it / p.stages;
                 if (!mbar_wait(bar.empty(s), (n & 1) ^ 1, abort, 2u, &g_fault_bwd)) break;
                 mbar_arrive_expect_tx(bar.full(s), tx);
                 const uint32_t st = sb + s * p.stage_bytes;
@@ -212,20 +211,28 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
                     tma_load_3d(st + 2 * p.xy_tile_bytes + j * p.z_slab, &tm_z, bar.full(s), 8 * j, id.t0, id.b);
             }
             const int issued = tend - tbeg;
-            for (int s = 0; s < kStages && s < issued; ++s) {
-                const int last = issued - 1 - ((issued - 1 - s) % kStages);
-                mbar_wait(bar.full(s), (last / kStages) & 1, abort, 0u, &g_fault_bwd);
+            for (int s = 0; s < p.stages && s < issued; ++s) {
+                const int last = issued - 1 - ((issued - 1 - s) % p.stages);
+                mbar_wait(bar.full(s), (last / p.stages) & 1, abort, 0u, &g_fault_bwd);
             }
         }
         __syncwarp();
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
+        // Order per tile i: recompute(i) as soon as the epilogue has read w(i-1), then the
+        // dz / dU products of tile i-1 once its dw is written, so that they run while the
+        // epilogue computes dx of tile i.  Across a slice change the pending dz / dU go
+        // first: they release the U buffer the next slice may need.
         if (lane == 0) {
-            int prev = -1, v = -1, ub = 0;
+            int prev_slice = -1, v = -1, ub = 0;
+            struct Pending {
+                int it, s, ub;
+                bool seg_first, last_of_slice;
+            } pend = {-1, 0, 0, false, false};
             bool seg_first = true;
-            // recompute MMAs of one tile (W shifted products, N = NGp per tap)
+            bool ok = true;
             auto recompute = [&](int it, int ubuf) {
-                const int s = it % kStages;
+                const int s = it % p.stages;
                 const uint32_t zs = sb + s * p.stage_bytes + 2 * p.xy_tile_bytes;
                 const uint32_t us = sb + p.off_u + ubuf * p.u_bytes;
                 const uint32_t idesc = idesc_bf16(128, p.NGp, false, true);
@@ -240,56 +247,66 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
                 }
                 mma_commit(bar.wfull());
             };
-            for (int i = tbeg; i < tend; ++i) {
+            auto dzdu = [&](const Pending &t) -> bool {
+                if (!mbar_wait(bar.dwready(), t.it & 1, abort, 32u, &g_fault_bwd)) return false;
+                tc_fence_after();
+                const uint32_t us = sb + p.off_u + t.ub * p.u_bytes;
+                const uint32_t idz = idesc_bf16(128, p.R, false, false);
+                for (int kk = 0; kk < p.SC / 16; ++kk) {
+                    const int j0 = 16 * kk;
+                    const uint64_t bd =
+                        smem_desc(us + (j0 / 64) * (uint32_t)(p.R * 128) + (j0 % 64) * 2, 16, 1024, kSw128);
+                    mma_bf16_ts(tmem + p.tm_dz, tmem + p.tm_dw + 8 * kk, bd, idz, kk > 0 ? 1u : 0u);
+                }
+                const uint32_t zs = sb + t.s * p.stage_bytes + 2 * p.xy_tile_bytes;
+                const uint32_t idu = idesc_bf16(128, p.R, true, true);
+                for (int mb = 0; mb < p.SCp / 128; ++mb)
+                    for (int kk = 0; kk < kTt / 16; ++kk) {
+                        const uint64_t ad =
+                            smem_desc(sb + p.off_dw + mb * 2 * 16384 + kk * 2048, 16384, 1024, kSw128);
+                        const uint64_t bd = smem_desc(zs + kk * 256, 128, p.z_slab, kSwNone);
+                        mma_bf16_ss(tmem + p.tm_du + mb * p.R, ad, bd, idu, (t.seg_first && kk == 0) ? 0u : 1u);
+                    }
+                mma_commit(bar.mm2());
+                if (t.last_of_slice) mma_commit(bar.ue(t.ub));
+                return true;
+            };
+            for (int i = tbeg; i < tend && ok; ++i) {
                 const int it = i - tbeg;
                 const TileId id = tile_id(p, i);
-                if (id.slice != prev) {
-                    prev = id.slice;
+                if (id.slice != prev_slice) {
+                    if (pend.it >= 0) {
+                        if (!dzdu(pend)) { ok = false; break; }
+                        pend.it = -1;
+                    }
+                    prev_slice = id.slice;
                     ++v;
                     ub = v % p.nU;
                     seg_first = true;
-                    if (!mbar_wait(bar.uf(ub), (v / p.nU) & 1, abort, 4u, &g_fault_bwd)) break;
+                    if (!mbar_wait(bar.uf(ub), (v / p.nU) & 1, abort, 4u, &g_fault_bwd)) { ok = false; break; }
                 }
-                const int s = it % kStages, n = it / kStages;
-                if (!mbar_wait(bar.full(s), n & 1, abort, 8u, &g_fault_bwd)) break;
-                if (!mbar_wait(bar.wempty(), (it & 1) ^ 1, abort, 16u, &g_fault_bwd)) break;
+                const int s = it % p.stages, n = it / p.stages;
+                if (!mbar_wait(bar.full(s), n & 1, abort, 8u, &g_fault_bwd)) { ok = false; break; }
+                if (!mbar_wait(bar.wempty(), (it & 1) ^ 1, abort, 16u, &g_fault_bwd)) { ok = false; break; }
                 tc_fence_after();
                 recompute(it, ub);
-                // dz and dU once the epilogue has written dw
-                if (!mbar_wait(bar.dwready(), it & 1, abort, 32u, &g_fault_bwd)) break;
-                tc_fence_after();
-                {
-                    const uint32_t us = sb + p.off_u + ub * p.u_bytes;
-                    const uint32_t idesc = idesc_bf16(128, p.R, false, false);
-                    for (int kk = 0; kk < p.SC / 16; ++kk) {
-                        const int j0 = 16 * kk;
-                        const uint64_t bd = smem_desc(us + (j0 / 64) * (uint32_t)(p.R * 128) + (j0 % 64) * 2, 16,
-                                                      1024, kSw128);
-                        mma_bf16_ts(tmem + p.tm_dz, tmem + p.tm_dw + 8 * kk, bd, idesc, kk > 0 ? 1u : 0u);
-                    }
+                if (pend.it >= 0) {
+                    if (!dzdu(pend)) { ok = false; break; }
                 }
-                {
-                    const uint32_t zs = sb + s * p.stage_bytes + 2 * p.xy_tile_bytes;
-                    const uint32_t idesc = idesc_bf16(128, p.R, true, true);
-                    for (int mb = 0; mb < p.SCp / 128; ++mb) {
-                        for (int kk = 0; kk < kTt / 16; ++kk) {
-                            const uint64_t ad = smem_desc(sb + p.off_dw + mb * 2 * 16384 + kk * 2048, 16384, 1024, kSw128);
-                            const uint64_t bd = smem_desc(zs + kk * 256, 128, p.z_slab, kSwNone);
-                            mma_bf16_ss(tmem + p.tm_du + mb * p.R, ad, bd, idesc,
-                                        (seg_first && kk == 0) ? 0u : 1u);
-                        }
-                    }
-                }
+                pend.it = it;
+                pend.s = s;
+                pend.ub = ub;
+                pend.seg_first = seg_first;
+                pend.last_of_slice = (i + 1 == tend) || ((i + 1) / p.per_slice != id.slice);
                 seg_first = false;
-                mma_commit(bar.mm2());
-                const bool last_of_slice = (i + 1 == tend) || ((i + 1) / p.per_slice != id.slice);
-                if (last_of_slice) mma_commit(bar.ue(ub));
             }
+            if (ok && pend.it >= 0) dzdu(pend);
             mma_commit(bar.done());
         }
         __syncwarp();
     } else {
         // ---------------------------------------------------------- epilogue
+        // Per tile i:  A1(i) dx  ->  B(i-1) dz partial, dU flush, stage release  ->  A2(i) dw.
         const int ew = warp - 2;
         const int q = warp & 3;              // TMEM lane quarter == token rows 32q..32q+31
         const int h = ew >> 2;               // channel half of the slice (32 channels)
@@ -309,53 +326,98 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
         const uint32_t dwrow = sb + p.off_dw + (uint32_t)row * 128u;
         const uint32_t dwsw = (uint32_t)(row & 7) << 4;
         const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
-        int prev = -1, seg = 0, cfirst = 0;
+
+        struct Prev {
+            int it, s, slice, b, t0, seg;
+            bool last_of_slice;
+        } pv = {-1, 0, 0, 0, 0, 0, false};
+        // B: dz partial of a finished tile, its slice segment's dU partial, stage release
+        auto phase_b = [&](const Prev &t) -> bool {
+            if (!warp_wait(bar.mm2(), t.it & 1, abort, 256u, &g_fault_bwd)) return false;
+            tc_fence_after();
+            if (h == 0) {
+                const int tok = t.t0 + row;
+                float *dst = p.dz_part + ((size_t)t.slice * p.B * p.T + (size_t)t.b * p.T + tok) * p.R;
+#pragma unroll 1
+                for (int c0 = 0; c0 < p.R; c0 += 16) {
+                    uint32_t v[16];
+                    tmem_ld<16>(tl + p.tm_dz + c0, v);
+                    tmem_wait_ld_regs(v);
+                    if (tok < p.T) {
+#pragma unroll
+                        for (int m2 = 0; m2 < 4; ++m2)
+                            *reinterpret_cast<uint4 *>(dst + c0 + 4 * m2) =
+                                make_uint4(v[4 * m2], v[4 * m2 + 1], v[4 * m2 + 2], v[4 * m2 + 3]);
+                    }
+                }
+            }
+            if (t.last_of_slice && h < p.SCp / 128) {
+                // lane j' of dU^T M-block h -> natural column g*W + k
+                const int jp = 128 * h + row;
+                const int jn = (jp % p.NGs) * W + jp / p.NGs;
+                float *dst = p.du_part + ((size_t)t.slice * p.maxseg + t.seg) * p.R * p.SC + jn;
+#pragma unroll 1
+                for (int c0 = 0; c0 < p.R; c0 += 16) {
+                    uint32_t v[16];
+                    tmem_ld<16>(tl + p.tm_du + h * p.R + c0, v);     // all lanes: warp-collective
+                    tmem_wait_ld_regs(v);
+                    if (jp < p.SC) {
+#pragma unroll
+                        for (int m2 = 0; m2 < 16; ++m2) dst[(size_t)(c0 + m2) * p.SC] = __uint_as_float(v[m2]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar.empty(t.s));
+            return true;
+        };
+
+        int prev_slice = -1, seg = 0;
+        bool ok = true;
         for (int i = tbeg; i < tend; ++i) {
             const int it = i - tbeg;
             const TileId id = tile_id(p, i);
-            if (id.slice != prev) {
-                prev = id.slice;
-                cfirst = owner_of((long long)id.slice * p.per_slice, p.n_tiles, gridDim.x);
-                seg = (int)blockIdx.x - cfirst;
+            if (id.slice != prev_slice) {
+                prev_slice = id.slice;
+                seg = (int)blockIdx.x - owner_of((long long)id.slice * p.per_slice, p.n_tiles, gridDim.x);
             }
-            const int s = it % kStages, n = it / kStages;
-            if (!warp_wait(bar.full(s), n & 1, abort, 64u, &g_fault_bwd)) break;
-            if (!warp_wait(bar.wfull(), it & 1, abort, 128u, &g_fault_bwd)) break;
+            const int s = it % p.stages, n = it / p.stages;
+            if (!warp_wait(bar.full(s), n & 1, abort, 64u, &g_fault_bwd)) { ok = false; break; }
+            if (!warp_wait(bar.wfull(), it & 1, abort, 128u, &g_fault_bwd)) { ok = false; break; }
             tc_fence_after();
             if (lane == 0) bulk_wait_read<0>();
             __syncwarp();
             const uint32_t st = sb + s * p.stage_bytes;
             const uint32_t dys = st, xs = st + p.xy_tile_bytes;
+            // ---- A1: dx[t,c] = dy[t,c] + sum_k w[t+k,g,k] dy[t+k,c]
 #pragma unroll 1
             for (int cq = 0; cq < 4; ++cq) {
-                const int c8 = 32 * h + 8 * cq;      // first channel of the chunk in the slice
-                const int g8 = c8 / G;               // first filter group of the chunk
+                const int g8 = (32 * h + 8 * cq) / G;      // first filter group of the chunk
                 uint32_t wr[W][NG8];
 #pragma unroll
                 for (int k = 0; k < W; ++k) tmem_ld<NG8>(tl + p.tm_w + k * p.NGp + g8, wr[k]);
-                float dyv[W][8], xv[W][8];
+                uint4 du[W];
 #pragma unroll
-                for (int k = 0; k < W; ++k) {
-                    unpack8(lds128(dys + (dyr[k] ^ ((uint32_t)cq << 4))), dyv[k]);
-                    unpack8(lds128(xs + (xr[k] ^ ((uint32_t)cq << 4))), xv[k]);
-                }
-#pragma unroll
-                for (int k = 0; k < W; ++k)
-#pragma unroll
-                    for (int e = 0; e < NG8; ++e) asm volatile("" : "+r"(wr[k][e]));
+                for (int k = 0; k < W; ++k) du[k] = lds128(dys + (dyr[k] ^ ((uint32_t)cq << 4)));
                 tmem_wait_ld();
 #pragma unroll
                 for (int k = 0; k < W; ++k)
 #pragma unroll
                     for (int e = 0; e < NG8; ++e) asm volatile("" : "+r"(wr[k][e]));
-                // dx[t,c] = dy[t,c] + sum_k w[t+k,g,k] dy[t+k,c]
                 float dx[8];
+                {
+                    float d0[8];
+                    unpack8(du[0], d0);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    float acc = dyv[0][e];
+                    for (int e = 0; e < 8; ++e) dx[e] = fmaf(__uint_as_float(wr[0][e / G]), d0[e], d0[e]);
+                }
 #pragma unroll
-                    for (int k = 0; k < W; ++k) acc = fmaf(__uint_as_float(wr[k][e / G]), dyv[k][e], acc);
-                    dx[e] = acc;
+                for (int k = 1; k < W; ++k) {
+                    float dk[8];
+                    unpack8(du[k], dk);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) dx[e] = fmaf(__uint_as_float(wr[k][e / G]), dk[e], dx[e]);
                 }
                 uint4 o;
                 o.x = pack_bf16x2(dx[0], dx[1]);
@@ -363,27 +425,54 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
                 o.z = pack_bf16x2(dx[4], dx[5]);
                 o.w = pack_bf16x2(dx[6], dx[7]);
                 sts128(dxrow ^ ((uint32_t)cq << 4), o);
-                // dw[t,g,k] = sum_{c in g} dy[t,c] x[t-k,c], stored tap-major (column k*NG + g)
+            }
+            tc_fence_before();
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(bar.wempty());
+                tma_store_3d(&tm_dx, dxstage, id.slice * kDt + 32 * h, id.t0 + 32 * q, id.b);
+                bulk_commit();
+            }
+            // ---- B of the previous tile (its dz / dU MMAs ran during A1)
+            if (pv.it >= 0 && !phase_b(pv)) { ok = false; break; }
+            // ---- A2: dw[t,g,k] = sum_{c in g} dy[t,c] x[t-k,c], tap-major column k*NG + g
+#pragma unroll 1
+            for (int cq = 0; cq < 4; ++cq) {
+                const int g8 = (32 * h + 8 * cq) / G;
+                const uint4 d0 = lds128(dys + (dyr[0] ^ ((uint32_t)cq << 4)));
 #pragma unroll
                 for (int k = 0; k < W; ++k) {
-                    float dw[NG8];
+                    const uint4 xu = lds128(xs + (xr[k] ^ ((uint32_t)cq << 4)));
+                    uint32_t pk[4];
+                    if constexpr (G == 1) {
+                        // one channel per group: dw = dy * x, exact in fp32 and rounded once to
+                        // bf16, which is what the packed bf16 multiply computes
+                        pk[0] = bf16x2_mul(d0.x, xu.x);
+                        pk[1] = bf16x2_mul(d0.y, xu.y);
+                        pk[2] = bf16x2_mul(d0.z, xu.z);
+                        pk[3] = bf16x2_mul(d0.w, xu.w);
+                    } else {
+                        float dv[8], xv[8], dw[NG8];
+                        unpack8(d0, dv);
+                        unpack8(xu, xv);
 #pragma unroll
-                    for (int gl = 0; gl < NG8; ++gl) {
-                        float acc = 0.f;
+                        for (int gl = 0; gl < NG8; ++gl) {
+                            float acc = 0.f;
 #pragma unroll
-                        for (int e = gl * G; e < (gl + 1) * G; ++e) acc = fmaf(dyv[0][e], xv[k][e], acc);
-                        dw[gl] = acc;
+                            for (int e = gl * G; e < (gl + 1) * G; ++e) acc = fmaf(dv[e], xv[e], acc);
+                            dw[gl] = acc;
+                        }
+#pragma unroll
+                        for (int m2 = 0; m2 < NG8 / 2; ++m2) pk[m2] = pack_bf16x2(dw[2 * m2], dw[2 * m2 + 1]);
                     }
                     const int jp = k * p.NGs + g8;                    // first tap-major column
                     const uint32_t atom = (uint32_t)(jp >> 6), within = (uint32_t)(jp & 63);
                     const uint32_t a = dwrow + atom * 16384u + ((((within >> 3) << 4) ^ dwsw) | ((within & 7) * 2));
-                    uint32_t pk[NG8 / 2 > 0 ? NG8 / 2 : 1];
-#pragma unroll
-                    for (int m2 = 0; m2 < NG8 / 2; ++m2) pk[m2] = pack_bf16x2(dw[2 * m2], dw[2 * m2 + 1]);
-                    if (NG8 == 8) {
+                    if constexpr (NG8 == 8) {
                         sts128(a, make_uint4(pk[0], pk[1], pk[2], pk[3]));
                         tmem_st_n<4>(tl + p.tm_dw + jp / 2, pk);
-                    } else if (NG8 == 4) {
+                    } else if constexpr (NG8 == 4) {
                         sts64(a, pk[0], pk[1]);
                         tmem_st_n<2>(tl + p.tm_dw + jp / 2, pk);
                     } else {
@@ -396,54 +485,16 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             tc_fence_before();
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(bar.wempty());
-                mbar_arrive(bar.dwready());
-                tma_store_3d(&tm_dx, dxstage, id.slice * kDt + 32 * h, id.t0 + 32 * q, id.b);
-                bulk_commit();
-            }
-            // dz partial of this slice, once the dz/dU MMAs are done
-            if (!warp_wait(bar.mm2(), it & 1, abort, 256u, &g_fault_bwd)) break;
-            tc_fence_after();
-            if (h == 0) {
-                const int t = id.t0 + row;
-                float *dst = p.dz_part + ((size_t)id.slice * p.B * p.T + (size_t)id.b * p.T + t) * p.R;
-#pragma unroll 1
-                for (int c0 = 0; c0 < p.R; c0 += 16) {
-                    uint32_t v[16];
-                    tmem_ld<16>(tl + p.tm_dz + c0, v);
-                    tmem_wait_ld_regs(v);
-                    if (t < p.T) {
-#pragma unroll
-                        for (int m2 = 0; m2 < 4; ++m2)
-                            *reinterpret_cast<uint4 *>(dst + c0 + 4 * m2) =
-                                make_uint4(v[4 * m2], v[4 * m2 + 1], v[4 * m2 + 2], v[4 * m2 + 3]);
-                    }
-                }
-            }
-            const bool last_of_slice = (i + 1 == tend) || ((i + 1) / p.per_slice != id.slice);
-            if (last_of_slice) {
-                // dU^T partial of this CTA's segment of the slice: lane j' of M-block h
-                if (h < p.SCp / 128) {
-                    const int jp = 128 * h + row;
-                    const int jn = (jp % p.NGs) * W + jp / p.NGs;        // natural column g*W + k
-                    float *dst = p.du_part + ((size_t)id.slice * p.maxseg + seg) * p.R * p.SC + jn;
-#pragma unroll 1
-                    for (int c0 = 0; c0 < p.R; c0 += 16) {
-                        uint32_t v[16];
-                        tmem_ld<16>(tl + p.tm_du + h * p.R + c0, v);     // all lanes: warp-collective
-                        tmem_wait_ld_regs(v);
-                        if (jp < p.SC) {
-#pragma unroll
-                            for (int m2 = 0; m2 < 16; ++m2) dst[(size_t)(c0 + m2) * p.SC] = __uint_as_float(v[m2]);
-                        }
-                    }
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar.empty(s));
+            if (lane == 0) mbar_arrive(bar.dwready());
+            pv.it = it;
+            pv.s = s;
+            pv.slice = id.slice;
+            pv.b = id.b;
+            pv.t0 = id.t0;
+            pv.seg = seg;
+            pv.last_of_slice = (i + 1 == tend) || ((i + 1) / p.per_slice != id.slice);
         }
+        if (ok && pv.it >= 0) phase_b(pv);
         if (lane == 0) bulk_wait_all();
         __syncwarp();
     }
@@ -583,10 +634,12 @@ bool plan_bwd(int B, int T, int D, int G, int W, int R, int grid, BwdParams &p) 
     p.z_bytes = (uint32_t)(R / 8) * p.z_slab;
     p.stage_bytes = (2 * p.xy_tile_bytes + p.z_bytes + 1023) / 1024 * 1024;
     p.u_bytes = (uint32_t)(p.u_boxes * R * 128);
-    for (int nU = 2; nU >= 1; --nU) {
-        p.nU = nU;
-        p.off_u = kStages * p.stage_bytes;
-        p.off_dw = p.off_u + nU * p.u_bytes;
+    const int options[4][2] = {{3, 2}, {3, 1}, {2, 2}, {2, 1}};   // (stages, U buffers)
+    for (auto &o : options) {
+        p.stages = o[0];
+        p.nU = o[1];
+        p.off_u = p.stages * p.stage_bytes;
+        p.off_dw = p.off_u + p.nU * p.u_bytes;
         p.off_dw = (p.off_dw + 1023) / 1024 * 1024;
         p.off_dx = p.off_dw + (uint32_t)(p.SCp / 64) * 16384u;
         p.off_bar = p.off_dx + kEpiWarps * 2048;

@@ -76,7 +76,9 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     while (true) {
-        if (mbar_try_wait(bar, parity)) return true;
+#pragma unroll 1
+        for (int i = 0; i < 32; ++i)
+            if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
         if (globaltimer() - t0 > kWaitLimitNs) {
             *abort = 1;
@@ -260,6 +262,13 @@ template <> __device__ __forceinline__ void tmem_ld<32>(uint32_t a, uint32_t *r)
 template <> __device__ __forceinline__ void tmem_ld<64>(uint32_t a, uint32_t *r) {
     tmem_ld<32>(a, r);
     tmem_ld<32>(a + 32, r + 32);
+}
+
+// Packed bf16 pair product, rounded to nearest even.
+__device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
 }
 
 // Packed fp32 pair arithmetic (sm_100): d = a * b + c on both halves.
