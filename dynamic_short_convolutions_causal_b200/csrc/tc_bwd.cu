@@ -41,7 +41,9 @@ __device__ unsigned int g_fault_bwd = 0;
 
 constexpr int kTt = 128;
 constexpr int kDt = 64;
-constexpr int kEpiWarps = 8;
+constexpr int kEpiWarps = 16;           // 4 lane quarters x 4 channel groups of 16
+constexpr int kCPW = 16;                // channels per epilogue warp
+constexpr int kDxBuf = 32 * kCPW * 2;   // one warp's dx staging: 32 rows x 16 bf16
 constexpr int kThreads = 32 * (2 + kEpiWarps);
 
 struct BwdParams {
@@ -254,9 +256,13 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
                 const uint32_t idz = idesc_bf16(128, p.R, false, false);
                 for (int kk = 0; kk < p.SC / 16; ++kk) {
                     const int j0 = 16 * kk;
+                    // A = dw [128 tokens x SC], the same shared-memory tile as dU^T's A operand,
+                    // read K-major (rows = tokens); B = Up slice, K-major (rows = r)
+                    const uint64_t ad =
+                        smem_desc(sb + p.off_dw + (j0 / 64) * 16384u + (j0 % 64) * 2, 16, 1024, kSw128);
                     const uint64_t bd =
                         smem_desc(us + (j0 / 64) * (uint32_t)(p.R * 128) + (j0 % 64) * 2, 16, 1024, kSw128);
-                    mma_bf16_ts(tmem + p.tm_dz, tmem + p.tm_dw + 8 * kk, bd, idz, kk > 0 ? 1u : 0u);
+                    mma_bf16_ss(tmem + p.tm_dz, ad, bd, idz, kk > 0 ? 1u : 0u);
                 }
                 const uint32_t zs = sb + t.s * p.stage_bytes + 2 * p.xy_tile_bytes;
                 const uint32_t idu = idesc_bf16(128, p.R, true, true);
@@ -309,18 +315,19 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
         // Per tile i:  A1(i) dx  ->  B(i-1) dz partial, dU flush, stage release  ->  A2(i) dw.
         const int ew = warp - 2;
         const int q = warp & 3;              // TMEM lane quarter == token rows 32q..32q+31
-        const int h = ew >> 2;               // channel half of the slice (32 channels)
+        const int h = ew >> 2;               // channel group of the slice (16 channels)
         const int row = 32 * q + lane;
-        const uint32_t dxstage = sb + p.off_dx + (uint32_t)ew * 2048;
-        const uint32_t dxrow = (dxstage + lane * 64) ^ ((uint32_t)((lane >> 1) & 3) << 4);
+        const uint32_t dxstage = sb + p.off_dx + (uint32_t)ew * kDxBuf;
+        // 32-byte staging rows in the TMA store's 32-byte swizzle (16-byte chunk ^ (lane/4)%2)
+        const uint32_t dxrow = (dxstage + lane * 32) ^ ((uint32_t)((lane >> 2) & 1) << 4);
         // dy rows r = row + k and x rows r = row + W-1-k of the 128-byte-swizzled tiles
         uint32_t dyr[W], xr[W];
 #pragma unroll
         for (int k = 0; k < W; ++k) {
             uint32_t r = (uint32_t)(row + k);
-            dyr[k] = (r * 128u) ^ ((r & 7u) << 4) ^ ((uint32_t)(4 * h) << 4);
+            dyr[k] = (r * 128u) ^ ((r & 7u) << 4) ^ ((uint32_t)(2 * h) << 4);
             r = (uint32_t)(row + (W - 1) - k);
-            xr[k] = (r * 128u) ^ ((r & 7u) << 4) ^ ((uint32_t)(4 * h) << 4);
+            xr[k] = (r * 128u) ^ ((r & 7u) << 4) ^ ((uint32_t)(2 * h) << 4);
         }
         // dw^T shared-memory tile: MN-major, 128B swizzle, atoms of 64 columns x 128 rows
         const uint32_t dwrow = sb + p.off_dw + (uint32_t)row * 128u;
@@ -335,20 +342,17 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
         auto phase_b = [&](const Prev &t) -> bool {
             if (!warp_wait(bar.mm2(), t.it & 1, abort, 256u, &g_fault_bwd)) return false;
             tc_fence_after();
-            if (h == 0) {
+            {
+                // dz partial: every warp reads R/4 of the columns of its 32 rows
                 const int tok = t.t0 + row;
-                float *dst = p.dz_part + ((size_t)t.slice * p.B * p.T + (size_t)t.b * p.T + tok) * p.R;
+                const int nc = p.R / 4;
+                float *dst = p.dz_part + ((size_t)t.slice * p.B * p.T + (size_t)t.b * p.T + tok) * p.R + h * nc;
 #pragma unroll 1
-                for (int c0 = 0; c0 < p.R; c0 += 16) {
-                    uint32_t v[16];
-                    tmem_ld<16>(tl + p.tm_dz + c0, v);
+                for (int c0 = 0; c0 < nc; c0 += 4) {
+                    uint32_t v[4];
+                    tmem_ld<4>(tl + p.tm_dz + h * nc + c0, v);
                     tmem_wait_ld_regs(v);
-                    if (tok < p.T) {
-#pragma unroll
-                        for (int m2 = 0; m2 < 4; ++m2)
-                            *reinterpret_cast<uint4 *>(dst + c0 + 4 * m2) =
-                                make_uint4(v[4 * m2], v[4 * m2 + 1], v[4 * m2 + 2], v[4 * m2 + 3]);
-                    }
+                    if (tok < p.T) *reinterpret_cast<uint4 *>(dst + c0) = make_uint4(v[0], v[1], v[2], v[3]);
                 }
             }
             if (t.last_of_slice && h < p.SCp / 128) {
@@ -391,97 +395,109 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             const uint32_t st = sb + s * p.stage_bytes;
             const uint32_t dys = st, xs = st + p.xy_tile_bytes;
             // ---- A1: dx[t,c] = dy[t,c] + sum_k w[t+k,g,k] dy[t+k,c]
-#pragma unroll 1
-            for (int cq = 0; cq < 4; ++cq) {
-                const int g8 = (32 * h + 8 * cq) / G;      // first filter group of the chunk
-                uint32_t wr[W][NG8];
+            // All shared-memory loads of the phase are issued before its first store (the
+            // stores are ordered asm statements and would otherwise serialise the loads).
+            constexpr int CH = kCPW / 8;
+            {
+                uint4 du[CH][W];
 #pragma unroll
-                for (int k = 0; k < W; ++k) tmem_ld<NG8>(tl + p.tm_w + k * p.NGp + g8, wr[k]);
-                uint4 du[W];
+                for (int cq = 0; cq < CH; ++cq)
 #pragma unroll
-                for (int k = 0; k < W; ++k) du[k] = lds128(dys + (dyr[k] ^ ((uint32_t)cq << 4)));
+                    for (int k = 0; k < W; ++k) du[cq][k] = lds128(dys + (dyr[k] ^ ((uint32_t)cq << 4)));
+                uint4 dxo[CH];
+                constexpr int NGW = kCPW / G;                  // filter groups of the warp's channels
+                uint32_t wr[W][NGW];
+#pragma unroll
+                for (int k = 0; k < W; ++k) tmem_ld<NGW>(tl + p.tm_w + k * p.NGp + (kCPW * h) / G, wr[k]);
                 tmem_wait_ld();
 #pragma unroll
                 for (int k = 0; k < W; ++k)
 #pragma unroll
-                    for (int e = 0; e < NG8; ++e) asm volatile("" : "+r"(wr[k][e]));
-                float dx[8];
-                {
-                    float d0[8];
-                    unpack8(du[0], d0);
+                    for (int e = 0; e < NGW; ++e) asm volatile("" : "+r"(wr[k][e]));
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) dx[e] = fmaf(__uint_as_float(wr[0][e / G]), d0[e], d0[e]);
+                for (int cq = 0; cq < CH; ++cq) {
+                    const int gq = (8 * cq) / G;                   // chunk's first group within the warp's
+                    float dx[8];
+                    {
+                        float d0[8];
+                        unpack8(du[cq][0], d0);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) dx[e] = fmaf(__uint_as_float(wr[0][gq + e / G]), d0[e], d0[e]);
+                    }
+#pragma unroll
+                    for (int k = 1; k < W; ++k) {
+                        float dk[8];
+                        unpack8(du[cq][k], dk);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) dx[e] = fmaf(__uint_as_float(wr[k][gq + e / G]), dk[e], dx[e]);
+                    }
+                    dxo[cq].x = pack_bf16x2(dx[0], dx[1]);
+                    dxo[cq].y = pack_bf16x2(dx[2], dx[3]);
+                    dxo[cq].z = pack_bf16x2(dx[4], dx[5]);
+                    dxo[cq].w = pack_bf16x2(dx[6], dx[7]);
                 }
 #pragma unroll
-                for (int k = 1; k < W; ++k) {
-                    float dk[8];
-                    unpack8(du[k], dk);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) dx[e] = fmaf(__uint_as_float(wr[k][e / G]), dk[e], dx[e]);
-                }
-                uint4 o;
-                o.x = pack_bf16x2(dx[0], dx[1]);
-                o.y = pack_bf16x2(dx[2], dx[3]);
-                o.z = pack_bf16x2(dx[4], dx[5]);
-                o.w = pack_bf16x2(dx[6], dx[7]);
-                sts128(dxrow ^ ((uint32_t)cq << 4), o);
+                for (int cq = 0; cq < CH; ++cq) sts128(dxrow ^ ((uint32_t)cq << 4), dxo[cq]);
             }
             tc_fence_before();
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(bar.wempty());
-                tma_store_3d(&tm_dx, dxstage, id.slice * kDt + 32 * h, id.t0 + 32 * q, id.b);
+                tma_store_3d(&tm_dx, dxstage, id.slice * kDt + kCPW * h, id.t0 + 32 * q, id.b);
                 bulk_commit();
             }
             // ---- B of the previous tile (its dz / dU MMAs ran during A1)
             if (pv.it >= 0 && !phase_b(pv)) { ok = false; break; }
             // ---- A2: dw[t,g,k] = sum_{c in g} dy[t,c] x[t-k,c], tap-major column k*NG + g
-#pragma unroll 1
-            for (int cq = 0; cq < 4; ++cq) {
-                const int g8 = (32 * h + 8 * cq) / G;
-                const uint4 d0 = lds128(dys + (dyr[0] ^ ((uint32_t)cq << 4)));
+            {
+                uint4 d0[CH], xu[CH][W];
 #pragma unroll
-                for (int k = 0; k < W; ++k) {
-                    const uint4 xu = lds128(xs + (xr[k] ^ ((uint32_t)cq << 4)));
-                    uint32_t pk[4];
-                    if constexpr (G == 1) {
-                        // one channel per group: dw = dy * x, exact in fp32 and rounded once to
-                        // bf16, which is what the packed bf16 multiply computes
-                        pk[0] = bf16x2_mul(d0.x, xu.x);
-                        pk[1] = bf16x2_mul(d0.y, xu.y);
-                        pk[2] = bf16x2_mul(d0.z, xu.z);
-                        pk[3] = bf16x2_mul(d0.w, xu.w);
-                    } else {
-                        float dv[8], xv[8], dw[NG8];
-                        unpack8(d0, dv);
-                        unpack8(xu, xv);
+                for (int cq = 0; cq < CH; ++cq) {
+                    d0[cq] = lds128(dys + (dyr[0] ^ ((uint32_t)cq << 4)));
 #pragma unroll
-                        for (int gl = 0; gl < NG8; ++gl) {
-                            float acc = 0.f;
+                    for (int k = 0; k < W; ++k) xu[cq][k] = lds128(xs + (xr[k] ^ ((uint32_t)cq << 4)));
+                }
 #pragma unroll
-                            for (int e = gl * G; e < (gl + 1) * G; ++e) acc = fmaf(dv[e], xv[e], acc);
-                            dw[gl] = acc;
+                for (int cq = 0; cq < CH; ++cq) {
+                    const int g8 = (kCPW * h + 8 * cq) / G;
+#pragma unroll
+                    for (int k = 0; k < W; ++k) {
+                        uint32_t pk[4];
+                        if constexpr (G == 1) {
+                            // one channel per group: dw = dy * x, exact in fp32 and rounded once
+                            // to bf16, which is what the packed bf16 multiply computes
+                            pk[0] = bf16x2_mul(d0[cq].x, xu[cq][k].x);
+                            pk[1] = bf16x2_mul(d0[cq].y, xu[cq][k].y);
+                            pk[2] = bf16x2_mul(d0[cq].z, xu[cq][k].z);
+                            pk[3] = bf16x2_mul(d0[cq].w, xu[cq][k].w);
+                        } else {
+                            float dv[8], xv[8], dw[NG8];
+                            unpack8(d0[cq], dv);
+                            unpack8(xu[cq][k], xv);
+#pragma unroll
+                            for (int gl = 0; gl < NG8; ++gl) {
+                                float acc = 0.f;
+#pragma unroll
+                                for (int e = gl * G; e < (gl + 1) * G; ++e) acc = fmaf(dv[e], xv[e], acc);
+                                dw[gl] = acc;
+                            }
+#pragma unroll
+                            for (int m2 = 0; m2 < NG8 / 2; ++m2) pk[m2] = pack_bf16x2(dw[2 * m2], dw[2 * m2 + 1]);
                         }
-#pragma unroll
-                        for (int m2 = 0; m2 < NG8 / 2; ++m2) pk[m2] = pack_bf16x2(dw[2 * m2], dw[2 * m2 + 1]);
-                    }
-                    const int jp = k * p.NGs + g8;                    // first tap-major column
-                    const uint32_t atom = (uint32_t)(jp >> 6), within = (uint32_t)(jp & 63);
-                    const uint32_t a = dwrow + atom * 16384u + ((((within >> 3) << 4) ^ dwsw) | ((within & 7) * 2));
-                    if constexpr (NG8 == 8) {
-                        sts128(a, make_uint4(pk[0], pk[1], pk[2], pk[3]));
-                        tmem_st_n<4>(tl + p.tm_dw + jp / 2, pk);
-                    } else if constexpr (NG8 == 4) {
-                        sts64(a, pk[0], pk[1]);
-                        tmem_st_n<2>(tl + p.tm_dw + jp / 2, pk);
-                    } else {
-                        sts32(a, pk[0]);
-                        tmem_st_n<1>(tl + p.tm_dw + jp / 2, pk);
+                        const int jp = k * p.NGs + g8;                    // first tap-major column
+                        const uint32_t atom = (uint32_t)(jp >> 6), within = (uint32_t)(jp & 63);
+                        const uint32_t a = dwrow + atom * 16384u + ((((within >> 3) << 4) ^ dwsw) | ((within & 7) * 2));
+                        if constexpr (NG8 == 8) {
+                            sts128(a, make_uint4(pk[0], pk[1], pk[2], pk[3]));
+                        } else if constexpr (NG8 == 4) {
+                            sts64(a, pk[0], pk[1]);
+                        } else {
+                            sts32(a, pk[0]);
+                        }
                     }
                 }
             }
-            tmem_wait_st();
             tc_fence_before();
             fence_proxy_async_smem();
             __syncwarp();
@@ -619,10 +635,10 @@ bool plan_bwd(int B, int T, int D, int G, int W, int R, int grid, BwdParams &p) 
     }
     p.maxseg = maxseg;
     p.u_boxes = (p.SC + 63) / 64;
-    // TMEM: w (W tap blocks) | dw (bf16 pairs) | dz | dU^T
+    // TMEM: w (W tap blocks) | dz | dU^T
     p.tm_w = 0;
-    p.tm_dw = (uint32_t)(W * p.NGp + 31) / 32 * 32;
-    p.tm_dz = p.tm_dw + (uint32_t)(p.SC / 2 + 31) / 32 * 32;
+    p.tm_dw = 0;   // unused: dw lives in shared memory only
+    p.tm_dz = (uint32_t)(W * p.NGp + 31) / 32 * 32;
     p.tm_du = p.tm_dz + (uint32_t)R;
     const uint32_t used = p.tm_du + (uint32_t)(p.SCp / 128) * R;
     if (used > 512) return false;
@@ -642,7 +658,7 @@ bool plan_bwd(int B, int T, int D, int G, int W, int R, int grid, BwdParams &p) 
         p.off_dw = p.off_u + p.nU * p.u_bytes;
         p.off_dw = (p.off_dw + 1023) / 1024 * 1024;
         p.off_dx = p.off_dw + (uint32_t)(p.SCp / 64) * 16384u;
-        p.off_bar = p.off_dx + kEpiWarps * 2048;
+        p.off_bar = p.off_dx + kEpiWarps * kDxBuf;
         if (p.off_bar + kBarBytes + 16 + 1024 <= kSmemLimit) return true;
     }
     return false;
@@ -717,12 +733,12 @@ cudaError_t launch_tc_lowrank_bwd(const void *x, const void *z, const void *U, c
     const uint32_t bz[3] = {8, p.rows, 1};
     const uint64_t du[2] = {(uint64_t)N, (uint64_t)R};
     const uint32_t bu[2] = {64, (uint32_t)R};
-    const uint32_t bdx[3] = {32, 32, 1};
+    const uint32_t bdx[3] = {(uint32_t)kCPW, 32, 1};
     if (!make_map(&m[0], dy, 3, dxyz, bxy, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) ||
         !make_map(&m[1], x, 3, dxyz, bxy, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) ||
         !make_map(&m[2], z, 3, dzz, bz, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
         !make_map(&m[3], Up, 2, du, bu, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
-        !make_map(&m[4], dx, 3, dxyz, bdx, CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B)) {
+        !make_map(&m[4], dx, 3, dxyz, bdx, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B)) {
         set_last_error("dsc_bwd_lowrank: cuTensorMapEncodeTiled failed");
         return cudaErrorInvalidValue;
     }
