@@ -130,12 +130,8 @@ def barrier(world):
 
 
 def max_over_ranks(v, world, device):
-    if world == 1:
-        return v
-    import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device=device)
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    from dynamic_short_convolutions_causal_b200 import dp
+    return dp.max_over_ranks(v, device) if world > 1 else v
 
 
 # ------------------------------------------------------------------ CPU oracle baseline
@@ -204,8 +200,7 @@ def run_ours(args, wl, world, rank, local):
     ws = dsc.workspace(dsc.dsc_bwd_lowrank_workspace_bytes(wl.B, wl.T, wl.D, G, W, R, x.dtype), dev)
     path = dsc.dsc_lowrank_path(wl.B, wl.T, wl.D, G, W, R, x.dtype)
     stream = torch.cuda.current_stream(dev)
-    if world > 1:
-        import torch.distributed as dist
+    from dynamic_short_convolutions_causal_b200 import dp
 
     def step(ev=None):
         if ev is not None:
@@ -217,7 +212,7 @@ def run_ours(args, wl, world, rank, local):
         if ev is not None:
             ev[2].record(stream)
         if world > 1:
-            dist.all_reduce(dU)
+            dp.allreduce_weight_grad(dU)
 
     for _ in range(args.warmup):
         step()
@@ -317,8 +312,7 @@ def measure_e2e(dsc, t, y, dx, dz, dU, ws, wl, world, dev, args):
     stream = torch.cuda.current_stream(dev)
     h2d = sum(a.numel() * a.element_size() for a in (hx, hz, hU, hdy))
     d2h = sum(a.numel() * a.element_size() for a in (hy, hdx, hdz, hdU))
-    if world > 1:
-        import torch.distributed as dist
+    from dynamic_short_convolutions_causal_b200 import dp
 
     def step():
         x.copy_(hx, non_blocking=True)
@@ -328,7 +322,7 @@ def measure_e2e(dsc, t, y, dx, dz, dU, ws, wl, world, dev, args):
         dsc.dsc_fwd_lowrank(x, z, U, y, G, W)
         dsc.dsc_bwd_lowrank(x, z, U, dy, dx, dz, dU, ws, G, W)
         if world > 1:
-            dist.all_reduce(dU)
+            dp.allreduce_weight_grad(dU)
         hy.copy_(y, non_blocking=True)
         hdx.copy_(dx, non_blocking=True)
         hdz.copy_(dz, non_blocking=True)
