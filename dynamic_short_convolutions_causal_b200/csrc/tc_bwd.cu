@@ -233,19 +233,29 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             } pend = {-1, 0, 0, false, false};
             bool seg_first = true;
             bool ok = true;
+            // descriptor templates (fixed fields); per MMA only the start address changes
+            const uint64_t t_zk = desc_tmpl(p.z_slab, 128, kSwNone);              // z, K-major, no swizzle
+            const uint64_t t_u_mn = desc_tmpl((uint32_t)(p.R * 128), 1024, kSw128); // Up as MN-major B
+            const uint64_t t_k128 = desc_tmpl(16, 1024, kSw128);                    // K-major, 128B swizzle
+            const uint64_t t_dwt = desc_tmpl(16384, 1024, kSw128);                  // dw^T, MN-major A
+            const uint64_t t_zmn = desc_tmpl(128, p.z_slab, kSwNone);              // z, MN-major B
+            const uint32_t i_rec = idesc_bf16(128, p.NGp, false, true);
+            const uint32_t i_dz = idesc_bf16(128, p.R, false, false);
+            const uint32_t i_du = idesc_bf16(128, p.R, true, true);
+            const int ksr = p.R / 16, ksc = p.SC / 16, nmb = p.SCp / 128;
+            const uint32_t ubox = (uint32_t)(p.R * 128);
             auto recompute = [&](int it, int ubuf) {
                 const int s = it % p.stages;
                 const uint32_t zs = sb + s * p.stage_bytes + 2 * p.xy_tile_bytes;
                 const uint32_t us = sb + p.off_u + ubuf * p.u_bytes;
-                const uint32_t idesc = idesc_bf16(128, p.NGp, false, true);
+#pragma unroll
                 for (int k = 0; k < W; ++k) {
-                    const int col0 = k * p.NGs;
-                    const uint32_t ub0 = us + (col0 / 64) * (uint32_t)(p.R * 128) + (col0 % 64) * 2;
-                    for (int kk = 0; kk < p.R / 16; ++kk) {
-                        const uint64_t ad = smem_desc(zs + 16 * k + kk * 2 * p.z_slab, p.z_slab, 128, kSwNone);
-                        const uint64_t bd = smem_desc(ub0 + kk * 2048, (uint32_t)(p.R * 128), 1024, kSw128);
-                        mma_bf16_ss(tmem + p.tm_w + k * p.NGp, ad, bd, idesc, kk > 0 ? 1u : 0u);
-                    }
+                    const int col0 = k * (kDt / G);
+                    const uint32_t ub0 = us + (col0 / 64) * ubox + (col0 % 64) * 2;
+                    const uint32_t d = tmem + p.tm_w + k * p.NGp;
+                    for (int kk = 0; kk < ksr; ++kk)
+                        mma_bf16_ss(d, desc_at(t_zk, zs + 16 * k + kk * 2 * p.z_slab), desc_at(t_u_mn, ub0 + kk * 2048),
+                                    i_rec, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(bar.wfull());
             };
@@ -253,26 +263,25 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
                 if (!mbar_wait(bar.dwready(), t.it & 1, abort, 32u, &g_fault_bwd)) return false;
                 tc_fence_after();
                 const uint32_t us = sb + p.off_u + t.ub * p.u_bytes;
-                const uint32_t idz = idesc_bf16(128, p.R, false, false);
-                for (int kk = 0; kk < p.SC / 16; ++kk) {
-                    const int j0 = 16 * kk;
-                    // A = dw [128 tokens x SC], the same shared-memory tile as dU^T's A operand,
-                    // read K-major (rows = tokens); B = Up slice, K-major (rows = r)
-                    const uint64_t ad =
-                        smem_desc(sb + p.off_dw + (j0 / 64) * 16384u + (j0 % 64) * 2, 16, 1024, kSw128);
-                    const uint64_t bd =
-                        smem_desc(us + (j0 / 64) * (uint32_t)(p.R * 128) + (j0 % 64) * 2, 16, 1024, kSw128);
-                    mma_bf16_ss(tmem + p.tm_dz, ad, bd, idz, kk > 0 ? 1u : 0u);
+                const uint32_t dw0 = sb + p.off_dw;
+                // dz = dw Up^T: A = dw tile (K-major view), B = Up slice (K-major), 16 columns per step
+                uint32_t a_off = 0, b_off = 0;
+                for (int kk = 0; kk < ksc; ++kk) {
+                    mma_bf16_ss(tmem + p.tm_dz, desc_at(t_k128, dw0 + a_off), desc_at(t_k128, us + b_off), i_dz,
+                                kk > 0 ? 1u : 0u);
+                    // next 16 columns: +32 bytes within a 64-column atom, next atom every 4 steps
+                    const bool wrap = (kk & 3) == 3;
+                    a_off += wrap ? (16384u - 96u) : 32u;
+                    b_off += wrap ? (ubox - 96u) : 32u;
                 }
+                // dU^T += dw^T z: A = dw^T (MN-major), B = z tile rows 0..127 (MN-major)
                 const uint32_t zs = sb + t.s * p.stage_bytes + 2 * p.xy_tile_bytes;
-                const uint32_t idu = idesc_bf16(128, p.R, true, true);
-                for (int mb = 0; mb < p.SCp / 128; ++mb)
-                    for (int kk = 0; kk < kTt / 16; ++kk) {
-                        const uint64_t ad =
-                            smem_desc(sb + p.off_dw + mb * 2 * 16384 + kk * 2048, 16384, 1024, kSw128);
-                        const uint64_t bd = smem_desc(zs + kk * 256, 128, p.z_slab, kSwNone);
-                        mma_bf16_ss(tmem + p.tm_du + mb * p.R, ad, bd, idu, (t.seg_first && kk == 0) ? 0u : 1u);
-                    }
+                for (int mb = 0; mb < nmb; ++mb) {
+                    const uint32_t d = tmem + p.tm_du + mb * p.R;
+                    for (int kk = 0; kk < kTt / 16; ++kk)
+                        mma_bf16_ss(d, desc_at(t_dwt, dw0 + mb * 32768u + kk * 2048u), desc_at(t_zmn, zs + kk * 256u),
+                                    i_du, (t.seg_first && kk == 0) ? 0u : 1u);
+                }
                 mma_commit(bar.mm2());
                 if (t.last_of_slice) mma_commit(bar.ue(t.ub));
                 return true;

@@ -317,6 +317,16 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint
     return d;
 }
 
+// Descriptor with start address 0 (the fixed fields), and the same descriptor at a
+// shared-memory address: the start address is the only per-MMA field, so issuing
+// loops precompute the template once and OR in (address >> 4) per instruction.
+__device__ __forceinline__ uint64_t desc_tmpl(uint32_t lbo, uint32_t sbo, uint32_t layout) {
+    return smem_desc(0, lbo, sbo, layout);
+}
+__device__ __forceinline__ uint64_t desc_at(uint64_t tmpl, uint32_t saddr) {
+    return tmpl | (uint64_t)((saddr >> 4) & 0x3FFFu);
+}
+
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.
 //   [4,6) D format (1 = f32), [7,10) A format (1 = bf16), [10,13) B format (1 = bf16),
 //   [15] A major (0 = K, 1 = MN), [16] B major, [17,23) N >> 3, [24,29) M >> 4.

@@ -215,7 +215,13 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
             const int nchunks = (p.n_pad + 255) / 256;
-            const uint32_t zsbo = 8u * p.R * 2u;
+            const uint32_t ubox = (uint32_t)(p.R * 128);
+            const int ksteps = p.R / 16;
+            // descriptor templates: only the start address changes per MMA
+            const uint64_t t_z = desc_tmpl(16, 8u * p.R * 2u, p.z_layout);   // z tile, K-major
+            const uint64_t t_u = desc_tmpl(ubox, 1024, kSw128);              // U slice, MN-major
+            const uint32_t i_full = idesc_bf16(128, 256, false, true);
+            const uint32_t i_last = idesc_bf16(128, p.n_pad - 256 * (nchunks - 1), false, true);
             int it = 0;
             for (int i = blockIdx.x; i < p.n_tiles; i += gridDim.x, ++it) {
                 const int s = it % S, n = it / S;
@@ -227,14 +233,10 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
                 const uint32_t za = sb + s * p.stage_bytes + p.off_z;
                 const uint32_t ua = sb + s * p.stage_bytes + p.off_u;
                 for (int nc = 0; nc < nchunks; ++nc) {
-                    const int ncols = min(256, p.n_pad - 256 * nc);
-                    const uint32_t idesc = idesc_bf16(128, ncols, false, true);
-                    for (int kk = 0; kk < p.R / 16; ++kk) {
-                        const uint64_t ad = smem_desc(za + kk * 32, 16, zsbo, p.z_layout);
-                        const uint64_t bd = smem_desc(ua + nc * 4 * (uint32_t)(p.R * 128) + kk * 2048,
-                                                      (uint32_t)(p.R * 128), 1024, kSw128);
-                        mma_bf16_ss(d + 256 * nc, ad, bd, idesc, kk > 0 ? 1u : 0u);
-                    }
+                    const uint32_t idesc = nc + 1 < nchunks ? i_full : i_last;
+                    for (int kk = 0; kk < ksteps; ++kk)
+                        mma_bf16_ss(d + 256 * nc, desc_at(t_z, za + kk * 32),
+                                    desc_at(t_u, ua + nc * 4 * ubox + kk * 2048), idesc, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(bar.accf(a));
             }
