@@ -15,10 +15,11 @@
 //        Wk[t, g] = sum_r z[t0+t+k, r] Up[r, k*NG+g]   (Up: U with the slice's columns
 //      reordered tap-major by a pre-pass), so TMEM lane t holds w[t+k, g, k] for every k;
 //   2. epilogue (one token row per thread): dx and dw on CUDA cores; dx is stored by TMA,
-//      dw (bf16) is written to TMEM and to shared memory;
-//   3. dz partial = dw Up^T   (A = dw in TMEM, B = Up slice, M=128 tokens, N=R);
-//      dU^T     += dw^T z     (A = dw in shared memory, B = z tile, M=128 columns, N=R),
-//      accumulated in TMEM over all tiles of the slice that the CTA processes.
+//      dw (bf16) is written to shared memory;
+//   3. dz partial = dw Up^T   (A = dw tile, B = Up slice, M=128 tokens, N=R);
+//      dU^T     += dw^T z     (A = the same tile read MN-major, B = z tile, M=128 columns,
+//      N=R), accumulated in TMEM over all tiles of the slice that the CTA processes.
+//   Recompute, dz and dU are issued by three MMA warps, each on its own SM sub-partition.
 // Persistent CTAs own contiguous tile ranges in slice-major order.  dz partials (per
 // slice) and dU partials (per CTA segment of a slice) go to the workspace and are summed
 // in a fixed order by two small kernels, so results are deterministic.
@@ -44,7 +45,13 @@ constexpr int kDt = 64;
 constexpr int kEpiWarps = 16;           // 4 lane quarters x 4 channel groups of 16
 constexpr int kCPW = 16;                // channels per epilogue warp
 constexpr int kDxBuf = 32 * kCPW * 2;   // one warp's dx staging: 32 rows x 16 bf16
-constexpr int kThreads = 32 * (2 + kEpiWarps);
+// Warp roles: 0 TMA producer, 1 recompute MMAs, 2..17 epilogue, 18 dz MMAs, 19 dU MMAs.
+// The three MMA streams are issued from warps on three different SM sub-partitions: one
+// warp issuing all of them shares its issue slots with four busy epilogue warps and
+// cannot keep the tensor pipe fed.  Twenty warps keep the 96-register budget of eighteen.
+constexpr int kDzWarp = 2 + kEpiWarps;
+constexpr int kDuWarp = 3 + kEpiWarps;
+constexpr int kThreads = 32 * (4 + kEpiWarps);
 
 struct BwdParams {
     int B, T, D, G, W, R;
@@ -147,13 +154,13 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
         }
         for (int u = 0; u < 2; ++u) {
             mbar_init(bar.uf(u), 1);
-            mbar_init(bar.ue(u), 1);
+            mbar_init(bar.ue(u), 2);        // recompute and dz streams
         }
         mbar_init(bar.wfull(), 1);
         mbar_init(bar.wempty(), kEpiWarps);
         mbar_init(bar.dwready(), kEpiWarps);
-        mbar_init(bar.mm2(), 1);
-        mbar_init(bar.done(), 1);
+        mbar_init(bar.mm2(), 2);            // dz and dU streams
+        mbar_init(bar.done(), 3);           // all three MMA streams
         *abort = 0;
         fence_barrier_init();
     }
@@ -220,106 +227,55 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ---------------------------------------------------------- MMA issuer
-        // Order per tile i: recompute(i) as soon as the epilogue has read w(i-1), then the
-        // dz / dU products of tile i-1 once its dw is written, so that they run while the
-        // epilogue computes dx of tile i.  Across a slice change the pending dz / dU go
-        // first: they release the U buffer the next slice may need.
-        if (lane == 0) {
-            int prev_slice = -1, v = -1, ub = 0;
-            struct Pending {
-                int it, s, ub;
-                bool seg_first, last_of_slice;
-            } pend = {-1, 0, 0, false, false};
-            bool seg_first = true;
-            bool ok = true;
-            // descriptor templates (fixed fields); per MMA only the start address changes
-            const uint64_t t_zk = desc_tmpl(p.z_slab, 128, kSwNone);              // z, K-major, no swizzle
-            const uint64_t t_u_mn = desc_tmpl((uint32_t)(p.R * 128), 1024, kSw128); // Up as MN-major B
-            const uint64_t t_k128 = desc_tmpl(16, 1024, kSw128);                    // K-major, 128B swizzle
-            const uint64_t t_dwt = desc_tmpl(16384, 1024, kSw128);                  // dw^T, MN-major A
-            const uint64_t t_zmn = desc_tmpl(128, p.z_slab, kSwNone);              // z, MN-major B
-            const uint32_t i_rec = idesc_bf16(128, p.NGp, false, true);
-            const uint32_t i_dz = idesc_bf16(128, p.R, false, false);
-            const uint32_t i_du = idesc_bf16(128, p.R, true, true);
-            const int ksr = p.R / 16, ksc = p.SC / 16, nmb = p.SCp / 128;
-            const uint32_t ubox = (uint32_t)(p.R * 128);
-            auto recompute = [&](int it, int ubuf) {
-                const int s = it % p.stages;
-                const uint32_t zs = sb + s * p.stage_bytes + 2 * p.xy_tile_bytes;
-                const uint32_t us = sb + p.off_u + ubuf * p.u_bytes;
-#pragma unroll
-                for (int k = 0; k < W; ++k) {
-                    const int col0 = k * (kDt / G);
-                    const uint32_t ub0 = us + (col0 / 64) * ubox + (col0 % 64) * 2;
-                    const uint32_t d = tmem + p.tm_w + k * p.NGp;
-                    for (int kk = 0; kk < ksr; ++kk)
-                        mma_bf16_ss(d, desc_at(t_zk, zs + 16 * k + kk * 2 * p.z_slab), desc_at(t_u_mn, ub0 + kk * 2048),
-                                    i_rec, kk > 0 ? 1u : 0u);
-                }
-                mma_commit(bar.wfull());
-            };
-            auto dzdu = [&](const Pending &t) -> bool {
-                if (!mbar_wait(bar.dwready(), t.it & 1, abort, 32u, &g_fault_bwd)) return false;
-                tc_fence_after();
-                const uint32_t us = sb + p.off_u + t.ub * p.u_bytes;
-                const uint32_t dw0 = sb + p.off_dw;
-                // dz = dw Up^T: A = dw tile (K-major view), B = Up slice (K-major), 16 columns per step
-                uint32_t a_off = 0, b_off = 0;
-                for (int kk = 0; kk < ksc; ++kk) {
-                    mma_bf16_ss(tmem + p.tm_dz, desc_at(t_k128, dw0 + a_off), desc_at(t_k128, us + b_off), i_dz,
-                                kk > 0 ? 1u : 0u);
-                    // next 16 columns: +32 bytes within a 64-column atom, next atom every 4 steps
-                    const bool wrap = (kk & 3) == 3;
-                    a_off += wrap ? (16384u - 96u) : 32u;
-                    b_off += wrap ? (ubox - 96u) : 32u;
-                }
-                // dU^T += dw^T z: A = dw^T (MN-major), B = z tile rows 0..127 (MN-major)
-                const uint32_t zs = sb + t.s * p.stage_bytes + 2 * p.xy_tile_bytes;
-                for (int mb = 0; mb < nmb; ++mb) {
-                    const uint32_t d = tmem + p.tm_du + mb * p.R;
-                    for (int kk = 0; kk < kTt / 16; ++kk)
-                        mma_bf16_ss(d, desc_at(t_dwt, dw0 + mb * 32768u + kk * 2048u), desc_at(t_zmn, zs + kk * 256u),
-                                    i_du, (t.seg_first && kk == 0) ? 0u : 1u);
-                }
-                mma_commit(bar.mm2());
-                if (t.last_of_slice) mma_commit(bar.ue(t.ub));
-                return true;
-            };
-            for (int i = tbeg; i < tend && ok; ++i) {
-                const int it = i - tbeg;
-                const TileId id = tile_id(p, i);
-                if (id.slice != prev_slice) {
-                    if (pend.it >= 0) {
-                        if (!dzdu(pend)) { ok = false; break; }
-                        pend.it = -1;
-                    }
-                    prev_slice = id.slice;
-                    ++v;
-                    ub = v % p.nU;
-                    seg_first = true;
-                    if (!mbar_wait(bar.uf(ub), (v / p.nU) & 1, abort, 4u, &g_fault_bwd)) { ok = false; break; }
-                }
-                const int s = it % p.stages, n = it / p.stages;
-                if (!mbar_wait(bar.full(s), n & 1, abort, 8u, &g_fault_bwd)) { ok = false; break; }
-                if (!mbar_wait(bar.wempty(), (it & 1) ^ 1, abort, 16u, &g_fault_bwd)) { ok = false; break; }
-                tc_fence_after();
-                recompute(it, ub);
-                if (pend.it >= 0) {
-                    if (!dzdu(pend)) { ok = false; break; }
-                }
-                pend.it = it;
-                pend.s = s;
-                pend.ub = ub;
-                pend.seg_first = seg_first;
-                pend.last_of_slice = (i + 1 == tend) || ((i + 1) / p.per_slice != id.slice);
-                seg_first = false;
+        // ---------------------------------------------------------- MMA issuer: recompute
+        // Each MMA warp runs its schedule warp-uniformly; one elected lane issues each
+        // tcgen05 instruction, and descriptors advance by adding to their start field.
+        // Tile i's filters are recomputed once the epilogue has read those of tile i-1.
+        const uint64_t t_zk = desc_tmpl(p.z_slab, 128, kSwNone);               // z, K-major, no swizzle
+        const uint64_t t_u_mn = desc_tmpl((uint32_t)(p.R * 128), 1024, kSw128);  // Up as MN-major B
+        const uint32_t i_rec = idesc_bf16(128, p.NGp, false, true);
+        const int ksr = p.R / 16;
+        const uint32_t ubox = (uint32_t)(p.R * 128);
+        const uint64_t st_zk = (2 * p.z_slab) >> 4;   // 16 more z columns (start field units)
+        int prev_slice = -1, v = -1, ub = 0;
+        for (int i = tbeg; i < tend; ++i) {
+            const int it = i - tbeg;
+            const TileId id = tile_id(p, i);
+            if (id.slice != prev_slice) {
+                prev_slice = id.slice;
+                ++v;
+                ub = v % p.nU;
+                if (!warp_wait(bar.uf(ub), (v / p.nU) & 1, abort, 4u, &g_fault_bwd)) break;
             }
-            if (ok && pend.it >= 0) dzdu(pend);
-            mma_commit(bar.done());
+            const int s = it % p.stages, n = it / p.stages;
+            if (!warp_wait(bar.full(s), n & 1, abort, 8u, &g_fault_bwd)) break;
+            if (!warp_wait(bar.wempty(), (it & 1) ^ 1, abort, 16u, &g_fault_bwd)) break;
+            tc_fence_after();
+            const uint32_t zs = sb + s * p.stage_bytes + 2 * p.xy_tile_bytes;
+            const uint32_t us = sb + p.off_u + ub * p.u_bytes;
+#pragma unroll
+            for (int k = 0; k < W; ++k) {
+                const int col0 = k * (kDt / G);
+                uint64_t da = desc_at(t_zk, zs + 16 * k);
+                uint64_t db = desc_at(t_u_mn, us + (col0 / 64) * ubox + (col0 % 64) * 2);
+                const uint32_t d = tmem + p.tm_w + k * p.NGp;
+                for (int kk = 0; kk < ksr; ++kk) {
+                    if (elect_one()) mma_bf16_ss(d, da, db, i_rec, kk > 0 ? 1u : 0u);
+                    __syncwarp();
+                    da += st_zk;
+                    db += 2048u >> 4;
+                }
+            }
+            const bool last_of_slice = (i + 1 == tend) || ((i + 1) / p.per_slice != id.slice);
+            if (elect_one()) {
+                mma_commit(bar.wfull());
+                if (last_of_slice) mma_commit(bar.ue(ub));
+            }
+            __syncwarp();
         }
+        if (elect_one()) mma_commit(bar.done());
         __syncwarp();
-    } else {
+    } else if (warp < kDzWarp) {
         // ---------------------------------------------------------- epilogue
         // Per tile i:  A1(i) dx  ->  B(i-1) dz partial, dU flush, stage release  ->  A2(i) dw.
         const int ew = warp - 2;
@@ -521,6 +477,87 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
         }
         if (ok && pv.it >= 0) phase_b(pv);
         if (lane == 0) bulk_wait_all();
+        __syncwarp();
+    } else if (warp == kDzWarp) {
+        // ---------------------------------------------------------- MMA issuer: dz partial
+        // dz = dw Up^T once tile i's dw is written: A = dw tile (K-major view), B = Up slice
+        // (K-major), 16 columns per step (+32 bytes within a 64-column atom, the next atom
+        // every 4 steps).
+        const uint64_t t_k128 = desc_tmpl(16, 1024, kSw128);
+        const uint32_t i_dz = idesc_bf16(128, p.R, false, false);
+        const int ksc = p.SC / 16;
+        const uint32_t ubox = (uint32_t)(p.R * 128);
+        const uint64_t st_wrap_a = (16384u - 96u) >> 4;   // next 64-column dw atom
+        const uint64_t st_wrap_b = (ubox - 96u) >> 4;     // next 64-column Up box
+        const uint32_t dw0 = sb + p.off_dw;
+        int prev_slice = -1, v = -1, ub = 0;
+        for (int i = tbeg; i < tend; ++i) {
+            const int it = i - tbeg;
+            const TileId id = tile_id(p, i);
+            if (id.slice != prev_slice) {
+                prev_slice = id.slice;
+                ++v;
+                ub = v % p.nU;
+                if (!warp_wait(bar.uf(ub), (v / p.nU) & 1, abort, 4u, &g_fault_bwd)) break;
+            }
+            if (!warp_wait(bar.dwready(), it & 1, abort, 32u, &g_fault_bwd)) break;
+            tc_fence_after();
+            const uint32_t us = sb + p.off_u + ub * p.u_bytes;
+            uint64_t da = desc_at(t_k128, dw0), db = desc_at(t_k128, us);
+            for (int kk = 0; kk < ksc; ++kk) {
+                if (elect_one()) mma_bf16_ss(tmem + p.tm_dz, da, db, i_dz, kk > 0 ? 1u : 0u);
+                __syncwarp();
+                const bool wrap = (kk & 3) == 3;
+                da += wrap ? st_wrap_a : 2u;
+                db += wrap ? st_wrap_b : 2u;
+            }
+            const bool last_of_slice = (i + 1 == tend) || ((i + 1) / p.per_slice != id.slice);
+            if (elect_one()) {
+                mma_commit(bar.mm2());
+                if (last_of_slice) mma_commit(bar.ue(ub));
+            }
+            __syncwarp();
+        }
+        if (elect_one()) mma_commit(bar.done());
+        __syncwarp();
+    } else if (warp == kDuWarp) {
+        // ---------------------------------------------------------- MMA issuer: dU partial
+        // dU^T += dw^T z once tile i's dw is written: A = dw^T (MN-major), B = z tile rows
+        // 0..127 (MN-major), 16 tokens per step; the accumulator restarts with each slice
+        // segment of the CTA.
+        const uint64_t t_dwt = desc_tmpl(16384, 1024, kSw128);
+        const uint64_t t_zmn = desc_tmpl(128, p.z_slab, kSwNone);
+        const uint32_t i_du = idesc_bf16(128, p.R, true, true);
+        const int nmb = p.SCp / 128;
+        const uint32_t dw0 = sb + p.off_dw;
+        int prev_slice = -1;
+        bool seg_first = true;
+        for (int i = tbeg; i < tend; ++i) {
+            const int it = i - tbeg;
+            const TileId id = tile_id(p, i);
+            if (id.slice != prev_slice) {
+                prev_slice = id.slice;
+                seg_first = true;
+            }
+            if (!warp_wait(bar.dwready(), it & 1, abort, 32u, &g_fault_bwd)) break;
+            tc_fence_after();
+            const uint32_t zs = sb + (it % p.stages) * p.stage_bytes + 2 * p.xy_tile_bytes;
+            for (int mb = 0; mb < nmb; ++mb) {
+                const uint32_t d = tmem + p.tm_du + mb * p.R;
+                uint64_t da = desc_at(t_dwt, dw0 + mb * 32768u), db = desc_at(t_zmn, zs);
+#pragma unroll
+                for (int kk = 0; kk < kTt / 16; ++kk) {
+                    if (elect_one()) mma_bf16_ss(d, da, db, i_du, (seg_first && kk == 0) ? 0u : 1u);
+                    __syncwarp();
+                    da += 2048u >> 4;
+                    db += 256u >> 4;
+                }
+            }
+            if (elect_one()) mma_commit(bar.mm2());
+            __syncwarp();
+            seg_first = false;
+        }
+        if (elect_one()) mma_commit(bar.done());
         __syncwarp();
     }
 

@@ -41,44 +41,44 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                  : "memory");
 }
 
-// Suspend-time hint (ns) for try_wait; 0 uses the form without a hint.
-#ifndef DSC_WAIT_HINT_NS
-#define DSC_WAIT_HINT_NS 0
-#endif
-
+// mbarrier.try_wait, optionally with a suspend-time hint in ns (0: the form without a
+// hint).  With a hint the waiting thread sleeps until the phase completes or the hint
+// expires instead of polling, which frees issue slots for the warps that do the work.
+template <unsigned HintNs = 0>
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
-#if DSC_WAIT_HINT_NS > 0
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity), "r"((uint32_t)DSC_WAIT_HINT_NS)
-        : "memory");
-#else
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(parity)
-        : "memory");
-#endif
+    if constexpr (HintNs > 0) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity), "r"(HintNs)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
+    }
     return ok != 0;
 }
 
 // Waits for the phase of `bar` with the given parity to complete.  Gives up after
 // kWaitLimitNs, or as soon as another warp of the CTA has given up (*abort != 0);
 // on giving up it records `code` in the device fault word and returns false.
+template <unsigned HintNs = 0>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
                                           unsigned code, unsigned *fault) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait<HintNs>(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     while (true) {
 #pragma unroll 1
         for (int i = 0; i < 32; ++i)
-            if (mbar_try_wait(bar, parity)) return true;
+            if (mbar_try_wait<HintNs>(bar, parity)) return true;
         if (*abort) return false;
         if (globaltimer() - t0 > kWaitLimitNs) {
             *abort = 1;
@@ -89,9 +89,10 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 }
 
 // mbar_wait by every lane of a warp, with one warp-uniform outcome.
+template <unsigned HintNs = 0>
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int *abort, unsigned code,
                                           unsigned *fault) {
-    const bool ok = mbar_wait(bar, parity, abort, code, fault);
+    const bool ok = mbar_wait<HintNs>(bar, parity, abort, code, fault);
     return __all_sync(0xffffffffu, ok);
 }
 
@@ -336,6 +337,20 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool 
 }
 
 __device__ __forceinline__ uint32_t elect_lane0() { return (threadIdx.x & 31) == 0; }
+
+// One lane of a fully converged warp (elect.sync).  tcgen05 issue code runs the whole
+// schedule warp-uniformly (waits, addresses, descriptors) and predicates only the
+// instruction itself on this, which keeps the operands in uniform registers; with a
+// single-lane loop each MMA costs two to three times the tensor pipe's own time.
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile(
+        "{\n\t.reg .pred P;\n\t"
+        "elect.sync _|P, 0xffffffff;\n\t"
+        "selp.u32 %0, 1, 0, P;\n\t}"
+        : "=r"(pred));
+    return pred != 0;
+}
 
 }  // namespace tc
 }  // namespace dsc

@@ -33,6 +33,11 @@ namespace tc {
 
 __device__ unsigned int g_fault = 0;
 
+// Waiting warps sleep on their mbarrier (up to this many ns per try) rather than poll:
+// the two epilogue sets spend much of each tile waiting, and their polling takes issue
+// slots from the set that is computing (about 4% of the forward's time).
+constexpr unsigned kWaitHint = 2000;
+
 // Build-time tuning constants of the forward kernel.
 #ifndef DSC_FWD_SETS
 #define DSC_FWD_SETS 2         // epilogue warp sets working on alternating tiles (1 or 2)
@@ -194,7 +199,7 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
                 const int slice = i % p.n_slices, tl_ = i / p.n_slices;
                 const int b = tl_ / p.tiles_per_seq, t0 = (tl_ % p.tiles_per_seq) * kTt;
                 const int s = it % S, n = it / S;
-                if (!mbar_wait(bar.empty(s), (n & 1) ^ 1, abort, 2u, &g_fault)) break;
+                if (!mbar_wait<kWaitHint>(bar.empty(s), (n & 1) ^ 1, abort, 2u, &g_fault)) break;
                 mbar_arrive_expect_tx(bar.full(s), p.x_stage_tx + p.z_stage_bytes + p.u_bytes);
                 const uint32_t st = sb + s * p.stage_bytes;
                 tma_load_3d(st + p.off_x, &tm_x, bar.full(s), slice * kDt, t0 - (W - 1), b);
@@ -207,41 +212,45 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
             const int issued = it;
             for (int s = 0; s < S && s < issued; ++s) {
                 const int last = issued - 1 - ((issued - 1 - s) % S);   // last tile using stage s
-                mbar_wait(bar.full(s), (last / S) & 1, abort, 0u, &g_fault);
+                mbar_wait<kWaitHint>(bar.full(s), (last / S) & 1, abort, 0u, &g_fault);
             }
         }
         __syncwarp();
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            const int nchunks = (p.n_pad + 255) / 256;
-            const uint32_t ubox = (uint32_t)(p.R * 128);
-            const int ksteps = p.R / 16;
-            // descriptor templates: only the start address changes per MMA
-            const uint64_t t_z = desc_tmpl(16, 8u * p.R * 2u, p.z_layout);   // z tile, K-major
-            const uint64_t t_u = desc_tmpl(ubox, 1024, kSw128);              // U slice, MN-major
-            const uint32_t i_full = idesc_bf16(128, 256, false, true);
-            const uint32_t i_last = idesc_bf16(128, p.n_pad - 256 * (nchunks - 1), false, true);
-            int it = 0;
-            for (int i = blockIdx.x; i < p.n_tiles; i += gridDim.x, ++it) {
-                const int s = it % S, n = it / S;
-                const int a = it % p.nbuf, m = it / p.nbuf;
-                if (!mbar_wait(bar.full(s), n & 1, abort, 8u, &g_fault)) break;
-                if (!mbar_wait(bar.acce(a), (m & 1) ^ 1, abort, 16u, &g_fault)) break;
-                tc_fence_after();
-                const uint32_t d = tmem + a * p.bufcols;
-                const uint32_t za = sb + s * p.stage_bytes + p.off_z;
-                const uint32_t ua = sb + s * p.stage_bytes + p.off_u;
-                for (int nc = 0; nc < nchunks; ++nc) {
-                    const uint32_t idesc = nc + 1 < nchunks ? i_full : i_last;
-                    for (int kk = 0; kk < ksteps; ++kk)
-                        mma_bf16_ss(d + 256 * nc, desc_at(t_z, za + kk * 32),
-                                    desc_at(t_u, ua + nc * 4 * ubox + kk * 2048), idesc, kk > 0 ? 1u : 0u);
+        // The whole warp runs the schedule; one elected lane issues each tcgen05
+        // instruction, and descriptors advance by adding to their start-address field.
+        const int nchunks = (p.n_pad + 255) / 256;
+        const uint32_t ubox = (uint32_t)(p.R * 128);
+        const int ksteps = p.R / 16;
+        const uint64_t t_z = desc_tmpl(16, 8u * p.R * 2u, p.z_layout);   // z tile, K-major
+        const uint64_t t_u = desc_tmpl(ubox, 1024, kSw128);              // U slice, MN-major
+        const uint32_t i_full = idesc_bf16(128, 256, false, true);
+        const uint32_t i_last = idesc_bf16(128, p.n_pad - 256 * (nchunks - 1), false, true);
+        int it = 0;
+        for (int i = blockIdx.x; i < p.n_tiles; i += gridDim.x, ++it) {
+            const int s = it % S, n = it / S;
+            const int a = it % p.nbuf, m = it / p.nbuf;
+            if (!warp_wait<kWaitHint>(bar.full(s), n & 1, abort, 8u, &g_fault)) break;
+            if (!warp_wait<kWaitHint>(bar.acce(a), (m & 1) ^ 1, abort, 16u, &g_fault)) break;
+            tc_fence_after();
+            const uint32_t d = tmem + a * p.bufcols;
+            const uint32_t za = sb + s * p.stage_bytes + p.off_z;
+            const uint32_t ua = sb + s * p.stage_bytes + p.off_u;
+            for (int nc = 0; nc < nchunks; ++nc) {
+                const uint32_t idesc = nc + 1 < nchunks ? i_full : i_last;
+                uint64_t dz = desc_at(t_z, za), du = desc_at(t_u, ua + nc * 4 * ubox);
+                for (int kk = 0; kk < ksteps; ++kk) {
+                    if (elect_one()) mma_bf16_ss(d + 256 * nc, dz, du, idesc, kk > 0 ? 1u : 0u);
+                    __syncwarp();
+                    dz += 32u >> 4;
+                    du += 2048u >> 4;
                 }
-                mma_commit(bar.accf(a));
             }
-            mma_commit(bar.done());
+            if (elect_one()) mma_commit(bar.accf(a));
+            __syncwarp();
         }
+        if (elect_one()) mma_commit(bar.done());
         __syncwarp();
     } else {
         // ---------------------------------------------------------- epilogue
@@ -272,8 +281,8 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
             const int b = tlin / p.tiles_per_seq, t0 = (tlin - b * p.tiles_per_seq) * kTt;
             const int s = it % S, n = it / S;
             const int a = it % p.nbuf, m = it / p.nbuf;
-            if (!warp_wait(bar.full(s), n & 1, abort, 32u, &g_fault)) break;
-            if (!warp_wait(bar.accf(a), m & 1, abort, 64u, &g_fault)) break;
+            if (!warp_wait<kWaitHint>(bar.full(s), n & 1, abort, 32u, &g_fault)) break;
+            if (!warp_wait<kWaitHint>(bar.accf(a), m & 1, abort, 64u, &g_fault)) break;
             tc_fence_after();
             const int yb = yc & 1;
             if (lane == 0) bulk_wait_read<1>();
@@ -335,7 +344,7 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
 
     __syncthreads();
     if (warp == 1) {
-        if (lane == 0) mbar_wait(bar.done(), 0, abort, 0u, &g_fault);
+        if (lane == 0) mbar_wait<kWaitHint>(bar.done(), 0, abort, 0u, &g_fault);
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, p.tmem_cols);
