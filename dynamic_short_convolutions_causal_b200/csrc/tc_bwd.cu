@@ -360,49 +360,72 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             const uint32_t st = sb + s * p.stage_bytes;
             const uint32_t dys = st, xs = st + p.xy_tile_bytes;
             // ---- A1: dx[t,c] = dy[t,c] + sum_k w[t+k,g,k] dy[t+k,c]
-            // All shared-memory loads of the phase are issued before its first store (the
-            // stores are ordered asm statements and would otherwise serialise the loads).
+            // The warp's 16 channels are two 8-channel chunks, taken in batches of CB chunks:
+            // a batch's shared-memory and TMEM loads are all issued before its first store
+            // (the stores are ordered asm statements and would otherwise serialise the
+            // loads); with many taps one chunk per batch keeps the registers in budget.
             constexpr int CH = kCPW / 8;
-            {
-                uint4 du[CH][W];
+            constexpr int CB = (W * CH <= 8) ? CH : 1;
+            constexpr int NGB = 8 * CB / G;                 // filter groups of a batch
 #pragma unroll
-                for (int cq = 0; cq < CH; ++cq)
+            for (int c0 = 0; c0 < CH; c0 += CB) {
+                uint4 du[CB][W];
 #pragma unroll
-                    for (int k = 0; k < W; ++k) du[cq][k] = lds128(dys + (dyr[k] ^ ((uint32_t)cq << 4)));
-                uint4 dxo[CH];
-                constexpr int NGW = kCPW / G;                  // filter groups of the warp's channels
-                uint32_t wr[W][NGW];
+                for (int cb = 0; cb < CB; ++cb)
 #pragma unroll
-                for (int k = 0; k < W; ++k) tmem_ld<NGW>(tl + p.tm_w + k * p.NGp + (kCPW * h) / G, wr[k]);
+                    for (int k = 0; k < W; ++k) du[cb][k] = lds128(dys + (dyr[k] ^ ((uint32_t)(c0 + cb) << 4)));
+                uint32_t wr[W][NGB];
+#pragma unroll
+                for (int k = 0; k < W; ++k)
+                    tmem_ld<NGB>(tl + p.tm_w + k * p.NGp + (kCPW * h + 8 * c0) / G, wr[k]);
                 tmem_wait_ld();
 #pragma unroll
                 for (int k = 0; k < W; ++k)
 #pragma unroll
-                    for (int e = 0; e < NGW; ++e) asm volatile("" : "+r"(wr[k][e]));
+                    for (int e = 0; e < NGB; ++e) asm volatile("" : "+r"(wr[k][e]));
+                uint4 dxo[CB];
 #pragma unroll
-                for (int cq = 0; cq < CH; ++cq) {
-                    const int gq = (8 * cq) / G;                   // chunk's first group within the warp's
+                for (int cb = 0; cb < CB; ++cb) {
+                    const int gq = (8 * cb) / G;                   // chunk's first group within the batch
                     float dx[8];
-                    {
-                        float d0[8];
-                        unpack8(du[cq][0], d0);
+                    if constexpr (G == 1) {
+                        // channel pairs in packed fp32 FMAs (the same roundings as scalar fmaf)
+                        uint64_t acc[4];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) dx[e] = fmaf(__uint_as_float(wr[0][gq + e / G]), d0[e], d0[e]);
+                        for (int k = 0; k < W; ++k) {
+                            const uint32_t u[4] = {du[cb][k].x, du[cb][k].y, du[cb][k].z, du[cb][k].w};
+#pragma unroll
+                            for (int m = 0; m < 4; ++m) {
+                                const uint64_t d2 = f2pack(bf16_lo(u[m]), bf16_hi(u[m]));
+                                const uint64_t w2 = f2pack(__uint_as_float(wr[k][gq + 2 * m]),
+                                                           __uint_as_float(wr[k][gq + 2 * m + 1]));
+                                acc[m] = f2fma(w2, d2, k == 0 ? d2 : acc[m]);
+                            }
+                        }
+#pragma unroll
+                        for (int m = 0; m < 4; ++m) f2unpack(acc[m], dx[2 * m], dx[2 * m + 1]);
+                    } else {
+                        {
+                            float d0[8];
+                            unpack8(du[cb][0], d0);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) dx[e] = fmaf(__uint_as_float(wr[0][gq + e / G]), d0[e], d0[e]);
+                        }
+#pragma unroll
+                        for (int k = 1; k < W; ++k) {
+                            float dk[8];
+                            unpack8(du[cb][k], dk);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) dx[e] = fmaf(__uint_as_float(wr[k][gq + e / G]), dk[e], dx[e]);
+                        }
                     }
-#pragma unroll
-                    for (int k = 1; k < W; ++k) {
-                        float dk[8];
-                        unpack8(du[cq][k], dk);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) dx[e] = fmaf(__uint_as_float(wr[k][gq + e / G]), dk[e], dx[e]);
-                    }
-                    dxo[cq].x = pack_bf16x2(dx[0], dx[1]);
-                    dxo[cq].y = pack_bf16x2(dx[2], dx[3]);
-                    dxo[cq].z = pack_bf16x2(dx[4], dx[5]);
-                    dxo[cq].w = pack_bf16x2(dx[6], dx[7]);
+                    dxo[cb].x = pack_bf16x2(dx[0], dx[1]);
+                    dxo[cb].y = pack_bf16x2(dx[2], dx[3]);
+                    dxo[cb].z = pack_bf16x2(dx[4], dx[5]);
+                    dxo[cb].w = pack_bf16x2(dx[6], dx[7]);
                 }
 #pragma unroll
-                for (int cq = 0; cq < CH; ++cq) sts128(dxrow ^ ((uint32_t)cq << 4), dxo[cq]);
+                for (int cb = 0; cb < CB; ++cb) sts128(dxrow ^ ((uint32_t)(c0 + cb) << 4), dxo[cb]);
             }
             tc_fence_before();
             fence_proxy_async_smem();
@@ -415,16 +438,19 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             // ---- B of the previous tile (its dz / dU MMAs ran during A1)
             if (pv.it >= 0 && !phase_b(pv)) { ok = false; break; }
             // ---- A2: dw[t,g,k] = sum_{c in g} dy[t,c] x[t-k,c], tap-major column k*NG + g
-            {
-                uint4 d0[CH], xu[CH][W];
+            // (in batches of CB chunks, as A1)
 #pragma unroll
-                for (int cq = 0; cq < CH; ++cq) {
-                    d0[cq] = lds128(dys + (dyr[0] ^ ((uint32_t)cq << 4)));
+            for (int c0 = 0; c0 < CH; c0 += CB) {
+                uint4 d0[CB], xu[CB][W];
 #pragma unroll
-                    for (int k = 0; k < W; ++k) xu[cq][k] = lds128(xs + (xr[k] ^ ((uint32_t)cq << 4)));
+                for (int cb = 0; cb < CB; ++cb) {
+                    d0[cb] = lds128(dys + (dyr[0] ^ ((uint32_t)(c0 + cb) << 4)));
+#pragma unroll
+                    for (int k = 0; k < W; ++k) xu[cb][k] = lds128(xs + (xr[k] ^ ((uint32_t)(c0 + cb) << 4)));
                 }
 #pragma unroll
-                for (int cq = 0; cq < CH; ++cq) {
+                for (int cb = 0; cb < CB; ++cb) {
+                    const int cq = c0 + cb;
                     const int g8 = (kCPW * h + 8 * cq) / G;
 #pragma unroll
                     for (int k = 0; k < W; ++k) {
@@ -432,14 +458,14 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
                         if constexpr (G == 1) {
                             // one channel per group: dw = dy * x, exact in fp32 and rounded once
                             // to bf16, which is what the packed bf16 multiply computes
-                            pk[0] = bf16x2_mul(d0[cq].x, xu[cq][k].x);
-                            pk[1] = bf16x2_mul(d0[cq].y, xu[cq][k].y);
-                            pk[2] = bf16x2_mul(d0[cq].z, xu[cq][k].z);
-                            pk[3] = bf16x2_mul(d0[cq].w, xu[cq][k].w);
+                            pk[0] = bf16x2_mul(d0[cb].x, xu[cb][k].x);
+                            pk[1] = bf16x2_mul(d0[cb].y, xu[cb][k].y);
+                            pk[2] = bf16x2_mul(d0[cb].z, xu[cb][k].z);
+                            pk[3] = bf16x2_mul(d0[cb].w, xu[cb][k].w);
                         } else {
                             float dv[8], xv[8], dw[NG8];
-                            unpack8(d0[cq], dv);
-                            unpack8(xu[cq][k], xv);
+                            unpack8(d0[cb], dv);
+                            unpack8(xu[cb][k], xv);
 #pragma unroll
                             for (int gl = 0; gl < NG8; ++gl) {
                                 float acc = 0.f;
