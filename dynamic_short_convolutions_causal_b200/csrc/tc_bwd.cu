@@ -42,16 +42,24 @@ __device__ unsigned int g_fault_bwd = 0;
 
 constexpr int kTt = 128;
 constexpr int kDt = 64;
-constexpr int kEpiWarps = 16;           // 4 lane quarters x 4 channel groups of 16
-constexpr int kCPW = 16;                // channels per epilogue warp
-constexpr int kDxBuf = 32 * kCPW * 2;   // one warp's dx staging: 32 rows x 16 bf16
-// Warp roles: 0 TMA producer, 1 recompute MMAs, 2..17 epilogue, 18 dz MMAs, 19 dU MMAs.
+// Epilogue geometry: 16 warps of 16 channels (4 TMEM lane quarters x 4 channel groups).
+// (8 warps of 32 channels, with 168 registers a thread, measured slower at G=4, W=8:
+// 0.76 against 0.74 ms on the lowrank_mlp backward.)
+// Warp roles: 0 TMA producer, 1 recompute MMAs, 2..1+E epilogue, 2+E dz MMAs, 3+E dU MMAs.
 // The three MMA streams are issued from warps on three different SM sub-partitions: one
-// warp issuing all of them shares its issue slots with four busy epilogue warps and
-// cannot keep the tensor pipe fed.  Twenty warps keep the 96-register budget of eighteen.
-constexpr int kDzWarp = 2 + kEpiWarps;
-constexpr int kDuWarp = 3 + kEpiWarps;
-constexpr int kThreads = 32 * (4 + kEpiWarps);
+// warp issuing all of them shares its issue slots with the busy epilogue warps and cannot
+// keep the tensor pipe fed.
+template <int G>
+struct Geo {
+    static constexpr int kEpiWarps = 16;
+    static constexpr int kGroups = kEpiWarps / 4;      // channel groups of a slice
+    static constexpr int kCPW = kDt / kGroups;         // channels per epilogue warp
+    static constexpr int kDxBuf = 32 * kCPW * 2;       // one warp's dx staging: 32 rows x kCPW bf16
+    static constexpr int kDzWarp = 2 + kEpiWarps;
+    static constexpr int kDuWarp = 3 + kEpiWarps;
+    static constexpr int kThreads = 32 * (4 + kEpiWarps);
+};
+constexpr uint32_t kDxStageBytes = 4 * 32 * kDt * 2;   // all epilogue warps' dx staging
 
 struct BwdParams {
     int B, T, D, G, W, R;
@@ -133,11 +141,13 @@ __host__ __device__ inline int owner_of(long long i, long long n, long long g) {
 }
 
 template <int W, int G>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Geo<G>::kThreads, 1)
 k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ CUtensorMap tm_x,
                  const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_u,
                  const __grid_constant__ CUtensorMap tm_dx, const BwdParams p) {
     constexpr int NG8 = 8 / G;          // filter groups in one 8-channel chunk
+    constexpr int kEpiWarps = Geo<G>::kEpiWarps, kCPW = Geo<G>::kCPW, kDxBuf = Geo<G>::kDxBuf;
+    constexpr int kDzWarp = Geo<G>::kDzWarp, kDuWarp = Geo<G>::kDuWarp, kThreads = Geo<G>::kThreads;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sb = smem_u32(smem);
@@ -280,19 +290,21 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
         // Per tile i:  A1(i) dx  ->  B(i-1) dz partial, dU flush, stage release  ->  A2(i) dw.
         const int ew = warp - 2;
         const int q = warp & 3;              // TMEM lane quarter == token rows 32q..32q+31
-        const int h = ew >> 2;               // channel group of the slice (16 channels)
+        const int h = ew >> 2;               // channel group of the slice (kCPW channels)
         const int row = 32 * q + lane;
+        constexpr int CH = kCPW / 8;         // 16-byte chunks of the warp's channels in a row
         const uint32_t dxstage = sb + p.off_dx + (uint32_t)ew * kDxBuf;
-        // 32-byte staging rows in the TMA store's 32-byte swizzle (16-byte chunk ^ (lane/4)%2)
-        const uint32_t dxrow = (dxstage + lane * 32) ^ ((uint32_t)((lane >> 2) & 1) << 4);
+        // staging rows of kCPW*2 bytes in the TMA store's 32- or 64-byte swizzle: the 16-byte
+        // chunk index is XORed with address bits 7.. of the row start
+        const uint32_t dxrow = (dxstage + lane * (2 * kCPW)) ^ ((((uint32_t)lane * (2 * kCPW) >> 7) & (CH - 1)) << 4);
         // dy rows r = row + k and x rows r = row + W-1-k of the 128-byte-swizzled tiles
         uint32_t dyr[W], xr[W];
 #pragma unroll
         for (int k = 0; k < W; ++k) {
             uint32_t r = (uint32_t)(row + k);
-            dyr[k] = (r * 128u) ^ ((r & 7u) << 4) ^ ((uint32_t)(2 * h) << 4);
+            dyr[k] = (r * 128u) ^ ((r & 7u) << 4) ^ ((uint32_t)(CH * h) << 4);
             r = (uint32_t)(row + (W - 1) - k);
-            xr[k] = (r * 128u) ^ ((r & 7u) << 4) ^ ((uint32_t)(2 * h) << 4);
+            xr[k] = (r * 128u) ^ ((r & 7u) << 4) ^ ((uint32_t)(CH * h) << 4);
         }
         // dw^T shared-memory tile: MN-major, 128B swizzle, atoms of 64 columns x 128 rows
         const uint32_t dwrow = sb + p.off_dw + (uint32_t)row * 128u;
@@ -308,12 +320,22 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             if (!warp_wait(bar.mm2(), t.it & 1, abort, 256u, &g_fault_bwd)) return false;
             tc_fence_after();
             {
-                // dz partial: every warp reads R/4 of the columns of its 32 rows
+                // dz partial: every warp reads its group's share of the columns of its 32 rows
                 const int tok = t.t0 + row;
-                const int nc = p.R / 4;
+                const int nc = p.R / Geo<G>::kGroups;
                 float *dst = p.dz_part + ((size_t)t.slice * p.B * p.T + (size_t)t.b * p.T + tok) * p.R + h * nc;
+                int c0 = 0;
 #pragma unroll 1
-                for (int c0 = 0; c0 < nc; c0 += 4) {
+                for (; c0 + 8 <= nc; c0 += 8) {
+                    uint32_t v[8];
+                    tmem_ld<8>(tl + p.tm_dz + h * nc + c0, v);
+                    tmem_wait_ld_regs(v);
+                    if (tok < p.T) {
+                        *reinterpret_cast<uint4 *>(dst + c0) = make_uint4(v[0], v[1], v[2], v[3]);
+                        *reinterpret_cast<uint4 *>(dst + c0 + 4) = make_uint4(v[4], v[5], v[6], v[7]);
+                    }
+                }
+                if (c0 < nc) {   // nc = 4 (R = 16 with four channel groups)
                     uint32_t v[4];
                     tmem_ld<4>(tl + p.tm_dz + h * nc + c0, v);
                     tmem_wait_ld_regs(v);
@@ -363,11 +385,11 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             // The warp's 16 channels are two 8-channel chunks, taken in batches of CB chunks:
             // a batch's shared-memory and TMEM loads are all issued before its first store
             // (the stores are ordered asm statements and would otherwise serialise the
-            // loads); with many taps one chunk per batch keeps the registers in budget.
-            constexpr int CH = kCPW / 8;
+            // loads); with many taps one chunk per batch keeps the registers in budget, and
+            // the batch loop stays rolled so that the many-tap body fits the instruction cache.
             constexpr int CB = (W * CH <= 8) ? CH : 1;
             constexpr int NGB = 8 * CB / G;                 // filter groups of a batch
-#pragma unroll
+#pragma unroll 1
             for (int c0 = 0; c0 < CH; c0 += CB) {
                 uint4 du[CB][W];
 #pragma unroll
@@ -439,7 +461,7 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             if (pv.it >= 0 && !phase_b(pv)) { ok = false; break; }
             // ---- A2: dw[t,g,k] = sum_{c in g} dy[t,c] x[t-k,c], tap-major column k*NG + g
             // (in batches of CB chunks, as A1)
-#pragma unroll
+#pragma unroll 1
             for (int c0 = 0; c0 < CH; c0 += CB) {
                 uint4 d0[CB], xu[CB][W];
 #pragma unroll
@@ -730,7 +752,7 @@ bool plan_bwd(int B, int T, int D, int G, int W, int R, int grid, BwdParams &p) 
         p.off_dw = p.off_u + p.nU * p.u_bytes;
         p.off_dw = (p.off_dw + 1023) / 1024 * 1024;
         p.off_dx = p.off_dw + (uint32_t)(p.SCp / 64) * 16384u;
-        p.off_bar = p.off_dx + kEpiWarps * kDxBuf;
+        p.off_bar = p.off_dx + kDxStageBytes;
         if (p.off_bar + kBarBytes + 16 + 1024 <= kSmemLimit) return true;
     }
     return false;
@@ -742,7 +764,7 @@ cudaError_t launch_t(const CUtensorMap *m, const BwdParams &p, int grid, cudaStr
     const uint32_t smem = p.off_bar + kBarBytes + 16 + 1024;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, kThreads, smem, s>>>(m[0], m[1], m[2], m[3], m[4], p);
+    kern<<<grid, Geo<G>::kThreads, smem, s>>>(m[0], m[1], m[2], m[3], m[4], p);
     return cudaGetLastError();
 }
 
@@ -805,12 +827,15 @@ cudaError_t launch_tc_lowrank_bwd(const void *x, const void *z, const void *U, c
     const uint32_t bz[3] = {8, p.rows, 1};
     const uint64_t du[2] = {(uint64_t)N, (uint64_t)R};
     const uint32_t bu[2] = {64, (uint32_t)R};
+    constexpr int kCPW = Geo<1>::kCPW;   // the same for every G
+    static_assert(kCPW == 16 || kCPW == 32, "dx staging rows are 32 or 64 bytes");
     const uint32_t bdx[3] = {(uint32_t)kCPW, 32, 1};
     if (!make_map(&m[0], dy, 3, dxyz, bxy, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) ||
         !make_map(&m[1], x, 3, dxyz, bxy, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) ||
         !make_map(&m[2], z, 3, dzz, bz, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
         !make_map(&m[3], Up, 2, du, bu, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
-        !make_map(&m[4], dx, 3, dxyz, bdx, CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B)) {
+        !make_map(&m[4], dx, 3, dxyz, bdx, kCPW == 16 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B)) {
         set_last_error("dsc_bwd_lowrank: cuTensorMapEncodeTiled failed");
         return cudaErrorInvalidValue;
     }
