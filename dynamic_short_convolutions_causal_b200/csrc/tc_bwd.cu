@@ -618,16 +618,17 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
     }
 }
 
-// Up[r, s*SC + k*NG + g] = U[r, s*SC + g*W + k]  (tap-major columns within each slice)
+// Up[r, s*SC + k*NG + g] = U[r, s*SC + g*W + k]  (tap-major columns within each slice).
+// Grid (ceil(N/256), R): one row r per grid row, 32-bit index arithmetic.
 __global__ void k_permute_u(const bf16 *__restrict__ U, bf16 *__restrict__ Up, int R, int N, int SC, int NG,
                             int W) {
-    const size_t n = (size_t)R * N;
-    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n; e += (size_t)gridDim.x * blockDim.x) {
-        const int r = (int)(e / N), j = (int)(e % N);
-        const int s = j / SC, jl = j % SC;
-        const int k = jl / NG, g = jl % NG;
-        Up[e] = U[(size_t)r * N + (size_t)s * SC + g * W + k];
-    }
+    const int r = blockIdx.y;
+    const int j = blockIdx.x * blockDim.x + threadIdx.x;
+    if (r >= R || j >= N) return;
+    const int s = j / SC, jl = j - s * SC;
+    const int k = jl / NG, g = jl - k * NG;
+    const size_t row = (size_t)r * N;
+    Up[row + j] = U[row + s * SC + g * W + k];
 }
 
 // dz[bt, :] = sum_s part[s, bt, :]  (slices in order)
@@ -642,20 +643,24 @@ __global__ void k_reduce_dz(const float *__restrict__ part, float *__restrict__ 
     }
 }
 
-// dU[r, s*SC + j] = sum over the CTA segments of slice s of part[s, seg, r, j]  (in order)
+// dU[r, s*SC + j] = sum over the CTA segments of slice s of part[s, seg, r, j]  (in order).
+// Grid (ceil(N/1024), R): one row r per grid row, four consecutive columns per thread
+// (SC is a multiple of 8, so the four never straddle a slice).
 __global__ void k_reduce_du(const float *__restrict__ part, float *__restrict__ dU, int R, int SC, int n_slices,
                             int maxseg, int per_slice, int n_tiles, int grid) {
-    const size_t n = (size_t)R * SC * n_slices;
-    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n; e += (size_t)gridDim.x * blockDim.x) {
-        const int N = SC * n_slices;
-        const int r = (int)(e / N), j = (int)(e % N);
-        const int s = j / SC, jl = j % SC;
-        const int c0 = owner_of((long long)s * per_slice, n_tiles, grid);
-        const int c1 = owner_of((long long)(s + 1) * per_slice - 1, n_tiles, grid);
-        float acc = 0.f;
-        for (int seg = 0; seg <= c1 - c0; ++seg) acc += part[(((size_t)s * maxseg + seg) * R + r) * SC + jl];
-        dU[(size_t)r * N + j] = acc;
+    const int N = SC * n_slices;
+    const int r = blockIdx.y;
+    const int j = 4 * (blockIdx.x * blockDim.x + threadIdx.x);
+    if (r >= R || j >= N) return;
+    const int s = j / SC, jl = j - s * SC;
+    const int nseg = owner_of((long long)(s + 1) * per_slice - 1, n_tiles, grid) -
+                     owner_of((long long)s * per_slice, n_tiles, grid) + 1;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int seg = 0; seg < nseg; ++seg) {
+        const float4 v = *reinterpret_cast<const float4 *>(part + (((size_t)s * maxseg + seg) * R + r) * SC + jl);
+        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
     }
+    *reinterpret_cast<float4 *>(dU + (size_t)r * N + j) = acc;
 }
 
 // ------------------------------------------------------------------ host side
@@ -818,7 +823,7 @@ cudaError_t launch_tc_lowrank_bwd(const void *x, const void *z, const void *U, c
     p.dz_part = (float *)(w8 + l.dz);
     p.du_part = (float *)(w8 + l.du);
     const int N = p.n_slices * p.SC;
-    k_permute_u<<<std::min(4096, (R * N + 255) / 256), 256, 0, s>>>((const bf16 *)U, Up, R, N, p.SC, p.NGs, W);
+    k_permute_u<<<dim3((N + 255) / 256, R), 256, 0, s>>>((const bf16 *)U, Up, R, N, p.SC, p.NGs, W);
 
     CUtensorMap m[5];
     const uint64_t dxyz[3] = {(uint64_t)D, (uint64_t)T, (uint64_t)B};
@@ -853,9 +858,8 @@ cudaError_t launch_tc_lowrank_bwd(const void *x, const void *z, const void *U, c
     if (e != cudaSuccess) return e;
     const size_t n4 = (size_t)B * T * R / 4;
     k_reduce_dz<<<(unsigned)std::min<size_t>((n4 + 255) / 256, 8192), 256, 0, s>>>(p.dz_part, dz, p.n_slices, n4);
-    const size_t nu = (size_t)R * N;
-    k_reduce_du<<<(unsigned)std::min<size_t>((nu + 255) / 256, 8192), 256, 0, s>>>(
-        p.du_part, dU, R, p.SC, p.n_slices, p.maxseg, p.per_slice, p.n_tiles, grid);
+    k_reduce_du<<<dim3((N / 4 + 255) / 256, R), 256, 0, s>>>(p.du_part, dU, R, p.SC, p.n_slices, p.maxseg,
+                                                           p.per_slice, p.n_tiles, grid);
     return cudaGetLastError();
 }
 
