@@ -457,12 +457,12 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
                 tma_store_3d(&tm_dx, dxstage, id.slice * kDt + kCPW * h, id.t0 + 32 * q, id.b);
                 bulk_commit();
             }
-            // ---- B of the previous tile (its dz / dU MMAs ran during A1)
-            if (pv.it >= 0 && !phase_b(pv)) { ok = false; break; }
-            // ---- A2: dw[t,g,k] = sum_{c in g} dy[t,c] x[t-k,c], tap-major column k*NG + g
-            // (in batches of CB chunks, as A1)
-#pragma unroll 1
-            for (int c0 = 0; c0 < CH; c0 += CB) {
+            // ---- A2: dw[t,g,k] = sum_{c in g} dy[t,c] x[t-k,c], tap-major column k*NG + g,
+            // in batches of CB chunks as A1.  A batch is computed into registers (pk) and
+            // then stored; only the stores need the previous tile's dz / dU MMAs to be done
+            // with the dw tile, so a single-batch A2 is computed before B waits for them.
+            constexpr int NPK = (NG8 + 1) / 2;           // packed bf16 pairs per (chunk, tap)
+            auto a2_compute = [&](int c0, uint32_t (&pk)[CB][W][NPK]) {
                 uint4 d0[CB], xu[CB][W];
 #pragma unroll
                 for (int cb = 0; cb < CB; ++cb) {
@@ -471,19 +471,16 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
                     for (int k = 0; k < W; ++k) xu[cb][k] = lds128(xs + (xr[k] ^ ((uint32_t)(c0 + cb) << 4)));
                 }
 #pragma unroll
-                for (int cb = 0; cb < CB; ++cb) {
-                    const int cq = c0 + cb;
-                    const int g8 = (kCPW * h + 8 * cq) / G;
+                for (int cb = 0; cb < CB; ++cb)
 #pragma unroll
                     for (int k = 0; k < W; ++k) {
-                        uint32_t pk[4];
                         if constexpr (G == 1) {
                             // one channel per group: dw = dy * x, exact in fp32 and rounded once
                             // to bf16, which is what the packed bf16 multiply computes
-                            pk[0] = bf16x2_mul(d0[cb].x, xu[cb][k].x);
-                            pk[1] = bf16x2_mul(d0[cb].y, xu[cb][k].y);
-                            pk[2] = bf16x2_mul(d0[cb].z, xu[cb][k].z);
-                            pk[3] = bf16x2_mul(d0[cb].w, xu[cb][k].w);
+                            pk[cb][k][0] = bf16x2_mul(d0[cb].x, xu[cb][k].x);
+                            pk[cb][k][1] = bf16x2_mul(d0[cb].y, xu[cb][k].y);
+                            pk[cb][k][2] = bf16x2_mul(d0[cb].z, xu[cb][k].z);
+                            pk[cb][k][3] = bf16x2_mul(d0[cb].w, xu[cb][k].w);
                         } else {
                             float dv[8], xv[8], dw[NG8];
                             unpack8(d0[cb], dv);
@@ -496,19 +493,43 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
                                 dw[gl] = acc;
                             }
 #pragma unroll
-                            for (int m2 = 0; m2 < NG8 / 2; ++m2) pk[m2] = pack_bf16x2(dw[2 * m2], dw[2 * m2 + 1]);
+                            for (int m2 = 0; m2 < NG8 / 2; ++m2) pk[cb][k][m2] = pack_bf16x2(dw[2 * m2], dw[2 * m2 + 1]);
                         }
+                    }
+            };
+            auto a2_store = [&](int c0, const uint32_t (&pk)[CB][W][NPK]) {
+#pragma unroll
+                for (int cb = 0; cb < CB; ++cb) {
+                    const int g8 = (kCPW * h + 8 * (c0 + cb)) / G;
+#pragma unroll
+                    for (int k = 0; k < W; ++k) {
                         const int jp = k * p.NGs + g8;                    // first tap-major column
                         const uint32_t atom = (uint32_t)(jp >> 6), within = (uint32_t)(jp & 63);
                         const uint32_t a = dwrow + atom * 16384u + ((((within >> 3) << 4) ^ dwsw) | ((within & 7) * 2));
                         if constexpr (NG8 == 8) {
-                            sts128(a, make_uint4(pk[0], pk[1], pk[2], pk[3]));
+                            sts128(a, make_uint4(pk[cb][k][0], pk[cb][k][1], pk[cb][k][2], pk[cb][k][3]));
                         } else if constexpr (NG8 == 4) {
-                            sts64(a, pk[0], pk[1]);
+                            sts64(a, pk[cb][k][0], pk[cb][k][1]);
                         } else {
-                            sts32(a, pk[0]);
+                            sts32(a, pk[cb][k][0]);
                         }
                     }
+                }
+            };
+            if constexpr (CB == CH) {
+                uint32_t pk[CB][W][NPK];
+                a2_compute(0, pk);
+                // ---- B of the previous tile (its dz / dU MMAs ran during A1)
+                if (pv.it >= 0 && !phase_b(pv)) { ok = false; break; }
+                a2_store(0, pk);
+            } else {
+                // several batches (many taps): holding one across B cost more than it hid
+                if (pv.it >= 0 && !phase_b(pv)) { ok = false; break; }
+#pragma unroll 1
+                for (int c0 = 0; c0 < CH; c0 += CB) {
+                    uint32_t pk[CB][W][NPK];
+                    a2_compute(c0, pk);
+                    a2_store(c0, pk);
                 }
             }
             tc_fence_before();
