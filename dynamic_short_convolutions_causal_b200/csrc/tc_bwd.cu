@@ -375,10 +375,6 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             }
             const int s = it % p.stages, n = it / p.stages;
             if (!warp_wait(bar.full(s), n & 1, abort, 64u, &g_fault_bwd)) { ok = false; break; }
-            if (!warp_wait(bar.wfull(), it & 1, abort, 128u, &g_fault_bwd)) { ok = false; break; }
-            tc_fence_after();
-            if (lane == 0) bulk_wait_read<0>();
-            __syncwarp();
             const uint32_t st = sb + s * p.stage_bytes;
             const uint32_t dys = st, xs = st + p.xy_tile_bytes;
             // ---- A1: dx[t,c] = dy[t,c] + sum_k w[t+k,g,k] dy[t+k,c]
@@ -387,15 +383,28 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             // (the stores are ordered asm statements and would otherwise serialise the
             // loads); with many taps one chunk per batch keeps the registers in budget, and
             // the batch loop stays rolled so that the many-tap body fits the instruction cache.
+            // A single batch's dy rows are loaded before the wait for the recomputed filters.
             constexpr int CB = (W * CH <= 8) ? CH : 1;
             constexpr int NGB = 8 * CB / G;                 // filter groups of a batch
+            uint4 dpre[CB][W];
+            if constexpr (CB == CH) {
+#pragma unroll
+                for (int cb = 0; cb < CB; ++cb)
+#pragma unroll
+                    for (int k = 0; k < W; ++k) dpre[cb][k] = lds128(dys + (dyr[k] ^ ((uint32_t)cb << 4)));
+            }
+            if (!warp_wait(bar.wfull(), it & 1, abort, 128u, &g_fault_bwd)) { ok = false; break; }
+            tc_fence_after();
+            if (lane == 0) bulk_wait_read<0>();
+            __syncwarp();
 #pragma unroll 1
             for (int c0 = 0; c0 < CH; c0 += CB) {
                 uint4 du[CB][W];
 #pragma unroll
                 for (int cb = 0; cb < CB; ++cb)
 #pragma unroll
-                    for (int k = 0; k < W; ++k) du[cb][k] = lds128(dys + (dyr[k] ^ ((uint32_t)(c0 + cb) << 4)));
+                    for (int k = 0; k < W; ++k)
+                        du[cb][k] = (CB == CH) ? dpre[cb][k] : lds128(dys + (dyr[k] ^ ((uint32_t)(c0 + cb) << 4)));
                 uint32_t wr[W][NGB];
 #pragma unroll
                 for (int k = 0; k < W; ++k)
