@@ -661,33 +661,39 @@ __global__ void k_permute_u(const bf16 *__restrict__ U, bf16 *__restrict__ Up, i
     Up[row + j] = U[row + s * SC + g * W + k];
 }
 
-// dz[bt, :] = sum_s part[s, bt, :]  (slices in order)
-__global__ void k_reduce_dz(const float *__restrict__ part, float *__restrict__ dz, int n_slices, size_t n4) {
-    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n4; e += (size_t)gridDim.x * blockDim.x) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int s = 0; s < n_slices; ++s) {
-            const float4 v = reinterpret_cast<const float4 *>(part)[(size_t)s * n4 + e];
-            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+// Both reductions in one launch (they are independent, so the small dU sum runs beside
+// the dz sum instead of after it):
+//   blocks [0, nb_dz):  dz[bt, :] = sum_s part_dz[s, bt, :]  (slices in order), grid-stride
+//                       over float4 elements;
+//   blocks [nb_dz, ..): dU[r, s*SC + j] = sum over the CTA segments of slice s of
+//                       part_du[s, seg, r, j]  (in order); block nb_dz + r*nbx + bx covers row
+//                       r, columns 4*(256*bx + thread) .. +3 (SC is a multiple of 8, so the
+//                       four never straddle a slice).
+__global__ void k_reduce(const float *__restrict__ part_dz, float *__restrict__ dz, int n_slices, size_t n4,
+                         int nb_dz, const float *__restrict__ part_du, float *__restrict__ dU, int R, int SC,
+                         int maxseg, int per_slice, int n_tiles, int grid, int nbx) {
+    if ((int)blockIdx.x < nb_dz) {
+        for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n4; e += (size_t)nb_dz * blockDim.x) {
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int s = 0; s < n_slices; ++s) {
+                const float4 v = reinterpret_cast<const float4 *>(part_dz)[(size_t)s * n4 + e];
+                acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+            }
+            reinterpret_cast<float4 *>(dz)[e] = acc;
         }
-        reinterpret_cast<float4 *>(dz)[e] = acc;
+        return;
     }
-}
-
-// dU[r, s*SC + j] = sum over the CTA segments of slice s of part[s, seg, r, j]  (in order).
-// Grid (ceil(N/1024), R): one row r per grid row, four consecutive columns per thread
-// (SC is a multiple of 8, so the four never straddle a slice).
-__global__ void k_reduce_du(const float *__restrict__ part, float *__restrict__ dU, int R, int SC, int n_slices,
-                            int maxseg, int per_slice, int n_tiles, int grid) {
+    const int bid = (int)blockIdx.x - nb_dz;
+    const int r = bid / nbx;
     const int N = SC * n_slices;
-    const int r = blockIdx.y;
-    const int j = 4 * (blockIdx.x * blockDim.x + threadIdx.x);
+    const int j = 4 * ((bid - r * nbx) * (int)blockDim.x + (int)threadIdx.x);
     if (r >= R || j >= N) return;
     const int s = j / SC, jl = j - s * SC;
     const int nseg = owner_of((long long)(s + 1) * per_slice - 1, n_tiles, grid) -
                      owner_of((long long)s * per_slice, n_tiles, grid) + 1;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     for (int seg = 0; seg < nseg; ++seg) {
-        const float4 v = *reinterpret_cast<const float4 *>(part + (((size_t)s * maxseg + seg) * R + r) * SC + jl);
+        const float4 v = *reinterpret_cast<const float4 *>(part_du + (((size_t)s * maxseg + seg) * R + r) * SC + jl);
         acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
     }
     *reinterpret_cast<float4 *>(dU + (size_t)r * N + j) = acc;
@@ -887,9 +893,10 @@ cudaError_t launch_tc_lowrank_bwd(const void *x, const void *z, const void *U, c
     }
     if (e != cudaSuccess) return e;
     const size_t n4 = (size_t)B * T * R / 4;
-    k_reduce_dz<<<(unsigned)std::min<size_t>((n4 + 255) / 256, 8192), 256, 0, s>>>(p.dz_part, dz, p.n_slices, n4);
-    k_reduce_du<<<dim3((N / 4 + 255) / 256, R), 256, 0, s>>>(p.du_part, dU, R, p.SC, p.n_slices, p.maxseg,
-                                                           p.per_slice, p.n_tiles, grid);
+    const int nb_dz = (int)std::min<size_t>((n4 + 255) / 256, 8192);
+    const int nbx = (N / 4 + 255) / 256;
+    k_reduce<<<nb_dz + nbx * R, 256, 0, s>>>(p.dz_part, dz, p.n_slices, n4, nb_dz, p.du_part, dU, R, p.SC,
+                                             p.maxseg, p.per_slice, p.n_tiles, grid, nbx);
     return cudaGetLastError();
 }
 
