@@ -22,7 +22,7 @@
 //   Recompute, dz and dU are issued by three MMA warps, each on its own SM sub-partition.
 // Persistent CTAs own contiguous tile ranges in slice-major order.  dz partials (per
 // slice) and dU partials (per CTA segment of a slice) go to the workspace and are summed
-// in a fixed order by two small kernels, so results are deterministic.
+// in a fixed order by one small kernel, so results are deterministic.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
