@@ -649,16 +649,21 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
 }
 
 // Up[r, s*SC + k*NG + g] = U[r, s*SC + g*W + k]  (tap-major columns within each slice).
-// Grid (ceil(N/256), R): one row r per grid row, 32-bit index arithmetic.
+// Grid (ceil(N/2048), R): one row r per grid row; each thread writes 8 consecutive output
+// columns with one 16-byte store (NG is a multiple of 8, so the 8 share one tap k and read
+// source columns W apart).
 __global__ void k_permute_u(const bf16 *__restrict__ U, bf16 *__restrict__ Up, int R, int N, int SC, int NG,
                             int W) {
     const int r = blockIdx.y;
-    const int j = blockIdx.x * blockDim.x + threadIdx.x;
+    const int j = 8 * (blockIdx.x * blockDim.x + threadIdx.x);
     if (r >= R || j >= N) return;
     const int s = j / SC, jl = j - s * SC;
     const int k = jl / NG, g = jl - k * NG;
-    const size_t row = (size_t)r * N;
-    Up[row + j] = U[row + s * SC + g * W + k];
+    const unsigned short *src = reinterpret_cast<const unsigned short *>(U) + (size_t)r * N + s * SC + g * W + k;
+    uint32_t v[4];
+#pragma unroll
+    for (int m = 0; m < 4; ++m) v[m] = (uint32_t)src[(2 * m) * W] | ((uint32_t)src[(2 * m + 1) * W] << 16);
+    *reinterpret_cast<uint4 *>(Up + (size_t)r * N + j) = make_uint4(v[0], v[1], v[2], v[3]);
 }
 
 // Both reductions in one launch (they are independent, so the small dU sum runs beside
@@ -859,7 +864,7 @@ cudaError_t launch_tc_lowrank_bwd(const void *x, const void *z, const void *U, c
     p.dz_part = (float *)(w8 + l.dz);
     p.du_part = (float *)(w8 + l.du);
     const int N = p.n_slices * p.SC;
-    k_permute_u<<<dim3((N + 255) / 256, R), 256, 0, s>>>((const bf16 *)U, Up, R, N, p.SC, p.NGs, W);
+    k_permute_u<<<dim3((N / 8 + 255) / 256, R), 256, 0, s>>>((const bf16 *)U, Up, R, N, p.SC, p.NGs, W);
 
     CUtensorMap m[5];
     const uint64_t dxyz[3] = {(uint64_t)D, (uint64_t)T, (uint64_t)B};
