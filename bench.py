@@ -135,48 +135,68 @@ def max_over_ranks(v, world, device):
 
 
 # ------------------------------------------------------------------ CPU oracle baseline
+def _oracle_inputs(wl):
+    import numpy as np  # noqa: F401
+    t = di.make(di.scaled(wl, B=1, T=min(wl.T, 2048)), "cpu", ("x", "z", "U", "dy"))
+    return {k: v.to(torch.float64).numpy() for k, v in t.items()}
+
+
+def _oracle_step(f, wl, L):
+    """One oracle fwd + bwd on the first L tokens of one sequence; returns seconds."""
+    import oracle
+    t0 = time.perf_counter()
+    oracle.fwd_lowrank(f["x"][:, :L], f["z"][:, :L], f["U"], wl.G, wl.W)
+    oracle.bwd_lowrank(f["x"][:, :L], f["z"][:, :L], f["U"], f["dy"][:, :L], wl.G, wl.W)
+    return time.perf_counter() - t0
+
+
+def _oracle_sample_len(f, wl, budget_s):
+    """Tokens L of one sequence whose oracle fwd + bwd takes about budget_s."""
+    L0 = 16
+    dt0 = _oracle_step(f, wl, L0)
+    return int(max(L0, min(f["x"].shape[1], L0 * budget_s / max(dt0, 1e-6))))
+
+
+def _oracle_desc(wl, L):
+    return ("oracle fwd+bwd (plain C, fp64, 1 thread) on the first %d tokens of one "
+            "sequence of the %s workload (D=%d, R=%d, G=%d, W=%d)" % (L, wl.name, wl.D, wl.R, wl.G, wl.W))
+
+
 def oracle_sample_rate(wl, budget_s=15.0):
     """Time the CPU oracle (fwd + bwd) on a bounded sample of the workload: the first
     L tokens of one sequence, with L chosen so the run takes about `budget_s`.
     Returns (tokens/s, description, seconds)."""
-    import numpy as np
-    import oracle
-    t = di.make(di.scaled(wl, B=1, T=min(wl.T, 2048)), "cpu", ("x", "z", "U", "dy"))
-    f = {k: v.to(torch.float64).numpy() for k, v in t.items()}
-
-    def run(L):
-        t0 = time.perf_counter()
-        oracle.fwd_lowrank(f["x"][:, :L], f["z"][:, :L], f["U"], wl.G, wl.W)
-        oracle.bwd_lowrank(f["x"][:, :L], f["z"][:, :L], f["U"], f["dy"][:, :L], wl.G, wl.W)
-        return time.perf_counter() - t0
-
-    L0 = 16
-    dt0 = run(L0)
-    L = int(max(L0, min(f["x"].shape[1], L0 * budget_s / max(dt0, 1e-6))))
-    dt = run(L) if L != L0 else dt0
-    desc = ("oracle fwd+bwd (plain C, fp64, 1 thread) on the first %d tokens of one "
-            "sequence of the %s workload (D=%d, R=%d, G=%d, W=%d)" % (L, wl.name, wl.D, wl.R, wl.G, wl.W))
-    return L / dt, desc, dt
+    f = _oracle_inputs(wl)
+    L = _oracle_sample_len(f, wl, budget_s)
+    dt = _oracle_step(f, wl, L)
+    return L / dt, _oracle_desc(wl, L), dt
 
 
 def run_reference(args, wl, world, rank):
-    """The reference arm: the CPU oracle as it stands, on host cores."""
+    """The reference arm: the CPU oracle as it stands, on host cores.  A step is one
+    oracle fwd + bwd over a fixed sample of the workload (the first L tokens of one
+    sequence, L sized so the whole run takes a few minutes); ms_per_step is the time of
+    that sample, and the sample is named in config."""
     if rank != 0:
         return 0
-    rates = []
-    desc = ""
+    f = _oracle_inputs(wl)
+    per_step = max(0.05, args.ref_budget / max(1, args.steps + args.warmup))
+    L = _oracle_sample_len(f, wl, per_step)
+    times = []
     for i in range(args.warmup + args.steps):
-        rate, desc, _ = oracle_sample_rate(wl, budget_s=args.ref_budget)
+        dt = _oracle_step(f, wl, L)
         if i >= args.warmup:
-            rates.append(rate)
-    v = statistics.median(rates)
+            times.append(dt)
+    s_step = statistics.mean(times)
+    v = L / s_step
+    desc = _oracle_desc(wl, L)
     line = {
         "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1e3 * wl.tokens / v, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": 1e3 * s_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,s^2))",
         "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "D": wl.D, "G": wl.G, "W": wl.W,
-                   "R": wl.R, "tokens_per_step": wl.tokens},
+                   "R": wl.R, "tokens_per_step": L, "sample": desc},
         "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle", "sample": desc},
         "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
@@ -253,6 +273,12 @@ def run_ours(args, wl, world, rank, local):
     if not args.no_e2e:
         e2e = measure_e2e(dsc, t, y, dx, dz, dU, ws, wl, world, dev, args)
 
+    comps = None
+    if world == 1 and not args.no_comparators:
+        del t, x, z, U, dy, y, dx, dz, dU, ws
+        torch.cuda.empty_cache()
+        comps = measure_comparators(dsc, dev, peak, args)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, desc, _ = oracle_sample_rate(wl, budget_s=args.cpu_budget)
@@ -276,21 +302,120 @@ def run_ours(args, wl, world, rank, local):
                          "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": traffic, "algorithmic_bytes": dom[1]},
             "gpu_launches": (launches_fwd + launches_bwd) * args.steps,
-            "e2e": e2e, "cpu_baseline": cpu, "clocks": ck,
+            "e2e": e2e, "cpu_baseline": cpu, "clocks": ck, "comparators": comps,
         }
         print(json.dumps(line), flush=True)
     return 0
 
 
+def _time_calls(fn, stream, steps, warmup=3):
+    """Mean CUDA-event time (ms) of fn() on `stream`, after `warmup` untimed calls."""
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        fn()
+    e.record(stream)
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / steps
+
+
+def measure_comparators(dsc, dev, peak, args):
+    """Other paths timed in the same run, each on its own workload: the in-repo static
+    depthwise causal convolution (the primitive the method generalises) on the MLP-width
+    shape, the explicit-filter forward on the stacked-QKV shape, and the fused low-rank
+    step on the MLP-width shape.  Inputs exceed L2; times are CUDA events per call."""
+    stream = torch.cuda.current_stream(dev)
+    steps = max(3, min(args.steps, 10))
+    out = {}
+
+    def entry(ms, nbytes, tokens):
+        gbs = nbytes / (ms * 1e-3) / 1e9
+        return {"ms": ms, "algorithmic_bytes": nbytes, "gbs": gbs, "frac_of_peak": gbs / peak,
+                "tokens_per_s": tokens / (ms * 1e-3)}
+
+    # static depthwise causal conv, fwd + bwd, on the MLP-width shape
+    wl = di.WORKLOADS["lowrank_mlp"]
+    t = di.make(wl, dev, ("x", "dy", "ws"))
+    x, dy, w = t["x"], t["dy"], t["ws"]
+    y = torch.empty_like(x)
+    dx = torch.empty_like(x)
+    dw = torch.empty((wl.D, wl.W), dtype=torch.float32, device=dev)
+    ws = dsc.workspace(dsc.dsc_static_bwd_workspace_bytes(wl.B, wl.T, wl.D, wl.W), dev)
+    act = wl.tokens * wl.D * 2
+    fwd_ms = _time_calls(lambda: dsc.dsc_static_fwd(x, w, y), stream, steps)
+    bwd_ms = _time_calls(lambda: dsc.dsc_static_bwd(x, w, dy, dx, dw, ws), stream, steps)
+    sb_f = 2 * act + wl.D * wl.W * 2
+    sb_b = 3 * act + wl.D * wl.W * (2 + 4)
+    out["static_conv_" + wl.name] = {
+        "shape": {"B": wl.B, "T": wl.T, "D": wl.D, "W": wl.W},
+        "fwd": entry(fwd_ms, sb_f, wl.tokens), "bwd": entry(bwd_ms, sb_b, wl.tokens),
+        "fwd_bwd": entry(fwd_ms + bwd_ms, sb_f + sb_b, wl.tokens)}
+    del t, x, dy, w, y, dx, dw, ws
+
+    # fused low-rank fwd + bwd on the MLP-width shape
+    t = di.make(wl, dev, ("x", "z", "U", "dy"))
+    x, z, U, dy = t["x"], t["z"], t["U"], t["dy"]
+    y = torch.empty_like(x)
+    dx = torch.empty_like(x)
+    dz = torch.empty((wl.B, wl.T, wl.R), dtype=torch.float32, device=dev)
+    dU = torch.empty((wl.R, wl.N), dtype=torch.float32, device=dev)
+    ws = dsc.workspace(dsc.dsc_bwd_lowrank_workspace_bytes(wl.B, wl.T, wl.D, wl.G, wl.W, wl.R), dev)
+    fwd_ms = _time_calls(lambda: dsc.dsc_fwd_lowrank(x, z, U, y, wl.G, wl.W), stream, steps)
+    bwd_ms = _time_calls(lambda: dsc.dsc_bwd_lowrank(x, z, U, dy, dx, dz, dU, ws, wl.G, wl.W), stream, steps)
+    fb, bb = algorithmic_bytes(wl)
+    out["lowrank_" + wl.name.split("_", 1)[1]] = {
+        "shape": {"B": wl.B, "T": wl.T, "D": wl.D, "G": wl.G, "W": wl.W, "R": wl.R},
+        "fwd": entry(fwd_ms, fb, wl.tokens), "bwd": entry(bwd_ms, bb, wl.tokens),
+        "fwd_bwd": entry(fwd_ms + bwd_ms, fb + bb, wl.tokens),
+        "path": dsc.dsc_lowrank_path(wl.B, wl.T, wl.D, wl.G, wl.W, wl.R)}
+    del t, x, z, U, dy, y, dx, dz, dU, ws
+
+    # explicit-filter forward on the stacked-QKV shape
+    wl = di.WORKLOADS["tied_qkv"]
+    t = di.make(wl, dev, ("x", "w"))
+    x, w = t["x"], t["w"]
+    y = torch.empty_like(x)
+    ms = _time_calls(lambda: dsc.dsc_fwd(x, w, y, wl.G), stream, steps)
+    nb = 2 * wl.tokens * wl.D * 2 + wl.tokens * wl.NG * wl.W * 2
+    out["explicit_fwd_" + wl.name] = {"shape": {"B": wl.B, "T": wl.T, "D": wl.D, "G": wl.G, "W": wl.W},
+                                      "fwd": entry(ms, nb, wl.tokens)}
+    del t, x, w, y
+    torch.cuda.empty_cache()
+    return out
+
+
+def source_hash():
+    """Hash of the library's kernel and ABI sources (csrc/ and include/): a stored ncu
+    traffic figure is reported only for the build it was measured on."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    pkg = os.path.join(ROOT, "dynamic_short_convolutions_causal_b200", "csrc")
+    files = sorted(glob.glob(os.path.join(pkg, "*.cu")) + glob.glob(os.path.join(pkg, "*.cuh")) +
+                   glob.glob(os.path.join(pkg, "*.h")) + glob.glob(os.path.join(ROOT, "include", "*.h")))
+    for p in files:
+        h.update(os.path.basename(p).encode())
+        with open(p, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def load_traffic(kernel, wl):
-    """Per-launch DRAM bytes from a committed ncu summary, if one matches the current
-    kernel build (profiles/traffic.json); null otherwise."""
+    """Per-call DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum over the
+    call's kernels) from profiles/traffic.json, if its entry was captured on the
+    current sources (same source_hash()); null otherwise."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(p) as f:
             d = json.load(f)
         ent = d.get(wl.name, {}).get(kernel)
-        return ent["bytes_per_launch"] if ent else None
+        if not ent or ent.get("source_hash") != source_hash():
+            return None
+        return ent["bytes_per_launch"]
     except Exception:
         return None
 
@@ -356,7 +481,9 @@ def main(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
-    ap.add_argument("--ref-budget", type=float, default=8.0)
+    ap.add_argument("--ref-budget", type=float, default=120.0,
+                    help="seconds of oracle work for the whole reference run (warm-up + steps)")
+    ap.add_argument("--no-comparators", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -11,10 +11,12 @@
 // The array lives in device global memory as a file-scope __device__ variable; every
 // GPU that loads the library holds it until the process exits.  Host code cannot use
 // the array's name as a device address (on the host it names a stand-in object), so
-// the address is fetched once per device with cudaGetSymbolAddress, with that device
-// current, and passed to the kernels.
+// each call looks the address up with cudaGetSymbolAddress, with the calling device
+// current, and passes it to the kernels.  The lookup is a host-side query; doing it
+// on every call (rather than caching it) keeps the address right after the device's
+// context is torn down and the module is loaded again, for example after
+// cudaDeviceReset.
 #include <cstdio>
-#include <mutex>
 
 #include "../../include/dsc.h"
 #include "internal.h"
@@ -22,35 +24,22 @@
 namespace {
 
 constexpr size_t kScratchBytes = 16u << 20;   // 16 MiB
-constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) float g_static_bwd_scratch[kScratchBytes / sizeof(float)];
 
-std::mutex g_mu;
-float *g_scratch_addr[kMaxDevices] = {};
-
-// Address of the scratch array on the current device; set up on the first call on
-// each device.  Returns nullptr (and records why) on failure.
+// Address of the scratch array on the current device.  Returns nullptr (and records
+// why) on failure.  The first call on a device may load the library's module onto it.
 float *scratch_on_current_device() {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-        dsc::set_last_error("dsc_static_bwd_noalloc: no usable current CUDA device");
+    float *ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress((void **)&ptr, g_static_bwd_scratch);
+    if (e != cudaSuccess || !ptr) {
+        char msg[256];
+        snprintf(msg, sizeof(msg), "dsc_static_bwd_noalloc: cudaGetSymbolAddress failed: %s",
+                 cudaGetErrorString(e));
+        dsc::set_last_error(msg);
         return nullptr;
     }
-    std::lock_guard<std::mutex> lock(g_mu);
-    if (!g_scratch_addr[dev]) {
-        float *ptr = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress((void **)&ptr, g_static_bwd_scratch);
-        if (e != cudaSuccess || !ptr) {
-            char msg[256];
-            snprintf(msg, sizeof(msg), "dsc_static_bwd_noalloc: cudaGetSymbolAddress failed: %s",
-                     cudaGetErrorString(e));
-            dsc::set_last_error(msg);
-            return nullptr;
-        }
-        g_scratch_addr[dev] = ptr;
-    }
-    return g_scratch_addr[dev];
+    return ptr;
 }
 
 }  // namespace

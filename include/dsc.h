@@ -144,9 +144,10 @@ DSC_API dsc_status_t dsc_static_bwd(const void *x, const void *w, const void *dy
  *     (16 MiB) compiled into the library; every GPU that loads the library holds it
  *     until the process exits.  Sizes whose dsc_static_bwd_workspace_bytes() exceed it
  *     are rejected with DSC_ERR_UNSUPPORTED and a message naming both sizes.
- *   - The first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call before
- *     any stream capture.
+ *   - Each call looks up the array's device address (cudaGetSymbolAddress) with the
+ *     calling device current, so the address stays right if the device's context is
+ *     reset.  The first call on a device may load the library's module onto it; make
+ *     that first call before any stream capture.
  *   - All calls on a device share the array, which keeps the last call's contents.
  *     Calls that can overlap on the GPU (other streams, other host threads) race on
  *     it; the caller must order them.  No part of it needs to start at zero. */
