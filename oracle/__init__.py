@@ -58,6 +58,8 @@ def _bind(lib):
         "oracle_bwd_lowrank": (i, [dp, dp, dp, dp, dp, dp, dp, i, i, i, i, i, i]),
         "oracle_static_fwd": (None, [dp, dp, dp, i, i, i, i]),
         "oracle_static_bwd": (None, [dp, dp, dp, dp, dp, i, i, i, i]),
+        "oracle_decode": (None, [dp, dp, dp, dp, dp, i, i, i, i]),
+        "oracle_decode_lowrank": (i, [dp, dp, dp, dp, dp, dp, i, i, i, i, i]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -185,6 +187,40 @@ class Oracle:
         return dx, dws
 
 
+    def decode(self, x_t, w_t, state, G):
+        """One decode step with explicit filters: x_t [B,D], w_t [B,D/G,W], state
+        [B,W-1,D] (oldest row first).  Returns (y_t [B,D], new state [B,W-1,D])."""
+        x_t = np.asarray(x_t)
+        B, D = x_t.shape
+        W = np.asarray(w_t).shape[-1]
+        _check_dims(B, 1, D, G, W)
+        x_t = _in(x_t, (B, D))
+        w_t = _in(w_t, (B, D // G, W))
+        state = _in(state, (B, W - 1, D))
+        y = np.empty_like(x_t)
+        st = np.empty_like(state)
+        self._l.oracle_decode(_p(x_t), _p(w_t), _p(state), _p(y), _p(st), B, D, G, W)
+        return y, st
+
+    def decode_lowrank(self, x_t, z_t, U, state, G, W):
+        """One decode step with w_t = z_t U: x_t [B,D], z_t [B,R], U [R,(D/G)*W],
+        state [B,W-1,D].  Returns (y_t [B,D], new state [B,W-1,D])."""
+        x_t = np.asarray(x_t)
+        B, D = x_t.shape
+        R = np.asarray(z_t).shape[-1]
+        _check_dims(B, 1, D, G, W, R)
+        x_t = _in(x_t, (B, D))
+        z_t = _in(z_t, (B, R))
+        U = _in(U, (R, (D // G) * W))
+        state = _in(state, (B, W - 1, D))
+        y = np.empty_like(x_t)
+        st = np.empty_like(state)
+        if self._l.oracle_decode_lowrank(_p(x_t), _p(z_t), _p(U), _p(state), _p(y), _p(st),
+                                         B, D, G, W, R):
+            raise MemoryError("oracle_decode_lowrank")
+        return y, st
+
+
 def default() -> Oracle:
     global _default
     if _default is None:
@@ -229,3 +265,11 @@ def static_fwd(x, ws):
 
 def static_bwd(x, ws, dy):
     return default().static_bwd(x, ws, dy)
+
+
+def decode(x_t, w_t, state, G):
+    return default().decode(x_t, w_t, state, G)
+
+
+def decode_lowrank(x_t, z_t, U, state, G, W):
+    return default().decode_lowrank(x_t, z_t, U, state, G, W)

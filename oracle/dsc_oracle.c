@@ -211,3 +211,67 @@ void oracle_static_bwd(const double *x, const double *ws, const double *dy,
                 }
             }
 }
+
+/*
+ * One decode step: token t of each of B sequences, with the W-1 tokens before it
+ * taken from a rolling window instead of from the sequence itself (the page notes
+ * that inference still needs engineering: "Significancia e Alegacoes").  The same
+ * formula as above at a single position:
+ *   y_t[c] = x_t[c] + w_t[g(c),0] x_t[c] + sum_{k=1}^{W-1} w_t[g(c),k] x_{t-k}[c]
+ * Layouts (row-major):
+ *   x_t, y_t   : [B, D]
+ *   state      : [B, W-1, D], row i holds x_{t-(W-1)+i} (oldest first; zeros before
+ *                the start of a sequence), so x_{t-k} is row W-1-k
+ *   state_out  : [B, W-1, D], the window after the step: rows shifted by one, x_t last
+ */
+static void decode_one(const double *x_t, const double *wt, const double *state,
+                       double *y_t, double *state_out, int D, int G, int W)
+{
+    for (int c = 0; c < D; ++c) {
+        const int g = c / G;
+        double acc = x_t[c];
+        acc += wt[g * W + 0] * x_t[c];
+        for (int k = 1; k < W; ++k)
+            acc += wt[g * W + k] * state[(size_t)(W - 1 - k) * D + c];
+        y_t[c] = acc;
+    }
+    for (int i = 0; i + 1 < W - 1; ++i)
+        for (int c = 0; c < D; ++c)
+            state_out[(size_t)i * D + c] = state[(size_t)(i + 1) * D + c];
+    if (W > 1)
+        for (int c = 0; c < D; ++c)
+            state_out[(size_t)(W - 2) * D + c] = x_t[c];
+}
+
+/* Decode step with explicit filters w_t [B, D/G, W]. */
+void oracle_decode(const double *x_t, const double *w_t, const double *state,
+                   double *y_t, double *state_out, int B, int D, int G, int W)
+{
+    const int NG = D / G;
+    for (int b = 0; b < B; ++b)
+        decode_one(x_t + (size_t)b * D, w_t + (size_t)b * NG * W,
+                   state + (size_t)b * (W - 1) * D, y_t + (size_t)b * D,
+                   state_out + (size_t)b * (W - 1) * D, D, G, W);
+}
+
+/* Decode step with low-rank filters w_t = z_t U; z_t [B, R], U [R, (D/G)*W]. */
+int oracle_decode_lowrank(const double *x_t, const double *z_t, const double *U,
+                          const double *state, double *y_t, double *state_out,
+                          int B, int D, int G, int W, int R)
+{
+    const int N = (D / G) * W;
+    double *wt = (double *)malloc(sizeof(double) * (size_t)N);
+    if (!wt) return 1;
+    for (int b = 0; b < B; ++b) {
+        for (int j = 0; j < N; ++j) {
+            double s = 0.0;
+            for (int r = 0; r < R; ++r)
+                s += z_t[(size_t)b * R + r] * U[(size_t)r * N + j];
+            wt[j] = s;
+        }
+        decode_one(x_t + (size_t)b * D, wt, state + (size_t)b * (W - 1) * D,
+                   y_t + (size_t)b * D, state_out + (size_t)b * (W - 1) * D, D, G, W);
+    }
+    free(wt);
+    return 0;
+}

@@ -25,6 +25,12 @@ gist.science/pt/paper/2606.03825, "Metodologia > Convolucoes Curtas Dinamicas"):
                      Jacobian; y is linear in each argument separately, so central
                      differences are exact up to rounding.
   * invariant     -- sum(dU*U) == sum(dz*z) (both equal sum_t <dw_t, w_t>).
+  * decode        -- one decode step (a token with its W-1 predecessors held in a
+                     rolling window; "Significancia e Alegacoes" notes that inference
+                     still needs engineering) is the forward at the last position of
+                     the sequence [window rows, x_t]; stepping through a sequence from
+                     a zero window gives the pinned forward's outputs token by token,
+                     and the window then holds the last W-1 inputs.
 """
 from __future__ import annotations
 
@@ -314,6 +320,50 @@ def pin_adjoint_and_invariant(orc):
     assert abs(a - b) <= 1e-10 * max(1.0, abs(a)), "sum(dU*U) %r != sum(dz*z) %r" % (a, b)
 
 
+# ---------------------------------------------------------------- decode step
+def pin_decode_is_forward_at_last_position(orc):
+    """A window of W-1 rows (oldest first) and x_t, run through the forward as a
+    W-token sequence whose last token carries the step's filters, gives y_t."""
+    r = _rng(13)
+    for (B, D, G, W, R) in [(2, 8, 1, 4, 3), (3, 12, 3, 5, 2), (1, 6, 6, 2, 4), (2, 4, 2, 1, 2)]:
+        NG = D // G
+        state = r.standard_normal((B, W - 1, D))
+        x_t = r.standard_normal((B, D))
+        xs = np.concatenate([state, x_t[:, None]], axis=1)           # [B, W, D]
+        w_full = r.standard_normal((B, W, NG, W))
+        y, st = orc.decode(x_t, w_full[:, -1], state, G)
+        _close(y, orc.fwd(xs, w_full, G)[:, -1], 1e-13, "explicit decode vs forward")
+        _close(st, xs[:, 1:], 0, "window after the step")
+        z_full = r.standard_normal((B, W, R))
+        U = r.standard_normal((R, NG * W))
+        y, st = orc.decode_lowrank(x_t, z_full[:, -1], U, state, G, W)
+        _close(y, orc.fwd_lowrank(xs, z_full, U, G, W)[:, -1], 1e-13, "lowrank decode vs forward")
+        _close(st, xs[:, 1:], 0, "window after the step (lowrank)")
+
+
+def pin_decode_steps_match_forward(orc):
+    """Stepping from a zero window reproduces the forward token by token (T = 1
+    included), and after n steps the window holds x_{n-W+1..n-1} (zeros before 0)."""
+    r = _rng(14)
+    B, T, D, G, W, R = 2, 9, 8, 2, 4, 3
+    NG = D // G
+    x = r.standard_normal((B, T, D))
+    z = r.standard_normal((B, T, R))
+    U = r.standard_normal((R, NG * W))
+    w = r.standard_normal((B, T, NG, W))
+    ref_lr = orc.fwd_lowrank(x, z, U, G, W)
+    ref_ex = orc.fwd(x, w, G)
+    s_lr = np.zeros((B, W - 1, D))
+    s_ex = np.zeros((B, W - 1, D))
+    for t in range(T):
+        y, s_lr = orc.decode_lowrank(x[:, t], z[:, t], U, s_lr, G, W)
+        _close(y, ref_lr[:, t], 1e-13, "lowrank decode step %d" % t)
+        y, s_ex = orc.decode(x[:, t], w[:, t], s_ex, G)
+        _close(y, ref_ex[:, t], 1e-13, "explicit decode step %d" % t)
+        pad = np.concatenate([np.zeros((B, W - 1, D)), x[:, :t + 1]], axis=1)
+        _close(s_lr, pad[:, -(W - 1):] if W > 1 else pad[:, :0], 0, "window after step %d" % t)
+
+
 PINS = [
     pin_hand_example,
     pin_identity_filter_doubles,
@@ -328,4 +378,6 @@ PINS = [
     pin_fd_explicit,
     pin_fd_static,
     pin_adjoint_and_invariant,
+    pin_decode_is_forward_at_last_position,
+    pin_decode_steps_match_forward,
 ]

@@ -35,6 +35,15 @@ MUTANTS = [
     ("static dws shifted by one tap",
      "dws[(size_t)c * W + k] += gy * x[(bt - k) * D + c];",
      "dws[(size_t)c * W + k] += gy * x[(bt - (k > 0 ? k - 1 : 0)) * D + c];"),
+    ("decode window read newest first",
+     "acc += wt[g * W + k] * state[(size_t)(W - 1 - k) * D + c];",
+     "acc += wt[g * W + k] * state[(size_t)(k - 1) * D + c];"),
+    ("decode window not shifted",
+     "state_out[(size_t)i * D + c] = state[(size_t)(i + 1) * D + c];",
+     "state_out[(size_t)i * D + c] = state[(size_t)i * D + c];"),
+    ("decode drops the residual",
+     "double acc = x_t[c];\n        acc += wt[g * W + 0] * x_t[c];",
+     "double acc = 0.0;\n        acc += wt[g * W + 0] * x_t[c];"),
     ("explicit dw misses the group sum (last channel wins)",
      "dw[(bt * NG + g) * W + k] += gy * x[(bt - k) * D + c];",
      "dw[(bt * NG + g) * W + k] = gy * x[(bt - k) * D + c];"),
