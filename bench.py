@@ -384,6 +384,30 @@ def measure_comparators(dsc, dev, peak, args):
     out["explicit_fwd_" + wl.name] = {"shape": {"B": wl.B, "T": wl.T, "D": wl.D, "G": wl.G, "W": wl.W},
                                       "fwd": entry(ms, nb, wl.tokens)}
     del t, x, w, y
+
+    # decode step (one token per sequence, rolling window) on the stacked-QKV width
+    wl = di.WORKLOADS["lowrank_qkv"]
+    D, G, W, R, N = wl.D, wl.G, wl.W, wl.R, wl.N
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(wl.seed)
+    U = (torch.randn((R, N), generator=gen, device=dev) * R ** -0.5).to(torch.bfloat16)
+    dec = {}
+    for B in (1, 8, 64, 256):
+        x = torch.randn((B, D), generator=gen, device=dev).to(torch.bfloat16)
+        z = torch.randn((B, R), generator=gen, device=dev).to(torch.bfloat16)
+        st = torch.randn((B, W - 1, D), generator=gen, device=dev).to(torch.bfloat16)
+        y = torch.empty_like(x)
+        ms = _time_calls(lambda: dsc.dsc_decode_step_lowrank(x, z, U, st, y, G, W), stream, 200, warmup=10)
+        nb = R * N * 2 + B * (D * 2 + R * 2 + 2 * (W - 1) * D * 2 + D * 2)
+        fl = B * (2 * R * N + 2 * W * D)
+        dec["B=%d" % B] = {"us": ms * 1e3, "algorithmic_bytes": nb, "gbs": nb / (ms * 1e-3) / 1e9,
+                           "frac_of_hbm_peak": nb / (ms * 1e-3) / 1e9 / peak,
+                           "tflops": fl / (ms * 1e-3) / 1e12, "tokens_per_s": B / (ms * 1e-3)}
+    out["decode_lowrank_" + wl.name.split("_", 1)[1]] = {
+        "shape": {"D": D, "G": G, "W": W, "R": R}, "per_batch": dec,
+        "note": "one step per call, inputs and window resident in HBM; the w = z U product "
+                "(2*R*N FLOP per sequence) runs on CUDA cores"}
+    del U, x, z, st, y
     torch.cuda.empty_cache()
     return out
 

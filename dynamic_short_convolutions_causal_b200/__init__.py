@@ -21,6 +21,7 @@ __all__ = [
     "DscError", "lib", "lib_path", "dsc_fwd", "dsc_fwd_lowrank", "dsc_bwd_lowrank",
     "dsc_bwd_lowrank_workspace_bytes", "dsc_bwd", "dsc_static_fwd", "dsc_static_bwd",
     "dsc_static_bwd_workspace_bytes", "dsc_static_bwd_noalloc", "dsc_lowrank_path",
+    "dsc_decode_step", "dsc_decode_step_lowrank",
     "DSC_F32", "DSC_BF16",
 ]
 
@@ -56,6 +57,8 @@ def _load():
         "dsc_static_bwd_noalloc": (i, [vp, vp, vp, vp, fp, i, i, i, i, i, vp]),
         "dsc_static_bwd_noalloc_max_scratch_bytes": (sz, []),
         "dsc_lowrank_path": (i, [i, i, i, i, i, i, i]),
+        "dsc_decode_step": (i, [vp, vp, vp, vp, i, i, i, i, i, vp]),
+        "dsc_decode_step_lowrank": (i, [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]),
         "dsc_device_fault": (ctypes.c_uint, [i]),
         "dsc_status_string": (ctypes.c_char_p, [i]),
         "dsc_last_error": (ctypes.c_char_p, []),
@@ -196,6 +199,29 @@ def dsc_static_bwd_noalloc(x, w, dy, dx, dw):
         _check(lib.dsc_static_bwd_noalloc(_ptr(x), _ptr(w), _ptr(dy), _ptr(dx), _ptr(dw), B, T, D,
                                           W, _dt(x), _stream(x)))
     return dx, dw
+
+
+def dsc_decode_step(x_t, w_t, state, y_t, G: int):
+    """One decode step with explicit filters: x_t, y_t [B,D], w_t [B,D/G,W], state
+    [B,W-1,D] (oldest row first, updated in place; may be None when W = 1)."""
+    B, D = x_t.shape
+    W = w_t.shape[-1]
+    _same(x_t, w_t, y_t, *([state] if state is not None else []))
+    with torch.cuda.device(x_t.device):
+        _check(lib.dsc_decode_step(_ptr(x_t), _ptr(w_t), _ptr(state), _ptr(y_t), B, D, G, W, _dt(x_t),
+                                   _stream(x_t)))
+    return y_t
+
+
+def dsc_decode_step_lowrank(x_t, z_t, U, state, y_t, G: int, W: int):
+    """One decode step with w_t = z_t U: z_t [B,R], U [R,(D/G)*W]; see dsc_decode_step."""
+    B, D = x_t.shape
+    R = z_t.shape[-1]
+    _same(x_t, z_t, U, y_t, *([state] if state is not None else []))
+    with torch.cuda.device(x_t.device):
+        _check(lib.dsc_decode_step_lowrank(_ptr(x_t), _ptr(z_t), _ptr(U), _ptr(state), _ptr(y_t), B, D, G,
+                                           W, R, _dt(x_t), _stream(x_t)))
+    return y_t
 
 
 def dsc_device_fault(reset: bool = False) -> int:

@@ -190,9 +190,45 @@ DSC_API dsc_status_t dsc_static_bwd(const void *x, const void *w, const void *dy
         return fail(DSC_ERR_UNSUPPORTED, "%s: workspace of %zu bytes is below the %zu required", fn,
                     workspace_bytes, need);
     const bool bf16 = dt == DSC_BF16;
-    dsc::launch_conv_dx(w, false, dy, dx, B, T, D, 1, W, bf16, true, (cudaStream_t)stream);
-    dsc::launch_static_dw(x, dy, (float *)workspace, dw, B, T, D, W, bf16, (cudaStream_t)stream);
+    dsc::launch_static_bwd(x, w, dy, dx, (float *)workspace, dw, B, T, D, W, bf16, (cudaStream_t)stream);
     return check_launch(fn);
+}
+
+DSC_API dsc_status_t dsc_decode_step(const void *x_t, const void *w_t, void *state, void *y_t, int B, int D,
+                                     int G, int W, dsc_dtype_t dt, dsc_stream_t stream) {
+    const char *fn = "dsc_decode_step";
+    dsc_status_t st = check_dims(fn, Dims{B, 1, D, G, W, -1}, dt);
+    if (st != DSC_OK) return st;
+    const void *p[] = {x_t, w_t, y_t};
+    const char *n[] = {"x_t", "w_t", "y_t"};
+    if ((st = check_ptrs(fn, p, n, 3)) != DSC_OK) return st;
+    if (W > 1) {
+        const void *sp[] = {state};
+        const char *sn[] = {"state"};
+        if ((st = check_ptrs(fn, sp, sn, 1)) != DSC_OK) return st;
+    }
+    return check_launch(fn, dsc::launch_decode(x_t, w_t, state, y_t, B, D, G, W, dt == DSC_BF16,
+                                               (cudaStream_t)stream));
+}
+
+DSC_API dsc_status_t dsc_decode_step_lowrank(const void *x_t, const void *z_t, const void *U, void *state,
+                                             void *y_t, int B, int D, int G, int W, int R, dsc_dtype_t dt,
+                                             dsc_stream_t stream) {
+    const char *fn = "dsc_decode_step_lowrank";
+    dsc_status_t st = check_dims(fn, Dims{B, 1, D, G, W, R}, dt);
+    if (st != DSC_OK) return st;
+    const void *p[] = {x_t, z_t, U, y_t};
+    const char *n[] = {"x_t", "z_t", "U", "y_t"};
+    if ((st = check_ptrs(fn, p, n, 4)) != DSC_OK) return st;
+    if (W > 1) {
+        const void *sp[] = {state};
+        const char *sn[] = {"state"};
+        if ((st = check_ptrs(fn, sp, sn, 1)) != DSC_OK) return st;
+    }
+    if (!dsc::decode_supported(D, G, W, R))
+        return fail(DSC_ERR_UNSUPPORTED, "%s: R=%d with W=%d needs more shared memory than a block has", fn, R, W);
+    return check_launch(fn, dsc::launch_decode_lowrank(x_t, z_t, U, state, y_t, B, D, G, W, R, dt == DSC_BF16,
+                                                       (cudaStream_t)stream));
 }
 
 DSC_API int dsc_lowrank_path(int B, int T, int D, int G, int W, int R, dsc_dtype_t dt) {

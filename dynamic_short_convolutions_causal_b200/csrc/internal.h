@@ -10,14 +10,23 @@ namespace dsc {
 // Records the detail string that dsc_last_error() returns on this host thread.
 void set_last_error(const char *msg);
 
-// CUDA-core kernels (simt.cu)
+// Streaming CUDA-core kernels (stream.cu)
 void launch_conv_fwd(const void *x, const void *w, void *y, int B, int T, int D, int G, int W,
                      bool bf16, bool is_static, cudaStream_t s);
+int static_dw_partials(int B, int T);
+void launch_static_bwd(const void *x, const void *w, const void *dy, void *dx, float *part,
+                       float *dw, int B, int T, int D, int W, bool bf16, cudaStream_t s);
+
+// Decode step (decode.cu)
+bool decode_supported(int D, int G, int W, int R);
+cudaError_t launch_decode_lowrank(const void *x, const void *z, const void *U, void *state, void *y,
+                                  int B, int D, int G, int W, int R, bool bf16, cudaStream_t s);
+cudaError_t launch_decode(const void *x, const void *w, void *state, void *y, int B, int D, int G,
+                          int W, bool bf16, cudaStream_t s);
+
+// CUDA-core kernels (simt.cu)
 void launch_conv_dx(const void *w, bool w_is_f32, const void *dy, void *dx, int B, int T, int D,
                     int G, int W, bool bf16, bool is_static, cudaStream_t s);
-int static_dw_partials(int B, int T);
-void launch_static_dw(const void *x, const void *dy, float *part, float *dw, int B, int T, int D,
-                      int W, bool bf16, cudaStream_t s);
 void launch_dyn_dw(const void *x, const void *dy, float *dw, int B, int T, int D, int G, int W,
                    bool bf16, cudaStream_t s);
 void launch_lowrank_fwd_simt(const void *x, const void *z, const void *U, void *y, int B, int T,

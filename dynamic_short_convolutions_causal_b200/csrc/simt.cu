@@ -1,6 +1,7 @@
-// CUDA-core kernels: the HBM-streaming explicit and static convolutions (forward and
-// backward), and the general-shape low-rank path used where the tensor-core kernels
-// do not apply (fp32, or R / G / W outside the tensor-core shapes).
+// CUDA-core kernels: the explicit-filter backward (dx and the per-token filter
+// gradient), and the general-shape low-rank path used where the tensor-core kernels
+// do not apply (fp32, or R / G / W outside the tensor-core shapes).  The forward
+// kernels and the static backward are in stream.cu.
 //
 // The operation is the causal dynamic short convolution of "Convolucoes Curtas
 // Dinamicas Melhoram Transformers" (Metodologia > Convolucoes Curtas Dinamicas):
@@ -57,59 +58,6 @@ __device__ __forceinline__ void load_taps(const TW *__restrict__ w, size_t bt, i
 #pragma unroll
             for (int k = 0; k < W; ++k) f[k][i] = to_f(p[k]);
         }
-    }
-}
-
-// ------------------------------------------------------------------ forward
-template <typename T, int W, bool STATIC>
-__global__ void __launch_bounds__(128)
-k_conv_fwd(const T *__restrict__ x, const T *__restrict__ w, T *__restrict__ y,
-           int B, int T_, int D, int G, int chunk) {
-    constexpr int V = Vec<T>::N;
-    const int v = blockIdx.x * blockDim.x + threadIdx.x;
-    if (v >= D / V) return;
-    const int nchunks = cdiv(T_, chunk);
-    const int b = blockIdx.y / nchunks;
-    const int t0 = (blockIdx.y % nchunks) * chunk;
-    const int t1 = min(t0 + chunk, T_);
-    const int c0 = v * V;
-    const size_t row0 = (size_t)b * T_;
-
-    float win[W][V];   // win[k] = x_{t-k}; win[0] is filled each step
-#pragma unroll
-    for (int k = 1; k < W; ++k) {
-        const int t = t0 - k;
-        if (t >= 0) {
-            Vec<T>::load(x + (row0 + t) * D + c0, win[k]);
-        } else {
-#pragma unroll
-            for (int i = 0; i < V; ++i) win[k][i] = 0.f;
-        }
-    }
-    float f[W][V];
-    if (STATIC) {
-#pragma unroll
-        for (int i = 0; i < V; ++i)
-#pragma unroll
-            for (int k = 0; k < W; ++k) f[k][i] = to_f(w[(size_t)(c0 + i) * W + k]);
-    }
-    for (int t = t0; t < t1; ++t) {
-        const size_t bt = row0 + t;
-        Vec<T>::load(x + bt * D + c0, win[0]);
-        if (!STATIC) load_taps<T, T, W>(w, bt, c0, D, G, f);
-        float out[V];
-#pragma unroll
-        for (int i = 0; i < V; ++i) {
-            float acc = win[0][i];
-#pragma unroll
-            for (int k = 0; k < W; ++k) acc = fmaf(f[k][i], win[k][i], acc);
-            out[i] = acc;
-        }
-        Vec<T>::store(y + bt * D + c0, out);
-#pragma unroll
-        for (int k = W - 1; k >= 1; --k)
-#pragma unroll
-            for (int i = 0; i < V; ++i) win[k][i] = win[k - 1][i];
     }
 }
 
@@ -170,87 +118,6 @@ k_conv_bwd_dx(const TW *__restrict__ w, const T *__restrict__ dy, T *__restrict_
         const int row = tend - k;
         if (tend == T_ && row >= t0 && row < t1 && row > tend - W)
             Vec<T>::store(dx + (row0 + row) * D + c0, acc[k]);
-    }
-}
-
-// ------------------------------------------------------------------ static dw partials
-// Thread (vector v, token sub-chunk ty) accumulates dw[c,k] += dy_t[c] x_{t-k}[c] over its
-// tokens; the block sums its sub-chunks in a fixed order and writes one partial row
-// part[p, c, k] (p = blockIdx.y).
-template <typename T, int W>
-__global__ void __launch_bounds__(256)
-k_static_dw_partial(const T *__restrict__ x, const T *__restrict__ dy, float *__restrict__ part,
-                    int B, int T_, int D, int sub) {
-    constexpr int V = Vec<T>::N;
-    constexpr int BX = 32, BY = 8;
-    __shared__ float red[BY][BX][V];
-    const int v = blockIdx.x * BX + threadIdx.x;
-    const int per_block = BY * sub;
-    const int nblk = cdiv(T_, per_block);
-    const int b = blockIdx.y / nblk;
-    const int t0 = (blockIdx.y % nblk) * per_block + threadIdx.y * sub;
-    const int t1 = min(t0 + sub, T_);
-    const int c0 = v * V;
-    const bool active = v < D / V;
-    const size_t row0 = (size_t)b * T_;
-
-    float acc[W][V];
-#pragma unroll
-    for (int k = 0; k < W; ++k)
-#pragma unroll
-        for (int i = 0; i < V; ++i) acc[k][i] = 0.f;
-    if (active && t0 < t1) {
-        float win[W][V];
-#pragma unroll
-        for (int k = 1; k < W; ++k) {
-            const int t = t0 - k;
-            if (t >= 0) {
-                Vec<T>::load(x + (row0 + t) * D + c0, win[k]);
-            } else {
-#pragma unroll
-                for (int i = 0; i < V; ++i) win[k][i] = 0.f;
-            }
-        }
-        for (int t = t0; t < t1; ++t) {
-            const size_t bt = row0 + t;
-            float g[V];
-            Vec<T>::load(x + bt * D + c0, win[0]);
-            Vec<T>::load(dy + bt * D + c0, g);
-#pragma unroll
-            for (int k = 0; k < W; ++k)
-#pragma unroll
-                for (int i = 0; i < V; ++i) acc[k][i] = fmaf(g[i], win[k][i], acc[k][i]);
-#pragma unroll
-            for (int k = W - 1; k >= 1; --k)
-#pragma unroll
-                for (int i = 0; i < V; ++i) win[k][i] = win[k - 1][i];
-        }
-    }
-#pragma unroll
-    for (int k = 0; k < W; ++k) {
-#pragma unroll
-        for (int i = 0; i < V; ++i) red[threadIdx.y][threadIdx.x][i] = acc[k][i];
-        __syncthreads();
-        if (threadIdx.y == 0 && active) {
-#pragma unroll
-            for (int i = 0; i < V; ++i) {
-                float s = 0.f;
-                for (int y = 0; y < BY; ++y) s += red[y][threadIdx.x][i];
-                part[((size_t)blockIdx.y * D + c0 + i) * W + k] = s;
-            }
-        }
-        __syncthreads();
-    }
-}
-
-// out[e] = sum_{p < P} part[p * n + e], in order of p.
-__global__ void k_sum_partials(const float *__restrict__ part, float *__restrict__ out,
-                               int P, size_t n) {
-    for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n;
-         e += (size_t)gridDim.x * blockDim.x) {
-        float s = 0.f;
-        for (int p = 0; p < P; ++p) s += part[(size_t)p * n + e];
-        out[e] = s;
     }
 }
 
@@ -400,34 +267,6 @@ k_lowrank_dU(const T *__restrict__ z, const float *__restrict__ dw, float *__res
 // ------------------------------------------------------------------ launchers
 constexpr int kChunk = 32;
 
-template <typename T, bool STATIC>
-static void launch_fwd_T(const void *x, const void *w, void *y, int B, int T_, int D, int G, int W,
-                         cudaStream_t s) {
-    constexpr int V = Vec<T>::N;
-    const dim3 block(128);
-    const dim3 grid(cdiv(D / V, 128), B * cdiv(T_, kChunk));
-    const T *xp = (const T *)x;
-    const T *wp = (const T *)w;
-    T *yp = (T *)y;
-    switch (W) {
-#define DSC_CASE(WW) \
-    case WW: k_conv_fwd<T, WW, STATIC><<<grid, block, 0, s>>>(xp, wp, yp, B, T_, D, G, kChunk); break;
-        DSC_CASE(1) DSC_CASE(2) DSC_CASE(3) DSC_CASE(4) DSC_CASE(5) DSC_CASE(6) DSC_CASE(7) DSC_CASE(8)
-#undef DSC_CASE
-    }
-}
-
-void launch_conv_fwd(const void *x, const void *w, void *y, int B, int T, int D, int G, int W,
-                     bool bf16_, bool is_static, cudaStream_t s) {
-    if (bf16_) {
-        if (is_static) launch_fwd_T<bf16, true>(x, w, y, B, T, D, 1, W, s);
-        else launch_fwd_T<bf16, false>(x, w, y, B, T, D, G, W, s);
-    } else {
-        if (is_static) launch_fwd_T<float, true>(x, w, y, B, T, D, 1, W, s);
-        else launch_fwd_T<float, false>(x, w, y, B, T, D, G, W, s);
-    }
-}
-
 template <typename T, typename TW, bool STATIC>
 static void launch_dx_T(const void *w, const void *dy, void *dx, int B, int T_, int D, int G, int W,
                         cudaStream_t s) {
@@ -455,37 +294,6 @@ void launch_conv_dx(const void *w, bool w_is_f32, const void *dy, void *dx, int 
         if (is_static) launch_dx_T<float, float, true>(w, dy, dx, B, T, D, 1, W, s);
         else launch_dx_T<float, float, false>(w, dy, dx, B, T, D, G, W, s);
     }
-}
-
-constexpr int kStaticSub = 32;   // tokens per thread in the static dw partials
-constexpr int kStaticBY = 8;
-
-int static_dw_partials(int B, int T) { return B * cdiv(T, kStaticBY * kStaticSub); }
-
-template <typename T>
-static void launch_static_dw_T(const void *x, const void *dy, float *part, float *dw, int B, int T_,
-                               int D, int W, cudaStream_t s) {
-    constexpr int V = Vec<T>::N;
-    const dim3 block(32, kStaticBY);
-    const int P = static_dw_partials(B, T_);
-    const dim3 grid(cdiv(D / V, 32), P);
-    const T *xp = (const T *)x;
-    const T *gp = (const T *)dy;
-    switch (W) {
-#define DSC_CASE(WW) \
-    case WW: k_static_dw_partial<T, WW><<<grid, block, 0, s>>>(xp, gp, part, B, T_, D, kStaticSub); break;
-        DSC_CASE(1) DSC_CASE(2) DSC_CASE(3) DSC_CASE(4) DSC_CASE(5) DSC_CASE(6) DSC_CASE(7) DSC_CASE(8)
-#undef DSC_CASE
-    }
-    const size_t n = (size_t)D * W;
-    k_sum_partials<<<(unsigned)std::min<size_t>(cdiv((int)std::min<size_t>(n, 1u << 30), 256), 4096), 256, 0, s>>>(
-        part, dw, P, n);
-}
-
-void launch_static_dw(const void *x, const void *dy, float *part, float *dw, int B, int T, int D,
-                      int W, bool bf16_, cudaStream_t s) {
-    if (bf16_) launch_static_dw_T<bf16>(x, dy, part, dw, B, T, D, W, s);
-    else launch_static_dw_T<float>(x, dy, part, dw, B, T, D, W, s);
 }
 
 void launch_dyn_dw(const void *x, const void *dy, float *dw, int B, int T, int D, int G, int W,

@@ -8,21 +8,43 @@
 //   dz[t,r]   = sum_j dw[t,j] U[r,j]
 //   dU[r,j]   = sum_t z[t,r] dw[t,j]
 // The filters are recomputed from z and U rather than stored (storing them would move
-// W/G times the bytes of x).
+// W/G times the bytes of x), and dw never leaves the chip ("Implementacao de
+// Treinamento Eficiente": the kernels write only the final results to HBM).
 //
-// Work tile = 128 tokens of one sequence x one 64-channel slice.  Per tile:
-//   1. recompute, one MMA per tap k with the z tile shifted by k rows:
-//        Wk[t, g] = sum_r z[t0+t+k, r] Up[r, k*NG+g]   (Up: U with the slice's columns
-//      reordered tap-major by a pre-pass), so TMEM lane t holds w[t+k, g, k] for every k;
-//   2. epilogue (one token row per thread): dx and dw on CUDA cores; dx is stored by TMA,
-//      dw (bf16) is written to shared memory;
-//   3. dz partial = dw Up^T   (A = dw tile, B = Up slice, M=128 tokens, N=R);
-//      dU^T     += dw^T z     (A = the same tile read MN-major, B = z tile, M=128 columns,
-//      N=R), accumulated in TMEM over all tiles of the slice that the CTA processes.
-//   Recompute, dz and dU are issued by three MMA warps, each on its own SM sub-partition.
-// Persistent CTAs own contiguous tile ranges in slice-major order.  dz partials (per
-// slice) and dU partials (per CTA segment of a slice) go to the workspace and are summed
-// in a fixed order by one small kernel, so results are deterministic.
+// Work tile = 128 tokens of one sequence ("token tile") x one 64-channel slice.
+//
+// Schedule (one persistent CTA per SM, cooperative launch).  The grid is A x Bg
+// CTAs: CTA (a, b) owns the token tiles of range a and the S slices of group b, and
+// walks them token tile by token tile, its S slices innermost.  Hence
+//   - dz of a token tile accumulates over the CTA's S slices in TMEM and leaves the
+//     CTA once, as one partial of Bg;
+//   - dU of each of its slices accumulates over all its token tiles in TMEM and
+//     leaves the CTA once, as one partial of A.
+// The Bg CTAs of a token range move through the same token tiles at the same pace, so
+// the partials of a token tile are written close together in time and are summed
+// while they are still in L2: after writing its partial of token tile m, each CTA
+// counts itself in on a per-tile counter, and a reducer warp in every CTA sums its
+// share of the tile's rows (slice groups in a fixed order) once all Bg partials are
+// in.  The A dU partials of each slice group are summed the same way at the end.
+// Every sum runs in a fixed order, so results are deterministic.
+//
+// Per tile (token tile m, slice s) the CTA's warps do:
+//   warp 0      TMA: dy and x tiles (3-stage ring), z once per token tile, the
+//               tap-major U slice Up (resident when the CTA has at most two slices);
+//               TMA store of dx from the stage once the epilogue has written it there
+//   warp 1      recompute: one MMA per tap k with the z tile shifted by k rows,
+//                 Wk[t, g] = sum_r z[t0+t+k, r] Up[r, k*NG+g],
+//               so TMEM lane t holds w[t+k, g, k] for every k
+//   warp 2      dz[m] += dw Up^T  (A = dw tile, B = Up slice; M=128 tokens, N=R) and
+//               dU^T[s] += dw^T z  (A = dw tile read MN-major, B = z; M=128 columns)
+//   warp 3      reducer: sums the dz partials of its rows of each token tile
+//   warps 4-19  epilogue, one token row per thread, 16 channels per warp:
+//                 A2: dw (bf16) into the shared-memory dw tile;
+//                 A1: dx, written over the stage's x tile (dead after A2);
+//                 after a token tile's last slice: its dz partial to global memory
+// The recompute of tile i runs during A2 of tile i, and the dz/dU MMAs of tile i
+// during A1 of tile i.  Every wait is bounded (one second); a wait that runs out
+// makes the CTA leave its loops, record a fault code and free its TMEM.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -42,24 +64,16 @@ __device__ unsigned int g_fault_bwd = 0;
 
 constexpr int kTt = 128;
 constexpr int kDt = 64;
-// Epilogue geometry: 16 warps of 16 channels (4 TMEM lane quarters x 4 channel groups).
-// (8 warps of 32 channels, with 168 registers a thread, measured slower at G=4, W=8:
-// 0.76 against 0.74 ms on the lowrank_mlp backward.)
-// Warp roles: 0 TMA producer, 1 recompute MMAs, 2..1+E epilogue, 2+E dz MMAs, 3+E dU MMAs.
-// The three MMA streams are issued from warps on three different SM sub-partitions: one
-// warp issuing all of them shares its issue slots with the busy epilogue warps and cannot
-// keep the tensor pipe fed.
-template <int G>
-struct Geo {
-    static constexpr int kEpiWarps = 16;
-    static constexpr int kGroups = kEpiWarps / 4;      // channel groups of a slice
-    static constexpr int kCPW = kDt / kGroups;         // channels per epilogue warp
-    static constexpr int kDxBuf = 32 * kCPW * 2;       // one warp's dx staging: 32 rows x kCPW bf16
-    static constexpr int kDzWarp = 2 + kEpiWarps;
-    static constexpr int kDuWarp = 3 + kEpiWarps;
-    static constexpr int kThreads = 32 * (4 + kEpiWarps);
-};
-constexpr uint32_t kDxStageBytes = 4 * 32 * kDt * 2;   // all epilogue warps' dx staging
+constexpr int kEpiWarps = 16;                   // 4 TMEM lane quarters x 4 channel groups
+constexpr int kCPW = kDt / 4;                   // channels per epilogue warp
+// Warp roles.  Warps 0-3 sit on the SM's four sub-partitions, one each, and the
+// epilogue warps 4-19 four to a sub-partition; 20 warps keep 96 registers a thread.
+constexpr int kRecWarp = 1;
+constexpr int kMmaWarp = 2;                     // dz and dU MMAs
+constexpr int kRedWarp = 3;
+constexpr int kEpi0 = 4;
+constexpr int kThreads = 32 * (kEpi0 + kEpiWarps);
+constexpr int kMaxStages = 3;
 
 struct BwdParams {
     int B, T, D, G, W, R;
@@ -67,35 +81,45 @@ struct BwdParams {
     int NGp;                  // TMEM columns per tap block (NGs rounded up to 16)
     int SC;                   // filter columns per slice (NGs*W)
     int SCp;                  // SC rounded up to 128 (dU^T M-blocks)
-    int n_slices, tiles_per_seq, per_slice, n_tiles, maxseg;
+    int n_slices, tiles_per_seq, n_tt;
+    int A, Bg;                // token ranges x slice groups = grid
     int u_boxes;              // TMA boxes of 64 Up columns per slice
-    int nU, stages;
+    int stages, nU;           // ring depth; Up buffers (1 or 2)
     uint32_t rows;            // tile rows incl. halo: 128 + W - 1
     uint32_t xy_tile_bytes;   // one dy or x tile (rows x 128 B), 1024-aligned
-    uint32_t z_slab;          // stride of the 8-wide z slabs (rows x 16 B, rounded up to 128:
-                              // a TMA destination must be 128-byte aligned)
-    uint32_t z_bytes;         // R/8 slabs
-    uint32_t u_bytes;
-    uint32_t stage_bytes;     // dy tile + x tile + z tile
-    uint32_t off_u, off_dw, off_dx, off_bar;
-    uint32_t tm_w, tm_dw, tm_dz, tm_du, tmem_cols;   // TMEM column map
-    float *dz_part;           // [n_slices][B*T][R]
-    float *du_part;           // [n_slices][maxseg][R][SC]
+    uint32_t z_slab;          // stride of the 8-wide z slabs (rows x 16 B, rounded up to 128)
+    uint32_t z_bytes;         // one z buffer (R/8 slabs), 1024-aligned
+    uint32_t u_bytes;         // one Up buffer
+    uint32_t stage_bytes;     // dy tile + x tile
+    uint32_t off_z, off_u, off_dw, off_bar;
+    uint32_t tm_w, tm_dz, tm_du, tmem_cols;   // TMEM column map
+    float *dz_part;           // [Bg][B*T][R]
+    float *du_part;           // [A][R][N]
+    unsigned *flag_dz;        // [n_tt] partials written per token tile (16 per CTA)
+    unsigned *flag_du;        // [Bg]   dU partials written per slice group (16 per CTA)
+    float *dz;                // [B*T][R]
+    float *dU;                // [R][N]
 };
 
 struct Bars {
     uint32_t base;
     __device__ uint32_t full(int s) const { return base + 8 * s; }
-    __device__ uint32_t empty(int s) const { return base + 8 * (3 + s); }
-    __device__ uint32_t uf(int u) const { return base + 8 * (6 + u); }
-    __device__ uint32_t ue(int u) const { return base + 8 * (8 + u); }
-    __device__ uint32_t wfull() const { return base + 8 * 10; }
-    __device__ uint32_t wempty() const { return base + 8 * 11; }
-    __device__ uint32_t dwready() const { return base + 8 * 12; }
-    __device__ uint32_t mm2() const { return base + 8 * 13; }
-    __device__ uint32_t done() const { return base + 8 * 14; }
+    __device__ uint32_t dxr(int s) const { return base + 8 * (3 + s); }
+    __device__ uint32_t zfull(int z) const { return base + 8 * (6 + z); }
+    __device__ uint32_t zempty(int z) const { return base + 8 * (8 + z); }
+    __device__ uint32_t ufull(int u) const { return base + 8 * (10 + u); }
+    __device__ uint32_t uempty(int u) const { return base + 8 * (12 + u); }
+    __device__ uint32_t wfull() const { return base + 8 * 14; }
+    __device__ uint32_t wempty() const { return base + 8 * 15; }
+    __device__ uint32_t dwready() const { return base + 8 * 16; }
+    __device__ uint32_t dwfree() const { return base + 8 * 17; }
+    __device__ uint32_t dzfull(int d) const { return base + 8 * (18 + d); }
+    __device__ uint32_t dzempty(int d) const { return base + 8 * (20 + d); }
+    __device__ uint32_t dufull() const { return base + 8 * 22; }
+    __device__ uint32_t done() const { return base + 8 * 23; }
+    __device__ uint32_t xdead() const { return base + 8 * 24; }
 };
-constexpr uint32_t kBarBytes = 8 * 15;
+constexpr uint32_t kBarBytes = 8 * 25;
 
 __device__ __forceinline__ void unpack8(const uint4 &u, float (&v)[8]) {
     v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x);
@@ -104,16 +128,6 @@ __device__ __forceinline__ void unpack8(const uint4 &u, float (&v)[8]) {
     v[6] = bf16_lo(u.w); v[7] = bf16_hi(u.w);
 }
 
-template <int N> __device__ __forceinline__ void tmem_st_n(uint32_t a, const uint32_t *r);
-template <> __device__ __forceinline__ void tmem_st_n<1>(uint32_t a, const uint32_t *r) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(a), "r"(r[0]) : "memory");
-}
-template <> __device__ __forceinline__ void tmem_st_n<2>(uint32_t a, const uint32_t *r) {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1, %2};" ::"r"(a), "r"(r[0]), "r"(r[1])
-                 : "memory");
-}
-template <> __device__ __forceinline__ void tmem_st_n<4>(uint32_t a, const uint32_t *r) { tmem_st<4>(a, r); }
-
 __device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
@@ -121,33 +135,68 @@ __device__ __forceinline__ void sts64(uint32_t addr, uint32_t a, uint32_t b) {
     asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(addr), "r"(a), "r"(b) : "memory");
 }
 
-// Tile index -> (slice, sequence, first token)
-struct TileId {
-    int slice, b, t0;
-};
-__device__ __forceinline__ TileId tile_id(const BwdParams &p, int i) {
-    TileId id;
-    id.slice = i / p.per_slice;
-    const int rem = i - id.slice * p.per_slice;
-    id.b = rem / p.tiles_per_seq;
-    id.t0 = (rem - id.b * p.tiles_per_seq) * kTt;
-    return id;
+// ------------------------------------------------------------------ global counters
+// A writer's stores become visible before its count: every lane fences, the warp
+// synchronises, one lane adds with release semantics.  A reader polls with acquire
+// semantics (every lane), then reads the data through L2.
+__device__ __forceinline__ void fence_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
+
+__device__ __forceinline__ void red_release_add(unsigned *p, unsigned v) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// CTA that owns tile i when n tiles are split into contiguous ranges over g CTAs
-// (CTA c owns [c*n/g, (c+1)*n/g)).
-__host__ __device__ inline int owner_of(long long i, long long n, long long g) {
-    return (int)(((i + 1) * g - 1) / n);
+__device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Waits until *p >= target.  Gives up like mbar_wait: after kWaitLimitNs, or as soon
+// as another warp of the CTA has given up.
+__device__ __forceinline__ bool wait_count(const unsigned *p, unsigned target, volatile int *abort,
+                                           unsigned code) {
+    if (ld_acquire(p) >= target) return true;
+    const unsigned long long t0 = globaltimer();
+    while (true) {
+#pragma unroll 1
+        for (int i = 0; i < 16; ++i) {
+            __nanosleep(100);
+            if (ld_acquire(p) >= target) return true;
+        }
+        if (*abort) return false;
+        if (globaltimer() - t0 > kWaitLimitNs) {
+            *abort = 1;
+            atomicOr(&g_fault_bwd, code);
+            return false;
+        }
+    }
+}
+
+// Which token tiles and slices a CTA owns.
+struct Span {
+    int a, b;                 // token range, slice group
+    int m0, m1, s0, s1;       // token tiles [m0, m1), slices [s0, s1)
+    __device__ int S() const { return s1 - s0; }
+    __device__ int tiles() const { return (m1 - m0) * (s1 - s0); }
+};
+__device__ __forceinline__ Span span_of(const BwdParams &p) {
+    Span s;
+    s.a = (int)blockIdx.x / p.Bg;
+    s.b = (int)blockIdx.x - s.a * p.Bg;
+    s.m0 = (int)((long long)s.a * p.n_tt / p.A);
+    s.m1 = (int)((long long)(s.a + 1) * p.n_tt / p.A);
+    s.s0 = (int)((long long)s.b * p.n_slices / p.Bg);
+    s.s1 = (int)((long long)(s.b + 1) * p.n_slices / p.Bg);
+    return s;
 }
 
 template <int W, int G>
-__global__ void __launch_bounds__(Geo<G>::kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 1)
 k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ CUtensorMap tm_x,
                  const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_u,
                  const __grid_constant__ CUtensorMap tm_dx, const BwdParams p) {
     constexpr int NG8 = 8 / G;          // filter groups in one 8-channel chunk
-    constexpr int kEpiWarps = Geo<G>::kEpiWarps, kCPW = Geo<G>::kCPW, kDxBuf = Geo<G>::kDxBuf;
-    constexpr int kDzWarp = Geo<G>::kDzWarp, kDuWarp = Geo<G>::kDuWarp, kThreads = Geo<G>::kThreads;
+    constexpr int CH = kCPW / 8;        // 16-byte chunks of a warp's channels in a row
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     const uint32_t sb = smem_u32(smem);
@@ -156,21 +205,32 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
     const Bars bar{sb + p.off_bar};
     uint32_t *tmem_holder = (uint32_t *)(smem + p.off_bar + kBarBytes);
     volatile int *abort = (volatile int *)(smem + p.off_bar + kBarBytes + 8);
+    const Span sp = span_of(p);
+    const int S = sp.S();
+    const int nt = sp.tiles();
+    const int NST = p.stages;
+    const bool u_res = S <= p.nU;       // Up slices stay resident: buffer j holds slice s0+j
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < p.stages; ++s) {
+        for (int s = 0; s < NST; ++s) {
             mbar_init(bar.full(s), 1);
-            mbar_init(bar.empty(s), kEpiWarps);
+            mbar_init(bar.dxr(s), kEpiWarps);
         }
-        for (int u = 0; u < 2; ++u) {
-            mbar_init(bar.uf(u), 1);
-            mbar_init(bar.ue(u), 2);        // recompute and dz streams
+        for (int z = 0; z < 2; ++z) {
+            mbar_init(bar.zfull(z), 1);
+            mbar_init(bar.zempty(z), 2);        // recompute and dz/dU streams
+            mbar_init(bar.ufull(z), 1);
+            mbar_init(bar.uempty(z), 2);        // recompute and dz/dU streams
+            mbar_init(bar.dzfull(z), 1);
+            mbar_init(bar.dzempty(z), kEpiWarps);
         }
         mbar_init(bar.wfull(), 1);
         mbar_init(bar.wempty(), kEpiWarps);
         mbar_init(bar.dwready(), kEpiWarps);
-        mbar_init(bar.mm2(), 2);            // dz and dU streams
-        mbar_init(bar.done(), 3);           // all three MMA streams
+        mbar_init(bar.dwfree(), 1);
+        mbar_init(bar.dufull(), 1);
+        mbar_init(bar.done(), 2);               // recompute and dz/dU streams
+        mbar_init(bar.xdead(), kEpiWarps);      // every epilogue warp is past A2
         *abort = 0;
         fence_barrier_init();
     }
@@ -189,7 +249,7 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
         tma_prefetch(&tm_u);
         tma_prefetch(&tm_dx);
     }
-    if (warp == 1) {
+    if (warp == kRecWarp) {
         tmem_alloc(smem_u32(tmem_holder), p.tmem_cols);
         tmem_relinquish();
     }
@@ -197,71 +257,101 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-
-    const int tbeg = (int)((long long)blockIdx.x * p.n_tiles / gridDim.x);
-    const int tend = (int)((long long)(blockIdx.x + 1) * p.n_tiles / gridDim.x);
+    const int nmb = p.SCp / 128;        // dU^T M-blocks per slice
 
     if (warp == 0) {
         // ---------------------------------------------------------- TMA producer
         if (lane == 0) {
-            int prev = -1, v = -1;
-            const uint32_t tx = 2 * p.rows * 128 + (uint32_t)(p.R / 8) * p.rows * 16;   // bytes TMA delivers
-            for (int i = tbeg; i < tend; ++i) {
-                const int it = i - tbeg;
-                const TileId id = tile_id(p, i);
-                if (id.slice != prev) {
-                    prev = id.slice;
-                    ++v;
-                    const int ub = v % p.nU, un = v / p.nU;
-                    if (!mbar_wait(bar.ue(ub), (un & 1) ^ 1, abort, 1u, &g_fault_bwd)) break;
-                    mbar_arrive_expect_tx(bar.uf(ub), p.u_bytes);
-                    const uint32_t ud = sb + p.off_u + ub * p.u_bytes;
-                    for (int bx = 0; bx < p.u_boxes; ++bx)
-                        tma_load_2d(ud + bx * (uint32_t)(p.R * 128), &tm_u, bar.uf(ub),
-                                    id.slice * p.SC + 64 * bx, 0);
+            const uint32_t tx_xy = 2 * p.rows * 128;
+            const uint32_t tx_z = (uint32_t)(p.R / 8) * p.rows * 16;
+            auto load_up = [&](int ub, int slice) {
+                mbar_arrive_expect_tx(bar.ufull(ub), p.u_bytes);
+                const uint32_t ud = sb + p.off_u + ub * p.u_bytes;
+                for (int bx = 0; bx < p.u_boxes; ++bx)
+                    tma_load_2d(ud + bx * (uint32_t)(p.R * 128), &tm_u, bar.ufull(ub), slice * p.SC + 64 * bx, 0);
+            };
+            auto store_dx = [&](int i) {      // dx of tile i, from its stage's x region
+                const int m = sp.m0 + i / S, slice = sp.s0 + i % S;
+                const int b = m / p.tiles_per_seq, t0 = (m - b * p.tiles_per_seq) * kTt;
+                tma_store_3d(&tm_dx, sb + (i % NST) * p.stage_bytes + p.xy_tile_bytes, slice * kDt, t0, b);
+                bulk_commit();
+            };
+            int issued = 0, zissued = 0, uissued = 0;
+            bool ok = true;
+            if (u_res)
+                for (int j = 0; j < S; ++j) { load_up(j, sp.s0 + j); ++uissued; }
+            for (int i = 0; i < nt && ok; ++i) {
+                const int st = i % NST, n = i / NST;
+                const int j = i % S, mz = i / S;
+                const int m = sp.m0 + mz, slice = sp.s0 + j;
+                const int b = m / p.tiles_per_seq, t0 = (m - b * p.tiles_per_seq) * kTt;
+                if (i >= NST) {
+                    // the stage is free once tile i-NST's dx, written over its x tile, is stored
+                    if (!mbar_wait(bar.dxr(st), (n - 1) & 1, abort, 1u, &g_fault_bwd)) { ok = false; break; }
+                    store_dx(i - NST);
+                    bulk_wait_read<0>();
                 }
-                const int s = it % p.stages, n = it / p.stages;
-                if (!mbar_wait(bar.empty(s), (n & 1) ^ 1, abort, 2u, &g_fault_bwd)) break;
-                mbar_arrive_expect_tx(bar.full(s), tx);
-                const uint32_t st = sb + s * p.stage_bytes;
-                tma_load_3d(st, &tm_dy, bar.full(s), id.slice * kDt, id.t0, id.b);
-                tma_load_3d(st + p.xy_tile_bytes, &tm_x, bar.full(s), id.slice * kDt, id.t0 - (W - 1), id.b);
-                for (int j = 0; j < p.R / 8; ++j)
-                    tma_load_3d(st + 2 * p.xy_tile_bytes + j * p.z_slab, &tm_z, bar.full(s), 8 * j, id.t0, id.b);
+                if (j == 0) {
+                    const int zb = mz & 1;
+                    if (!mbar_wait(bar.zempty(zb), ((mz >> 1) & 1) ^ 1, abort, 2u, &g_fault_bwd)) { ok = false; break; }
+                    mbar_arrive_expect_tx(bar.zfull(zb), tx_z);
+                    const uint32_t zd = sb + p.off_z + zb * p.z_bytes;
+                    for (int r8 = 0; r8 < p.R / 8; ++r8)
+                        tma_load_3d(zd + r8 * p.z_slab, &tm_z, bar.zfull(zb), 8 * r8, t0, b);
+                    ++zissued;
+                }
+                if (!u_res) {
+                    const int ub = i & 1;
+                    if (!mbar_wait(bar.uempty(ub), ((i >> 1) & 1) ^ 1, abort, 2u, &g_fault_bwd)) { ok = false; break; }
+                    load_up(ub, slice);
+                    ++uissued;
+                }
+                mbar_arrive_expect_tx(bar.full(st), tx_xy);
+                const uint32_t sd = sb + st * p.stage_bytes;
+                tma_load_3d(sd, &tm_dy, bar.full(st), slice * kDt, t0, b);
+                tma_load_3d(sd + p.xy_tile_bytes, &tm_x, bar.full(st), slice * kDt, t0 - (W - 1), b);
+                ++issued;
             }
-            const int issued = tend - tbeg;
-            for (int s = 0; s < p.stages && s < issued; ++s) {
-                const int last = issued - 1 - ((issued - 1 - s) % p.stages);
-                mbar_wait(bar.full(s), (last / p.stages) & 1, abort, 0u, &g_fault_bwd);
+            if (ok) {
+                for (int i = (nt > NST ? nt - NST : 0); i < nt; ++i) {
+                    if (!mbar_wait(bar.dxr(i % NST), (i / NST) & 1, abort, 1u, &g_fault_bwd)) break;
+                    store_dx(i);
+                }
+            }
+            bulk_wait_all();
+            // Let every load this warp issued land before the CTA can exit (matters only
+            // when another warp gave up early; otherwise all of them were consumed).
+            for (int i = (issued > NST ? issued - NST : 0); i < issued; ++i)
+                mbar_drain(bar.full(i % NST), (i / NST) & 1);
+            for (int z = (zissued > 2 ? zissued - 2 : 0); z < zissued; ++z)
+                mbar_drain(bar.zfull(z & 1), (z >> 1) & 1);
+            if (u_res) {
+                for (int u = 0; u < uissued; ++u) mbar_drain(bar.ufull(u), 0);
+            } else {
+                for (int u = (uissued > 2 ? uissued - 2 : 0); u < uissued; ++u)
+                    mbar_drain(bar.ufull(u & 1), (u >> 1) & 1);
             }
         }
         __syncwarp();
-    } else if (warp == 1) {
+    } else if (warp == kRecWarp) {
         // ---------------------------------------------------------- MMA issuer: recompute
         // Each MMA warp runs its schedule warp-uniformly; one elected lane issues each
         // tcgen05 instruction, and descriptors advance by adding to their start field.
-        // Tile i's filters are recomputed once the epilogue has read those of tile i-1.
         const uint64_t t_zk = desc_tmpl(p.z_slab, 128, kSwNone);               // z, K-major, no swizzle
         const uint64_t t_u_mn = desc_tmpl((uint32_t)(p.R * 128), 1024, kSw128);  // Up as MN-major B
         const uint32_t i_rec = idesc_bf16(128, p.NGp, false, true);
         const int ksr = p.R / 16;
         const uint32_t ubox = (uint32_t)(p.R * 128);
         const uint64_t st_zk = (2 * p.z_slab) >> 4;   // 16 more z columns (start field units)
-        int prev_slice = -1, v = -1, ub = 0;
-        for (int i = tbeg; i < tend; ++i) {
-            const int it = i - tbeg;
-            const TileId id = tile_id(p, i);
-            if (id.slice != prev_slice) {
-                prev_slice = id.slice;
-                ++v;
-                ub = v % p.nU;
-                if (!warp_wait(bar.uf(ub), (v / p.nU) & 1, abort, 4u, &g_fault_bwd)) break;
-            }
-            const int s = it % p.stages, n = it / p.stages;
-            if (!warp_wait(bar.full(s), n & 1, abort, 8u, &g_fault_bwd)) break;
-            if (!warp_wait(bar.wempty(), (it & 1) ^ 1, abort, 16u, &g_fault_bwd)) break;
+        for (int i = 0; i < nt; ++i) {
+            const int j = i % S, mz = i / S, zb = mz & 1;
+            const int ub = u_res ? j : (i & 1);
+            const int upar = u_res ? 0 : ((i >> 1) & 1);
+            if (j == 0 && !warp_wait(bar.zfull(zb), (mz >> 1) & 1, abort, 4u, &g_fault_bwd)) break;
+            if (!warp_wait(bar.ufull(ub), upar, abort, 4u, &g_fault_bwd)) break;
+            if (!warp_wait(bar.wempty(), (i & 1) ^ 1, abort, 16u, &g_fault_bwd)) break;
             tc_fence_after();
-            const uint32_t zs = sb + s * p.stage_bytes + 2 * p.xy_tile_bytes;
+            const uint32_t zs = sb + p.off_z + zb * p.z_bytes;
             const uint32_t us = sb + p.off_u + ub * p.u_bytes;
 #pragma unroll
             for (int k = 0; k < W; ++k) {
@@ -276,28 +366,23 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
                     db += 2048u >> 4;
                 }
             }
-            const bool last_of_slice = (i + 1 == tend) || ((i + 1) / p.per_slice != id.slice);
             if (elect_one()) {
                 mma_commit(bar.wfull());
-                if (last_of_slice) mma_commit(bar.ue(ub));
+                if (j == S - 1) mma_commit(bar.zempty(zb));
+                if (!u_res) mma_commit(bar.uempty(ub));
             }
             __syncwarp();
         }
         if (elect_one()) mma_commit(bar.done());
         __syncwarp();
-    } else if (warp < kDzWarp) {
+    } else if (warp >= kEpi0) {
         // ---------------------------------------------------------- epilogue
-        // Per tile i:  A1(i) dx  ->  B(i-1) dz partial, dU flush, stage release  ->  A2(i) dw.
-        const int ew = warp - 2;
+        const int ew = warp - kEpi0;
         const int q = warp & 3;              // TMEM lane quarter == token rows 32q..32q+31
         const int h = ew >> 2;               // channel group of the slice (kCPW channels)
         const int row = 32 * q + lane;
-        constexpr int CH = kCPW / 8;         // 16-byte chunks of the warp's channels in a row
-        const uint32_t dxstage = sb + p.off_dx + (uint32_t)ew * kDxBuf;
-        // staging rows of kCPW*2 bytes in the TMA store's 32- or 64-byte swizzle: the 16-byte
-        // chunk index is XORed with address bits 7.. of the row start
-        const uint32_t dxrow = (dxstage + lane * (2 * kCPW)) ^ ((((uint32_t)lane * (2 * kCPW) >> 7) & (CH - 1)) << 4);
-        // dy rows r = row + k and x rows r = row + W-1-k of the 128-byte-swizzled tiles
+        // dy rows r = row + k and x rows r = row + W-1-k of the 128-byte-swizzled tiles;
+        // dx of row `row` is written to row `row` of the x tile
         uint32_t dyr[W], xr[W];
 #pragma unroll
         for (int k = 0; k < W; ++k) {
@@ -306,342 +391,355 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             r = (uint32_t)(row + (W - 1) - k);
             xr[k] = (r * 128u) ^ ((r & 7u) << 4) ^ ((uint32_t)(CH * h) << 4);
         }
+        const uint32_t dxr0 = ((uint32_t)row * 128u) ^ (((uint32_t)row & 7u) << 4) ^ ((uint32_t)(CH * h) << 4);
         // dw^T shared-memory tile: MN-major, 128B swizzle, atoms of 64 columns x 128 rows
         const uint32_t dwrow = sb + p.off_dw + (uint32_t)row * 128u;
         const uint32_t dwsw = (uint32_t)(row & 7) << 4;
         const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
+        const int nc = p.R / 4;              // dz columns a warp reads out (its group's share)
 
-        struct Prev {
-            int it, s, slice, b, t0, seg;
-            bool last_of_slice;
-        } pv = {-1, 0, 0, 0, 0, 0, false};
-        // B: dz partial of a finished tile, its slice segment's dU partial, stage release
-        auto phase_b = [&](const Prev &t) -> bool {
-            if (!warp_wait(bar.mm2(), t.it & 1, abort, 256u, &g_fault_bwd)) return false;
+        // dz partial of token tile mz (this CTA's slices) -> global memory; count in.
+        auto dz_out = [&](int mz) -> bool {
+            const int db = mz & 1;
+            if (!warp_wait(bar.dzfull(db), (mz >> 1) & 1, abort, 256u, &g_fault_bwd)) return false;
             tc_fence_after();
-            {
-                // dz partial: every warp reads its group's share of the columns of its 32 rows
-                const int tok = t.t0 + row;
-                const int nc = p.R / Geo<G>::kGroups;
-                float *dst = p.dz_part + ((size_t)t.slice * p.B * p.T + (size_t)t.b * p.T + tok) * p.R + h * nc;
-                int c0 = 0;
+            const int m = sp.m0 + mz;
+            const int b = m / p.tiles_per_seq, t0 = (m - b * p.tiles_per_seq) * kTt;
+            const int tok = t0 + row;
+            float *dst = p.dz_part + ((size_t)sp.b * p.B * p.T + (size_t)b * p.T + tok) * p.R + h * nc;
+            const uint32_t src = tl + p.tm_dz + db * p.R + h * nc;
 #pragma unroll 1
-                for (; c0 + 8 <= nc; c0 += 8) {
-                    uint32_t v[8];
-                    tmem_ld<8>(tl + p.tm_dz + h * nc + c0, v);
-                    tmem_wait_ld_regs(v);
-                    if (tok < p.T) {
-                        *reinterpret_cast<uint4 *>(dst + c0) = make_uint4(v[0], v[1], v[2], v[3]);
-                        *reinterpret_cast<uint4 *>(dst + c0 + 4) = make_uint4(v[4], v[5], v[6], v[7]);
-                    }
-                }
-                if (c0 < nc) {   // nc = 4 (R = 16 with four channel groups)
-                    uint32_t v[4];
-                    tmem_ld<4>(tl + p.tm_dz + h * nc + c0, v);
-                    tmem_wait_ld_regs(v);
-                    if (tok < p.T) *reinterpret_cast<uint4 *>(dst + c0) = make_uint4(v[0], v[1], v[2], v[3]);
-                }
-            }
-            if (t.last_of_slice && h < p.SCp / 128) {
-                // lane j' of dU^T M-block h -> natural column g*W + k
-                const int jp = 128 * h + row;
-                const int jn = (jp % p.NGs) * W + jp / p.NGs;
-                float *dst = p.du_part + ((size_t)t.slice * p.maxseg + t.seg) * p.R * p.SC + jn;
-#pragma unroll 1
-                for (int c0 = 0; c0 < p.R; c0 += 16) {
-                    uint32_t v[16];
-                    tmem_ld<16>(tl + p.tm_du + h * p.R + c0, v);     // all lanes: warp-collective
-                    tmem_wait_ld_regs(v);
-                    if (jp < p.SC) {
-#pragma unroll
-                        for (int m2 = 0; m2 < 16; ++m2) dst[(size_t)(c0 + m2) * p.SC] = __uint_as_float(v[m2]);
-                    }
-                }
+            for (int c0 = 0; c0 < nc; c0 += 4) {
+                uint32_t v[4];
+                tmem_ld<4>(src + c0, v);
+                tmem_wait_ld_regs(v);
+                if (tok < p.T) *reinterpret_cast<uint4 *>(dst + c0) = make_uint4(v[0], v[1], v[2], v[3]);
             }
             tc_fence_before();
+            fence_gpu();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar.empty(t.s));
+            if (lane == 0) {
+                mbar_arrive(bar.dzempty(db));
+                red_release_add(p.flag_dz + m, 1u);
+            }
             return true;
         };
 
-        int prev_slice = -1, seg = 0;
         bool ok = true;
-        for (int i = tbeg; i < tend; ++i) {
-            const int it = i - tbeg;
-            const TileId id = tile_id(p, i);
-            if (id.slice != prev_slice) {
-                prev_slice = id.slice;
-                seg = (int)blockIdx.x - owner_of((long long)id.slice * p.per_slice, p.n_tiles, gridDim.x);
-            }
-            const int s = it % p.stages, n = it / p.stages;
-            if (!warp_wait(bar.full(s), n & 1, abort, 64u, &g_fault_bwd)) { ok = false; break; }
-            const uint32_t st = sb + s * p.stage_bytes;
-            const uint32_t dys = st, xs = st + p.xy_tile_bytes;
-            // ---- A1: dx[t,c] = dy[t,c] + sum_k w[t+k,g,k] dy[t+k,c]
-            // The warp's 16 channels are two 8-channel chunks, taken in batches of CB chunks:
-            // a batch's shared-memory and TMEM loads are all issued before its first store
-            // (the stores are ordered asm statements and would otherwise serialise the
-            // loads); with many taps one chunk per batch keeps the registers in budget, and
-            // the batch loop stays rolled so that the many-tap body fits the instruction cache.
-            // A single batch's dy rows are loaded before the wait for the recomputed filters.
-            constexpr int CB = (W * CH <= 8) ? CH : 1;
-            constexpr int NGB = 8 * CB / G;                 // filter groups of a batch
-            uint4 dpre[CB][W];
-            if constexpr (CB == CH) {
-#pragma unroll
-                for (int cb = 0; cb < CB; ++cb)
-#pragma unroll
-                    for (int k = 0; k < W; ++k) dpre[cb][k] = lds128(dys + (dyr[k] ^ ((uint32_t)cb << 4)));
-            }
-            if (!warp_wait(bar.wfull(), it & 1, abort, 128u, &g_fault_bwd)) { ok = false; break; }
-            tc_fence_after();
-            if (lane == 0) bulk_wait_read<0>();
-            __syncwarp();
-#pragma unroll 1
-            for (int c0 = 0; c0 < CH; c0 += CB) {
-                uint4 du[CB][W];
-#pragma unroll
-                for (int cb = 0; cb < CB; ++cb)
-#pragma unroll
-                    for (int k = 0; k < W; ++k)
-                        du[cb][k] = (CB == CH) ? dpre[cb][k] : lds128(dys + (dyr[k] ^ ((uint32_t)(c0 + cb) << 4)));
-                uint32_t wr[W][NGB];
-#pragma unroll
-                for (int k = 0; k < W; ++k)
-                    tmem_ld<NGB>(tl + p.tm_w + k * p.NGp + (kCPW * h + 8 * c0) / G, wr[k]);
-                tmem_wait_ld();
-#pragma unroll
-                for (int k = 0; k < W; ++k)
-#pragma unroll
-                    for (int e = 0; e < NGB; ++e) asm volatile("" : "+r"(wr[k][e]));
-                uint4 dxo[CB];
-#pragma unroll
-                for (int cb = 0; cb < CB; ++cb) {
-                    const int gq = (8 * cb) / G;                   // chunk's first group within the batch
-                    float dx[8];
-                    if constexpr (G == 1) {
-                        // channel pairs in packed fp32 FMAs (the same roundings as scalar fmaf)
-                        uint64_t acc[4];
-#pragma unroll
-                        for (int k = 0; k < W; ++k) {
-                            const uint32_t u[4] = {du[cb][k].x, du[cb][k].y, du[cb][k].z, du[cb][k].w};
-#pragma unroll
-                            for (int m = 0; m < 4; ++m) {
-                                const uint64_t d2 = f2pack(bf16_lo(u[m]), bf16_hi(u[m]));
-                                const uint64_t w2 = f2pack(__uint_as_float(wr[k][gq + 2 * m]),
-                                                           __uint_as_float(wr[k][gq + 2 * m + 1]));
-                                acc[m] = f2fma(w2, d2, k == 0 ? d2 : acc[m]);
-                            }
-                        }
-#pragma unroll
-                        for (int m = 0; m < 4; ++m) f2unpack(acc[m], dx[2 * m], dx[2 * m + 1]);
-                    } else {
-                        {
-                            float d0[8];
-                            unpack8(du[cb][0], d0);
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) dx[e] = fmaf(__uint_as_float(wr[0][gq + e / G]), d0[e], d0[e]);
-                        }
-#pragma unroll
-                        for (int k = 1; k < W; ++k) {
-                            float dk[8];
-                            unpack8(du[cb][k], dk);
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) dx[e] = fmaf(__uint_as_float(wr[k][gq + e / G]), dk[e], dx[e]);
-                        }
-                    }
-                    dxo[cb].x = pack_bf16x2(dx[0], dx[1]);
-                    dxo[cb].y = pack_bf16x2(dx[2], dx[3]);
-                    dxo[cb].z = pack_bf16x2(dx[4], dx[5]);
-                    dxo[cb].w = pack_bf16x2(dx[6], dx[7]);
-                }
-#pragma unroll
-                for (int cb = 0; cb < CB; ++cb) sts128(dxrow ^ ((uint32_t)(c0 + cb) << 4), dxo[cb]);
-            }
-            tc_fence_before();
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(bar.wempty());
-                tma_store_3d(&tm_dx, dxstage, id.slice * kDt + kCPW * h, id.t0 + 32 * q, id.b);
-                bulk_commit();
-            }
-            // ---- A2: dw[t,g,k] = sum_{c in g} dy[t,c] x[t-k,c], tap-major column k*NG + g,
-            // in batches of CB chunks as A1.  A batch is computed into registers (pk) and
-            // then stored; only the stores need the previous tile's dz / dU MMAs to be done
-            // with the dw tile, so a single-batch A2 is computed before B waits for them.
+        for (int i = 0; i < nt; ++i) {
+            const int j = i % S, mz = i / S;
+            const int st = i % NST, n = i / NST;
+            if (!warp_wait(bar.full(st), n & 1, abort, 64u, &g_fault_bwd)) { ok = false; break; }
+            const uint32_t dys = sb + st * p.stage_bytes, xs = dys + p.xy_tile_bytes;
+
+            // ---- A2: dw[t,g,k] = sum_{c in g} dy[t,c] x[t-k,c], tap-major column k*NG + g.
+            // When they fit in registers the values of both chunks are computed before
+            // the wait: only their stores need the previous tile's dz / dU MMAs to be done
+            // with the dw tile.
             constexpr int NPK = (NG8 + 1) / 2;           // packed bf16 pairs per (chunk, tap)
-            auto a2_compute = [&](int c0, uint32_t (&pk)[CB][W][NPK]) {
-                uint4 d0[CB], xu[CB][W];
+            constexpr bool kPre = CH * W * NPK <= 32;
+            auto a2_compute = [&](int cq, uint32_t (&pk)[W][NPK]) {
+                const uint4 d0 = lds128(dys + (dyr[0] ^ ((uint32_t)cq << 4)));
+                uint4 xu[W];
 #pragma unroll
-                for (int cb = 0; cb < CB; ++cb) {
-                    d0[cb] = lds128(dys + (dyr[0] ^ ((uint32_t)(c0 + cb) << 4)));
+                for (int k = 0; k < W; ++k) xu[k] = lds128(xs + (xr[k] ^ ((uint32_t)cq << 4)));
 #pragma unroll
-                    for (int k = 0; k < W; ++k) xu[cb][k] = lds128(xs + (xr[k] ^ ((uint32_t)(c0 + cb) << 4)));
-                }
+                for (int k = 0; k < W; ++k) {
+                    if constexpr (G == 1) {
+                        // one channel per group: dw = dy * x, exact in fp32 and rounded once
+                        // to bf16, which is what the packed bf16 multiply computes
+                        pk[k][0] = bf16x2_mul(d0.x, xu[k].x);
+                        pk[k][1] = bf16x2_mul(d0.y, xu[k].y);
+                        pk[k][2] = bf16x2_mul(d0.z, xu[k].z);
+                        pk[k][3] = bf16x2_mul(d0.w, xu[k].w);
+                    } else {
+                        float dv[8], xv[8], dw[NG8];
+                        unpack8(d0, dv);
+                        unpack8(xu[k], xv);
 #pragma unroll
-                for (int cb = 0; cb < CB; ++cb)
+                        for (int gl = 0; gl < NG8; ++gl) {
+                            float acc = 0.f;
 #pragma unroll
-                    for (int k = 0; k < W; ++k) {
-                        if constexpr (G == 1) {
-                            // one channel per group: dw = dy * x, exact in fp32 and rounded once
-                            // to bf16, which is what the packed bf16 multiply computes
-                            pk[cb][k][0] = bf16x2_mul(d0[cb].x, xu[cb][k].x);
-                            pk[cb][k][1] = bf16x2_mul(d0[cb].y, xu[cb][k].y);
-                            pk[cb][k][2] = bf16x2_mul(d0[cb].z, xu[cb][k].z);
-                            pk[cb][k][3] = bf16x2_mul(d0[cb].w, xu[cb][k].w);
-                        } else {
-                            float dv[8], xv[8], dw[NG8];
-                            unpack8(d0[cb], dv);
-                            unpack8(xu[cb][k], xv);
-#pragma unroll
-                            for (int gl = 0; gl < NG8; ++gl) {
-                                float acc = 0.f;
-#pragma unroll
-                                for (int e = gl * G; e < (gl + 1) * G; ++e) acc = fmaf(dv[e], xv[e], acc);
-                                dw[gl] = acc;
-                            }
-#pragma unroll
-                            for (int m2 = 0; m2 < NG8 / 2; ++m2) pk[cb][k][m2] = pack_bf16x2(dw[2 * m2], dw[2 * m2 + 1]);
+                            for (int e = gl * G; e < (gl + 1) * G; ++e) acc = fmaf(dv[e], xv[e], acc);
+                            dw[gl] = acc;
                         }
-                    }
-            };
-            auto a2_store = [&](int c0, const uint32_t (&pk)[CB][W][NPK]) {
 #pragma unroll
-                for (int cb = 0; cb < CB; ++cb) {
-                    const int g8 = (kCPW * h + 8 * (c0 + cb)) / G;
-#pragma unroll
-                    for (int k = 0; k < W; ++k) {
-                        const int jp = k * p.NGs + g8;                    // first tap-major column
-                        const uint32_t atom = (uint32_t)(jp >> 6), within = (uint32_t)(jp & 63);
-                        const uint32_t a = dwrow + atom * 16384u + ((((within >> 3) << 4) ^ dwsw) | ((within & 7) * 2));
-                        if constexpr (NG8 == 8) {
-                            sts128(a, make_uint4(pk[cb][k][0], pk[cb][k][1], pk[cb][k][2], pk[cb][k][3]));
-                        } else if constexpr (NG8 == 4) {
-                            sts64(a, pk[cb][k][0], pk[cb][k][1]);
-                        } else {
-                            sts32(a, pk[cb][k][0]);
-                        }
+                        for (int m2 = 0; m2 < NG8 / 2; ++m2) pk[k][m2] = pack_bf16x2(dw[2 * m2], dw[2 * m2 + 1]);
                     }
                 }
             };
-            if constexpr (CB == CH) {
-                uint32_t pk[CB][W][NPK];
-                a2_compute(0, pk);
-                // ---- B of the previous tile (its dz / dU MMAs ran during A1)
-                if (pv.it >= 0 && !phase_b(pv)) { ok = false; break; }
-                a2_store(0, pk);
+            auto a2_store = [&](int cq, const uint32_t (&pk)[W][NPK]) {
+                const int g8 = (kCPW * h + 8 * cq) / G;
+#pragma unroll
+                for (int k = 0; k < W; ++k) {
+                    const int jp = k * p.NGs + g8;                    // first tap-major column
+                    const uint32_t atom = (uint32_t)(jp >> 6), within = (uint32_t)(jp & 63);
+                    const uint32_t a = dwrow + atom * 16384u + ((((within >> 3) << 4) ^ dwsw) | ((within & 7) * 2));
+                    if constexpr (NG8 == 8) {
+                        sts128(a, make_uint4(pk[k][0], pk[k][1], pk[k][2], pk[k][3]));
+                    } else if constexpr (NG8 == 4) {
+                        sts64(a, pk[k][0], pk[k][1]);
+                    } else {
+                        sts32(a, pk[k][0]);
+                    }
+                }
+            };
+            if constexpr (kPre) {
+                uint32_t pk[CH][W][NPK];
+#pragma unroll
+                for (int cq = 0; cq < CH; ++cq) a2_compute(cq, pk[cq]);
+                if (!warp_wait(bar.dwfree(), (i & 1) ^ 1, abort, 32u, &g_fault_bwd)) { ok = false; break; }
+#pragma unroll
+                for (int cq = 0; cq < CH; ++cq) a2_store(cq, pk[cq]);
             } else {
-                // several batches (many taps): holding one across B cost more than it hid
-                if (pv.it >= 0 && !phase_b(pv)) { ok = false; break; }
+                if (!warp_wait(bar.dwfree(), (i & 1) ^ 1, abort, 32u, &g_fault_bwd)) { ok = false; break; }
 #pragma unroll 1
-                for (int c0 = 0; c0 < CH; c0 += CB) {
-                    uint32_t pk[CB][W][NPK];
-                    a2_compute(c0, pk);
-                    a2_store(c0, pk);
+                for (int cq = 0; cq < CH; ++cq) {
+                    uint32_t pk[W][NPK];
+                    a2_compute(cq, pk);
+                    a2_store(cq, pk);
                 }
             }
-            tc_fence_before();
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar.dwready());
-            pv.it = it;
-            pv.s = s;
-            pv.slice = id.slice;
-            pv.b = id.b;
-            pv.t0 = id.t0;
-            pv.seg = seg;
-            pv.last_of_slice = (i + 1 == tend) || ((i + 1) / p.per_slice != id.slice);
+
+            // ---- A1: dx[t,c] = dy[t,c] + sum_k w[t+k,g,k] dy[t+k,c]
+            if (!warp_wait(bar.wfull(), i & 1, abort, 128u, &g_fault_bwd)) { ok = false; break; }
+            tc_fence_after();
+            constexpr int NGB = 8 / G;                      // filter groups of one chunk
+            constexpr int KB = (W * (4 + NGB) <= 48) ? W : 4;   // taps per batch
+            uint4 dxo[CH];
+#pragma unroll
+            for (int cq = 0; cq < CH; ++cq) {
+                float dx[8];
+                uint64_t acc[4];
+#pragma unroll
+                for (int k0 = 0; k0 < W; k0 += KB) {
+                    uint4 du[KB];
+                    uint32_t wr[KB][NGB];
+#pragma unroll
+                    for (int kb = 0; kb < KB; ++kb)
+                        if (k0 + kb < W) du[kb] = lds128(dys + (dyr[k0 + kb] ^ ((uint32_t)cq << 4)));
+#pragma unroll
+                    for (int kb = 0; kb < KB; ++kb)
+                        if (k0 + kb < W)
+                            tmem_ld<NGB>(tl + p.tm_w + (k0 + kb) * p.NGp + (kCPW * h + 8 * cq) / G, wr[kb]);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int kb = 0; kb < KB; ++kb)
+#pragma unroll
+                        for (int e = 0; e < NGB; ++e) asm volatile("" : "+r"(wr[kb][e]));
+#pragma unroll
+                    for (int kb = 0; kb < KB; ++kb) {
+                        const int k = k0 + kb;
+                        if (k >= W) break;
+                        if constexpr (G == 1) {
+                            // channel pairs in packed fp32 FMAs (the same roundings as scalar fmaf)
+                            const uint32_t u[4] = {du[kb].x, du[kb].y, du[kb].z, du[kb].w};
+#pragma unroll
+                            for (int m = 0; m < 4; ++m) {
+                                const uint64_t d2 = f2pack(bf16_lo(u[m]), bf16_hi(u[m]));
+                                const uint64_t w2 = f2pack(__uint_as_float(wr[kb][2 * m]), __uint_as_float(wr[kb][2 * m + 1]));
+                                acc[m] = f2fma(w2, d2, k == 0 ? d2 : acc[m]);
+                            }
+                        } else {
+                            float dk[8];
+                            unpack8(du[kb], dk);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e)
+                                dx[e] = fmaf(__uint_as_float(wr[kb][e / G]), dk[e], k == 0 ? dk[e] : dx[e]);
+                        }
+                    }
+                }
+                if constexpr (G == 1) {
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) f2unpack(acc[m], dx[2 * m], dx[2 * m + 1]);
+                }
+                dxo[cq].x = pack_bf16x2(dx[0], dx[1]);
+                dxo[cq].y = pack_bf16x2(dx[2], dx[3]);
+                dxo[cq].z = pack_bf16x2(dx[4], dx[5]);
+                dxo[cq].w = pack_bf16x2(dx[6], dx[7]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar.wempty());
+            // once every epilogue warp is past A2 the x tile is dead, and dx goes there
+            // (an mbarrier rather than a named barrier, so that the wait is bounded)
+            if (lane == 0) mbar_arrive(bar.xdead());
+            if (!warp_wait(bar.xdead(), i & 1, abort, 4096u, &g_fault_bwd)) { ok = false; break; }
+#pragma unroll
+            for (int cq = 0; cq < CH; ++cq) sts128(xs + (dxr0 ^ ((uint32_t)cq << 4)), dxo[cq]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar.dxr(st));
+
+            // ---- dz of the previous token tile, complete once its last slice's MMAs ran
+            if (j == 0 && mz > 0 && !dz_out(mz - 1)) { ok = false; break; }
         }
-        if (ok && pv.it >= 0) phase_b(pv);
-        if (lane == 0) bulk_wait_all();
+        if (ok && nt > 0) ok = dz_out(nt / S - 1);
+
+        // ---- dU: this CTA's partial of each of its slices, then the slice group's sum
+        if (ok && warp_wait(bar.dufull(), 0, abort, 512u, &g_fault_bwd)) {
+            tc_fence_after();
+            const int N = p.n_slices * p.SC;
+            for (int j = 0; j < S; ++j) {
+                const int slice = sp.s0 + j;
+                if (h < nmb) {
+                    // lane j' of dU^T M-block h -> natural column g*W + k
+                    const int jp = 128 * h + row;
+                    const int jn = (jp % p.NGs) * W + jp / p.NGs;
+                    float *dst = p.du_part + (size_t)sp.a * p.R * N + (size_t)slice * p.SC + jn;
+#pragma unroll 1
+                    for (int c0 = 0; c0 < p.R; c0 += 16) {
+                        uint32_t v[16];
+                        tmem_ld<16>(tl + p.tm_du + (j * nmb + h) * p.R + c0, v);   // warp-collective
+                        tmem_wait_ld_regs(v);
+                        if (jp < p.SC) {
+#pragma unroll
+                            for (int m2 = 0; m2 < 16; ++m2) dst[(size_t)(c0 + m2) * N] = __uint_as_float(v[m2]);
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            fence_gpu();
+            __syncwarp();
+            if (lane == 0) red_release_add(p.flag_du + sp.b, 1u);
+            if (wait_count(p.flag_du + sp.b, (unsigned)(kEpiWarps * p.A), abort, 1024u)) {
+                // this CTA's share (of A) of the group's R x (S*SC) block, float4-wise
+                const int cols = S * p.SC;
+                const long long n4 = (long long)p.R * cols / 4;
+                const long long e0 = n4 * sp.a / p.A, e1 = n4 * (sp.a + 1) / p.A;
+                const int et = threadIdx.x - 32 * kEpi0;
+                for (long long e = e0 + et; e < e1; e += 32 * kEpiWarps) {
+                    const int r = (int)(4 * e / cols), c = (int)(4 * e - (long long)r * cols);
+                    const size_t off = (size_t)r * N + (size_t)sp.s0 * p.SC + c;
+                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                    for (int a = 0; a < p.A; ++a) {
+                        const float4 v = __ldcg(reinterpret_cast<const float4 *>(p.du_part + (size_t)a * p.R * N + off));
+                        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+                    }
+                    *reinterpret_cast<float4 *>(p.dU + off) = acc;
+                }
+            }
+        }
         __syncwarp();
-    } else if (warp == kDzWarp) {
-        // ---------------------------------------------------------- MMA issuer: dz partial
-        // dz = dw Up^T once tile i's dw is written: A = dw tile (K-major view), B = Up slice
-        // (K-major), 16 columns per step (+32 bytes within a 64-column atom, the next atom
-        // every 4 steps).
+    } else if (warp == kMmaWarp) {
+        // ---------------------------------------------------------- MMA issuer: dz and dU
+        // Once tile i's dw is written:
+        //   dz[m] (+)= dw Up^T: A = dw tile (K-major view), B = Up slice (K-major), 16
+        //     columns per step (+32 bytes within a 64-column atom, the next atom every 4
+        //     steps); accumulates over the token tile's slices;
+        //   dU^T[slice] (+)= dw^T z: A = dw^T (MN-major), B = z tile rows 0..127
+        //     (MN-major), 16 tokens per step; accumulates over the CTA's token tiles.
+        // The step counts are compile-time, so the issue loops unroll fully.
+        constexpr int SC = (kDt / G) * W;
+        constexpr int KSC = SC / 16;
+        constexpr int NMB = (SC + 127) / 128;
         const uint64_t t_k128 = desc_tmpl(16, 1024, kSw128);
+        const uint64_t t_dwt = desc_tmpl(16384, 1024, kSw128);
+        const uint64_t t_zmn = desc_tmpl(128, p.z_slab, kSwNone);
         const uint32_t i_dz = idesc_bf16(128, p.R, false, false);
-        const int ksc = p.SC / 16;
+        const uint32_t i_du = idesc_bf16(128, p.R, true, true);
         const uint32_t ubox = (uint32_t)(p.R * 128);
         const uint64_t st_wrap_a = (16384u - 96u) >> 4;   // next 64-column dw atom
         const uint64_t st_wrap_b = (ubox - 96u) >> 4;     // next 64-column Up box
         const uint32_t dw0 = sb + p.off_dw;
-        int prev_slice = -1, v = -1, ub = 0;
-        for (int i = tbeg; i < tend; ++i) {
-            const int it = i - tbeg;
-            const TileId id = tile_id(p, i);
-            if (id.slice != prev_slice) {
-                prev_slice = id.slice;
-                ++v;
-                ub = v % p.nU;
-                if (!warp_wait(bar.uf(ub), (v / p.nU) & 1, abort, 4u, &g_fault_bwd)) break;
-            }
-            if (!warp_wait(bar.dwready(), it & 1, abort, 32u, &g_fault_bwd)) break;
+        for (int i = 0; i < nt; ++i) {
+            const int j = i % S, mz = i / S, db = mz & 1, zb = mz & 1;
+            const int ub = u_res ? j : (i & 1);
+            const int upar = u_res ? 0 : ((i >> 1) & 1);
+            if (!warp_wait(bar.ufull(ub), upar, abort, 4u, &g_fault_bwd)) break;
+            if (j == 0 && !warp_wait(bar.zfull(zb), (mz >> 1) & 1, abort, 4u, &g_fault_bwd)) break;
+            if (!warp_wait(bar.dwready(), i & 1, abort, 8u, &g_fault_bwd)) break;
+            if (j == 0 && !warp_wait(bar.dzempty(db), ((mz >> 1) & 1) ^ 1, abort, 8u, &g_fault_bwd)) break;
             tc_fence_after();
-            const uint32_t us = sb + p.off_u + ub * p.u_bytes;
-            uint64_t da = desc_at(t_k128, dw0), db = desc_at(t_k128, us);
-            for (int kk = 0; kk < ksc; ++kk) {
-                if (elect_one()) mma_bf16_ss(tmem + p.tm_dz, da, db, i_dz, kk > 0 ? 1u : 0u);
-                __syncwarp();
-                const bool wrap = (kk & 3) == 3;
-                da += wrap ? st_wrap_a : 2u;
-                db += wrap ? st_wrap_b : 2u;
-            }
-            const bool last_of_slice = (i + 1 == tend) || ((i + 1) / p.per_slice != id.slice);
-            if (elect_one()) {
-                mma_commit(bar.mm2());
-                if (last_of_slice) mma_commit(bar.ue(ub));
-            }
-            __syncwarp();
-        }
-        if (elect_one()) mma_commit(bar.done());
-        __syncwarp();
-    } else if (warp == kDuWarp) {
-        // ---------------------------------------------------------- MMA issuer: dU partial
-        // dU^T += dw^T z once tile i's dw is written: A = dw^T (MN-major), B = z tile rows
-        // 0..127 (MN-major), 16 tokens per step; the accumulator restarts with each slice
-        // segment of the CTA.
-        const uint64_t t_dwt = desc_tmpl(16384, 1024, kSw128);
-        const uint64_t t_zmn = desc_tmpl(128, p.z_slab, kSwNone);
-        const uint32_t i_du = idesc_bf16(128, p.R, true, true);
-        const int nmb = p.SCp / 128;
-        const uint32_t dw0 = sb + p.off_dw;
-        int prev_slice = -1;
-        bool seg_first = true;
-        for (int i = tbeg; i < tend; ++i) {
-            const int it = i - tbeg;
-            const TileId id = tile_id(p, i);
-            if (id.slice != prev_slice) {
-                prev_slice = id.slice;
-                seg_first = true;
-            }
-            if (!warp_wait(bar.dwready(), it & 1, abort, 32u, &g_fault_bwd)) break;
-            tc_fence_after();
-            const uint32_t zs = sb + (it % p.stages) * p.stage_bytes + 2 * p.xy_tile_bytes;
-            for (int mb = 0; mb < nmb; ++mb) {
-                const uint32_t d = tmem + p.tm_du + mb * p.R;
-                uint64_t da = desc_at(t_dwt, dw0 + mb * 32768u), db = desc_at(t_zmn, zs);
+            {
+                const uint32_t us = sb + p.off_u + ub * p.u_bytes;
+                uint64_t da = desc_at(t_k128, dw0), dbd = desc_at(t_k128, us);
+                const uint32_t d = tmem + p.tm_dz + db * p.R;
 #pragma unroll
-                for (int kk = 0; kk < kTt / 16; ++kk) {
-                    if (elect_one()) mma_bf16_ss(d, da, db, i_du, (seg_first && kk == 0) ? 0u : 1u);
+                for (int kk = 0; kk < KSC; ++kk) {
+                    if (elect_one()) mma_bf16_ss(d, da, dbd, i_dz, (j > 0 || kk > 0) ? 1u : 0u);
                     __syncwarp();
-                    da += 2048u >> 4;
-                    db += 256u >> 4;
+                    const bool wrap = (kk & 3) == 3;
+                    da += wrap ? st_wrap_a : 2u;
+                    dbd += wrap ? st_wrap_b : 2u;
                 }
             }
-            if (elect_one()) mma_commit(bar.mm2());
+            {
+                const uint32_t zs = sb + p.off_z + zb * p.z_bytes;
+#pragma unroll
+                for (int mb = 0; mb < NMB; ++mb) {
+                    const uint32_t d = tmem + p.tm_du + (j * NMB + mb) * p.R;
+                    uint64_t da = desc_at(t_dwt, dw0 + mb * 32768u), dbd = desc_at(t_zmn, zs);
+#pragma unroll
+                    for (int kk = 0; kk < kTt / 16; ++kk) {
+                        if (elect_one()) mma_bf16_ss(d, da, dbd, i_du, (mz == 0 && kk == 0) ? 0u : 1u);
+                        __syncwarp();
+                        da += 2048u >> 4;
+                        dbd += 256u >> 4;
+                    }
+                }
+            }
+            if (elect_one()) {
+                mma_commit(bar.dwfree());
+                if (!u_res) mma_commit(bar.uempty(ub));
+                if (j == S - 1) {
+                    mma_commit(bar.dzfull(db));
+                    mma_commit(bar.zempty(zb));
+                }
+            }
             __syncwarp();
-            seg_first = false;
         }
-        if (elect_one()) mma_commit(bar.done());
+        if (elect_one()) {
+            mma_commit(bar.dufull());
+            mma_commit(bar.done());
+        }
+        __syncwarp();
+    } else if (warp == kRedWarp) {
+        // ---------------------------------------------------------- dz reducer
+        // Once all Bg slice groups have written their partial of token tile m, sum this
+        // CTA's share of its rows over the groups in order and write dz.
+        const int r4 = p.R / 4;                   // float4 per row
+        const int rows_per_pass = 32 / r4;
+        const int lr = lane / r4, l4 = lane - lr * r4;
+        const size_t part_stride = (size_t)p.B * p.T * p.R;
+        const unsigned target = (unsigned)(kEpiWarps * p.Bg);
+        for (int m = sp.m0; m < sp.m1; ++m) {
+            if (!wait_count(p.flag_dz + m, target, abort, 2048u)) break;
+            const int b = m / p.tiles_per_seq, t0 = (m - b * p.tiles_per_seq) * kTt;
+            const int nrows = min(kTt, p.T - t0);
+            const int lo = (int)((long long)nrows * sp.b / p.Bg), hi = (int)((long long)nrows * (sp.b + 1) / p.Bg);
+            for (int r0 = lo; r0 < hi; r0 += rows_per_pass) {
+                const int rr = r0 + lr;
+                const bool act = rr < hi;
+                const size_t off = ((size_t)b * p.T + t0 + (act ? rr : lo)) * p.R + 4 * l4;
+                const float *src = p.dz_part + off;
+                // 8 loads in flight per lane; the sum runs over the groups in order
+                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int g0 = 0; g0 < p.Bg; g0 += 8) {
+                    float4 v[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        if (act && g0 + u < p.Bg)
+                            v[u] = __ldcg(reinterpret_cast<const float4 *>(src + (size_t)(g0 + u) * part_stride));
+#pragma unroll
+                    for (int u = 0; u < 8; ++u)
+                        if (act && g0 + u < p.Bg) {
+                            acc.x += v[u].x; acc.y += v[u].y; acc.z += v[u].z; acc.w += v[u].w;
+                        }
+                }
+                if (act) *reinterpret_cast<float4 *>(p.dz + off) = acc;
+            }
+        }
         __syncwarp();
     }
 
     __syncthreads();
-    if (warp == 1) {
-        if (lane == 0) mbar_wait(bar.done(), 0, abort, 0u, &g_fault_bwd);
+    if (warp == kRecWarp) {
+        if (lane == 0) mbar_drain(bar.done(), 0);
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, p.tmem_cols);
@@ -651,9 +749,11 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
 // Up[r, s*SC + k*NG + g] = U[r, s*SC + g*W + k]  (tap-major columns within each slice).
 // Grid (ceil(N/2048), R): one row r per grid row; each thread writes 8 consecutive output
 // columns with one 16-byte store (NG is a multiple of 8, so the 8 share one tap k and read
-// source columns W apart).
+// source columns W apart).  Block (0, 0) also clears the main kernel's counters.
 __global__ void k_permute_u(const bf16 *__restrict__ U, bf16 *__restrict__ Up, int R, int N, int SC, int NG,
-                            int W) {
+                            int W, unsigned *__restrict__ flags, int nflags) {
+    if (blockIdx.x == 0 && blockIdx.y == 0)
+        for (int f = threadIdx.x; f < nflags; f += blockDim.x) flags[f] = 0u;
     const int r = blockIdx.y;
     const int j = 8 * (blockIdx.x * blockDim.x + threadIdx.x);
     if (r >= R || j >= N) return;
@@ -664,44 +764,6 @@ __global__ void k_permute_u(const bf16 *__restrict__ U, bf16 *__restrict__ Up, i
 #pragma unroll
     for (int m = 0; m < 4; ++m) v[m] = (uint32_t)src[(2 * m) * W] | ((uint32_t)src[(2 * m + 1) * W] << 16);
     *reinterpret_cast<uint4 *>(Up + (size_t)r * N + j) = make_uint4(v[0], v[1], v[2], v[3]);
-}
-
-// Both reductions in one launch (they are independent, so the small dU sum runs beside
-// the dz sum instead of after it):
-//   blocks [0, nb_dz):  dz[bt, :] = sum_s part_dz[s, bt, :]  (slices in order), grid-stride
-//                       over float4 elements;
-//   blocks [nb_dz, ..): dU[r, s*SC + j] = sum over the CTA segments of slice s of
-//                       part_du[s, seg, r, j]  (in order); block nb_dz + r*nbx + bx covers row
-//                       r, columns 4*(256*bx + thread) .. +3 (SC is a multiple of 8, so the
-//                       four never straddle a slice).
-__global__ void k_reduce(const float *__restrict__ part_dz, float *__restrict__ dz, int n_slices, size_t n4,
-                         int nb_dz, const float *__restrict__ part_du, float *__restrict__ dU, int R, int SC,
-                         int maxseg, int per_slice, int n_tiles, int grid, int nbx) {
-    if ((int)blockIdx.x < nb_dz) {
-        for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < n4; e += (size_t)nb_dz * blockDim.x) {
-            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-            for (int s = 0; s < n_slices; ++s) {
-                const float4 v = reinterpret_cast<const float4 *>(part_dz)[(size_t)s * n4 + e];
-                acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-            }
-            reinterpret_cast<float4 *>(dz)[e] = acc;
-        }
-        return;
-    }
-    const int bid = (int)blockIdx.x - nb_dz;
-    const int r = bid / nbx;
-    const int N = SC * n_slices;
-    const int j = 4 * ((bid - r * nbx) * (int)blockDim.x + (int)threadIdx.x);
-    if (r >= R || j >= N) return;
-    const int s = j / SC, jl = j - s * SC;
-    const int nseg = owner_of((long long)(s + 1) * per_slice - 1, n_tiles, grid) -
-                     owner_of((long long)s * per_slice, n_tiles, grid) + 1;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int seg = 0; seg < nseg; ++seg) {
-        const float4 v = *reinterpret_cast<const float4 *>(part_du + (((size_t)s * maxseg + seg) * R + r) * SC + jl);
-        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-    }
-    *reinterpret_cast<float4 *>(dU + (size_t)r * N + j) = acc;
 }
 
 // ------------------------------------------------------------------ host side
@@ -750,10 +812,27 @@ int num_sms() {
 
 constexpr uint32_t kSmemLimit = 227 * 1024;
 size_t a256(size_t v) { return (v + 255) / 256 * 256; }
+uint32_t a1k(uint32_t v) { return (v + 1023) / 1024 * 1024; }
 
-bool plan_bwd(int B, int T, int D, int G, int W, int R, int grid, BwdParams &p) {
+uint32_t smem_bytes(const BwdParams &p) { return p.off_bar + kBarBytes + 16 + 1024; }
+
+// Shared-memory layout for a ring depth and number of Up buffers; false if it does not fit.
+bool layout_smem(BwdParams &p, int stages, int nU) {
+    p.stages = stages;
+    p.nU = nU;
+    p.off_z = stages * p.stage_bytes;
+    p.off_u = p.off_z + 2 * p.z_bytes;
+    p.off_dw = a1k(p.off_u + nU * p.u_bytes);
+    p.off_bar = p.off_dw + (uint32_t)(p.SCp / 64) * 16384u;
+    return smem_bytes(p) <= kSmemLimit;
+}
+
+// Plans the kernel for these sizes on `nsm` SMs: tile geometry, TMEM and shared-memory
+// layouts, and the A x Bg grid.  false: the tensor-core backward does not take them.
+bool plan_bwd(int B, int T, int D, int G, int W, int R, int nsm, BwdParams &p) {
     if (!(R == 16 || R == 32 || R == 64)) return false;
     if (D % kDt || !(G == 1 || G == 2 || G == 4) || W < 1 || W > 8) return false;
+    p = BwdParams{};
     p.B = B; p.T = T; p.D = D; p.G = G; p.W = W; p.R = R;
     p.NGs = kDt / G;
     p.NGp = p.NGs < 16 ? 16 : p.NGs;
@@ -762,69 +841,85 @@ bool plan_bwd(int B, int T, int D, int G, int W, int R, int grid, BwdParams &p) 
     p.SCp = (p.SC + 127) / 128 * 128;
     p.n_slices = D / kDt;
     p.tiles_per_seq = (T + kTt - 1) / kTt;
-    p.per_slice = B * p.tiles_per_seq;
-    const long long nt = (long long)p.n_slices * p.per_slice;
-    if (nt >= (1ll << 31)) return false;
-    p.n_tiles = (int)nt;
-    if (grid > p.n_tiles) grid = p.n_tiles;
-    int maxseg = 1;
-    for (int s = 0; s < p.n_slices; ++s) {
-        const int c0 = owner_of((long long)s * p.per_slice, p.n_tiles, grid);
-        const int c1 = owner_of((long long)(s + 1) * p.per_slice - 1, p.n_tiles, grid);
-        maxseg = std::max(maxseg, c1 - c0 + 1);
-    }
-    p.maxseg = maxseg;
+    const long long ntt = (long long)B * p.tiles_per_seq;
+    if (ntt >= (1ll << 30) || (long long)p.n_slices * ntt >= (1ll << 31)) return false;
+    p.n_tt = (int)ntt;
     p.u_boxes = (p.SC + 63) / 64;
-    // TMEM: w (W tap blocks) | dz | dU^T
+    // TMEM: w (W tap blocks) | dz (two buffers) | dU^T (one slot per slice of the CTA)
     p.tm_w = 0;
-    p.tm_dw = 0;   // unused: dw lives in shared memory only
     p.tm_dz = (uint32_t)(W * p.NGp + 31) / 32 * 32;
-    p.tm_du = p.tm_dz + (uint32_t)R;
-    const uint32_t used = p.tm_du + (uint32_t)(p.SCp / 128) * R;
-    if (used > 512) return false;
-    p.tmem_cols = 32;
-    while (p.tmem_cols < used) p.tmem_cols *= 2;
+    p.tm_du = p.tm_dz + 2u * (uint32_t)R;
+    const uint32_t slot = (uint32_t)(p.SCp / 128) * R;
+    if (p.tm_du + slot > 512) return false;
+    const int s_max_tmem = (int)((512 - p.tm_du) / slot);
+    // shared memory
     p.rows = kTt + W - 1;
-    p.xy_tile_bytes = (p.rows * 128 + 1023) / 1024 * 1024;
+    p.xy_tile_bytes = a1k(p.rows * 128);
     p.z_slab = (p.rows * 16 + 127) / 128 * 128;
-    p.z_bytes = (uint32_t)(R / 8) * p.z_slab;
-    p.stage_bytes = (2 * p.xy_tile_bytes + p.z_bytes + 1023) / 1024 * 1024;
+    p.z_bytes = a1k((uint32_t)(R / 8) * p.z_slab);
+    p.stage_bytes = 2 * p.xy_tile_bytes;
     p.u_bytes = (uint32_t)(p.u_boxes * R * 128);
-    const int options[4][2] = {{3, 2}, {3, 1}, {2, 2}, {2, 1}};   // (stages, U buffers)
-    for (auto &o : options) {
-        p.stages = o[0];
-        p.nU = o[1];
-        p.off_u = p.stages * p.stage_bytes;
-        p.off_dw = p.off_u + p.nU * p.u_bytes;
-        p.off_dw = (p.off_dw + 1023) / 1024 * 1024;
-        p.off_dx = p.off_dw + (uint32_t)(p.SCp / 64) * 16384u;
-        p.off_bar = p.off_dx + kDxStageBytes;
-        if (p.off_bar + kBarBytes + 16 + 1024 <= kSmemLimit) return true;
+    // grid: Bg slice groups (at most s_max_tmem slices each) x A token ranges; fewest
+    // tiles on the busiest CTA first, then fewest slice groups (fewer dz partials)
+    int best_bg = 0, best_a = 0;
+    long long best_cost = -1;
+    for (int bg = 1; bg <= std::min(p.n_slices, nsm); ++bg) {
+        const int smax = (p.n_slices + bg - 1) / bg;
+        if (smax > s_max_tmem) continue;
+        const int a = std::min(p.n_tt, nsm / bg);
+        if (a < 1) continue;
+        const long long cost = (long long)smax * ((p.n_tt + a - 1) / a);
+        if (best_cost < 0 || cost < best_cost) {
+            best_cost = cost;
+            best_bg = bg;
+            best_a = a;
+        }
     }
+    if (best_cost < 0) return false;
+    p.Bg = best_bg;
+    p.A = best_a;
+    const int smax = (p.n_slices + p.Bg - 1) / p.Bg;
+    p.tmem_cols = 32;
+    while (p.tmem_cols < p.tm_du + (uint32_t)smax * slot) p.tmem_cols *= 2;
+    // ring depth 3 if it fits, else 2; two Up buffers unless a CTA has one slice
+    const int nU = smax >= 2 ? 2 : 1;
+    for (int st = kMaxStages; st >= 2; --st)
+        if (layout_smem(p, st, nU)) return true;
     return false;
 }
 
 template <int W, int G>
-cudaError_t launch_t(const CUtensorMap *m, const BwdParams &p, int grid, cudaStream_t s) {
+cudaError_t launch_t(const CUtensorMap *m, const BwdParams &p, cudaStream_t s) {
     auto kern = k_tc_lowrank_bwd<W, G>;
-    const uint32_t smem = p.off_bar + kBarBytes + 16 + 1024;
+    const uint32_t smem = smem_bytes(p);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    kern<<<grid, Geo<G>::kThreads, smem, s>>>(m[0], m[1], m[2], m[3], m[4], p);
-    return cudaGetLastError();
+    // Cooperative launch: the CTAs wait on each other's partial sums, so all of them
+    // must be resident at once (the launch fails instead of starting otherwise).
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.A * p.Bg);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, m[0], m[1], m[2], m[3], m[4], p);
 }
 
 template <int W>
-cudaError_t launch_w(int G, const CUtensorMap *m, const BwdParams &p, int grid, cudaStream_t s) {
+cudaError_t launch_w(int G, const CUtensorMap *m, const BwdParams &p, cudaStream_t s) {
     switch (G) {
-        case 1: return launch_t<W, 1>(m, p, grid, s);
-        case 2: return launch_t<W, 2>(m, p, grid, s);
-        default: return launch_t<W, 4>(m, p, grid, s);
+        case 1: return launch_t<W, 1>(m, p, s);
+        case 2: return launch_t<W, 2>(m, p, s);
+        default: return launch_t<W, 4>(m, p, s);
     }
 }
 
 struct WsLayout {
-    size_t up, dz, du, total;
+    size_t up, dz, du, flags, total;
 };
 
 WsLayout ws_layout(const BwdParams &p) {
@@ -832,8 +927,9 @@ WsLayout ws_layout(const BwdParams &p) {
     const size_t N = (size_t)p.n_slices * p.SC;
     l.up = 0;
     l.dz = a256(l.up + (size_t)p.R * N * 2);
-    l.du = a256(l.dz + (size_t)p.n_slices * p.B * p.T * p.R * 4);
-    l.total = a256(l.du + (size_t)p.n_slices * p.maxseg * p.R * p.SC * 4);
+    l.du = a256(l.dz + (size_t)p.Bg * p.B * p.T * p.R * 4);
+    l.flags = a256(l.du + (size_t)p.A * p.R * N * 4);
+    l.total = a256(l.flags + (size_t)(p.n_tt + p.Bg) * 4);
     return l;
 }
 
@@ -856,15 +952,19 @@ cudaError_t launch_tc_lowrank_bwd(const void *x, const void *z, const void *U, c
                                   cudaStream_t s) {
     using namespace tcb;
     BwdParams p;
-    const int grid = std::min(num_sms(), (D / kDt) * B * ((T + kTt - 1) / kTt));
-    if (!plan_bwd(B, T, D, G, W, R, grid, p)) return cudaErrorNotSupported;
+    if (!plan_bwd(B, T, D, G, W, R, num_sms(), p)) return cudaErrorNotSupported;
     const WsLayout l = ws_layout(p);
     uint8_t *w8 = (uint8_t *)ws;
     bf16 *Up = (bf16 *)(w8 + l.up);
     p.dz_part = (float *)(w8 + l.dz);
     p.du_part = (float *)(w8 + l.du);
+    p.flag_dz = (unsigned *)(w8 + l.flags);
+    p.flag_du = p.flag_dz + p.n_tt;
+    p.dz = dz;
+    p.dU = dU;
     const int N = p.n_slices * p.SC;
-    k_permute_u<<<dim3((N / 8 + 255) / 256, R), 256, 0, s>>>((const bf16 *)U, Up, R, N, p.SC, p.NGs, W);
+    k_permute_u<<<dim3((N / 8 + 255) / 256, R), 256, 0, s>>>((const bf16 *)U, Up, R, N, p.SC, p.NGs, W,
+                                                              p.flag_dz, p.n_tt + p.Bg);
 
     CUtensorMap m[5];
     const uint64_t dxyz[3] = {(uint64_t)D, (uint64_t)T, (uint64_t)B};
@@ -873,36 +973,25 @@ cudaError_t launch_tc_lowrank_bwd(const void *x, const void *z, const void *U, c
     const uint32_t bz[3] = {8, p.rows, 1};
     const uint64_t du[2] = {(uint64_t)N, (uint64_t)R};
     const uint32_t bu[2] = {64, (uint32_t)R};
-    constexpr int kCPW = Geo<1>::kCPW;   // the same for every G
-    static_assert(kCPW == 16 || kCPW == 32, "dx staging rows are 32 or 64 bytes");
-    const uint32_t bdx[3] = {(uint32_t)kCPW, 32, 1};
+    const uint32_t bdx[3] = {(uint32_t)kDt, (uint32_t)kTt, 1};
     if (!make_map(&m[0], dy, 3, dxyz, bxy, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) ||
         !make_map(&m[1], x, 3, dxyz, bxy, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) ||
         !make_map(&m[2], z, 3, dzz, bz, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
         !make_map(&m[3], Up, 2, du, bu, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) ||
-        !make_map(&m[4], dx, 3, dxyz, bdx, kCPW == 16 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_64B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_128B)) {
+        !make_map(&m[4], dx, 3, dxyz, bdx, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B)) {
         set_last_error("dsc_bwd_lowrank: cuTensorMapEncodeTiled failed");
         return cudaErrorInvalidValue;
     }
-    cudaError_t e;
     switch (W) {
-        case 1: e = launch_w<1>(G, m, p, grid, s); break;
-        case 2: e = launch_w<2>(G, m, p, grid, s); break;
-        case 3: e = launch_w<3>(G, m, p, grid, s); break;
-        case 4: e = launch_w<4>(G, m, p, grid, s); break;
-        case 5: e = launch_w<5>(G, m, p, grid, s); break;
-        case 6: e = launch_w<6>(G, m, p, grid, s); break;
-        case 7: e = launch_w<7>(G, m, p, grid, s); break;
-        default: e = launch_w<8>(G, m, p, grid, s); break;
+        case 1: return launch_w<1>(G, m, p, s);
+        case 2: return launch_w<2>(G, m, p, s);
+        case 3: return launch_w<3>(G, m, p, s);
+        case 4: return launch_w<4>(G, m, p, s);
+        case 5: return launch_w<5>(G, m, p, s);
+        case 6: return launch_w<6>(G, m, p, s);
+        case 7: return launch_w<7>(G, m, p, s);
+        default: return launch_w<8>(G, m, p, s);
     }
-    if (e != cudaSuccess) return e;
-    const size_t n4 = (size_t)B * T * R / 4;
-    const int nb_dz = (int)std::min<size_t>((n4 + 255) / 256, 8192);
-    const int nbx = (N / 4 + 255) / 256;
-    k_reduce<<<nb_dz + nbx * R, 256, 0, s>>>(p.dz_part, dz, p.n_slices, n4, nb_dz, p.du_part, dU, R, p.SC,
-                                             p.maxseg, p.per_slice, p.n_tiles, grid, nbx);
-    return cudaGetLastError();
 }
 
 unsigned read_device_fault_bwd(bool reset) {

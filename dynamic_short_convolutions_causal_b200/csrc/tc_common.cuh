@@ -88,6 +88,16 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
     }
 }
 
+// Waits for a phase that is known to complete (a TMA load or MMAs already issued), even
+// after the CTA has given up on its other waits, so that nothing is still writing to
+// shared memory or TMEM when the CTA frees them and exits.  Bounded by kWaitLimitNs.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return;
+    const unsigned long long t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity))
+        if (globaltimer() - t0 > kWaitLimitNs) return;
+}
+
 // mbar_wait by every lane of a warp, with one warp-uniform outcome.
 template <unsigned HintNs = 0>
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int *abort, unsigned code,

@@ -212,7 +212,7 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
             const int issued = it;
             for (int s = 0; s < S && s < issued; ++s) {
                 const int last = issued - 1 - ((issued - 1 - s) % S);   // last tile using stage s
-                mbar_wait<kWaitHint>(bar.full(s), (last / S) & 1, abort, 0u, &g_fault);
+                mbar_drain(bar.full(s), (last / S) & 1);
             }
         }
         __syncwarp();
@@ -344,7 +344,7 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
 
     __syncthreads();
     if (warp == 1) {
-        if (lane == 0) mbar_wait<kWaitHint>(bar.done(), 0, abort, 0u, &g_fault);
+        if (lane == 0) mbar_drain(bar.done(), 0);
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, p.tmem_cols);

@@ -159,6 +159,31 @@ DSC_API dsc_status_t dsc_static_bwd_noalloc(const void *x, const void *w, const 
 /* Size in bytes of the fixed scratch array dsc_static_bwd_noalloc uses. */
 DSC_API size_t dsc_static_bwd_noalloc_max_scratch_bytes(void);
 
+/* One decode step for B sequences: the single new token x_t of each sequence, with its
+ * W-1 previous inputs held in a caller-owned rolling window (inference, which the page
+ * leaves to further engineering: "Significancia e Alegacoes").  For each b and c,
+ *   y_t[b,c] = x_t[b,c] + sum_{k=0}^{W-1} f(b,c,k) * x_{t-k}[b,c],
+ * where x_{t-k} for k >= 1 is row W-1-k of state[b] and f is
+ *   dsc_decode_step:          w_t[b, g(c), k]                    (explicit filters)
+ *   dsc_decode_step_lowrank:  sum_r z_t[b,r] U[r, g(c)*W + k]    (w_t = z_t U)
+ * Afterwards state[b] holds the window of the next step: its rows moved up by one and
+ * x_t in the last row (updated in place).
+ *   x_t, y_t [B,D];  w_t [B,D/G,W];  z_t [B,R];  U [R,(D/G)*W];
+ *   state [B,W-1,D], row 0 the oldest input; a sequence starts from a zeroed window
+ *   (inputs before its start count as zero, as in the forward).  state may be NULL
+ *   when W = 1.  Stepping a sequence from a zero window reproduces the forward's
+ *   outputs token by token.
+ * Same element type, alignment and error rules as the other entry points; y_t must not
+ * overlap x_t or state.  dsc_decode_step_lowrank returns DSC_ERR_UNSUPPORTED when R and W
+ * are too large for its shared-memory tile (R = 256 with W = 8). */
+DSC_API dsc_status_t dsc_decode_step(const void *x_t, const void *w_t, void *state, void *y_t,
+                                     int B, int D, int G, int W,
+                                     dsc_dtype_t dt, dsc_stream_t stream);
+DSC_API dsc_status_t dsc_decode_step_lowrank(const void *x_t, const void *z_t, const void *U,
+                                             void *state, void *y_t,
+                                             int B, int D, int G, int W, int R,
+                                             dsc_dtype_t dt, dsc_stream_t stream);
+
 /* Which implementations the low-rank entry points use for these sizes: bit 0 set when
  * dsc_fwd_lowrank runs on the tensor-core (tcgen05) kernel, bit 1 when
  * dsc_bwd_lowrank does; 0 = both on CUDA cores; -1 = invalid sizes.  The tensor-core
