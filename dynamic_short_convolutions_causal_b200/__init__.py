@@ -60,6 +60,7 @@ def _load():
         "dsc_decode_step": (i, [vp, vp, vp, vp, i, i, i, i, i, vp]),
         "dsc_decode_step_lowrank": (i, [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]),
         "dsc_device_fault": (ctypes.c_uint, [i]),
+        "dsc_test_arm_wait_timeout": (None, [ctypes.c_uint]),
         "dsc_status_string": (ctypes.c_char_p, [i]),
         "dsc_last_error": (ctypes.c_char_p, []),
     }

@@ -95,9 +95,25 @@ k_decode_lowrank(const T *__restrict__ x_t, const T *__restrict__ z_t, const T *
         const int r = e / kDcSeq, bl = e - r * kDcSeq;
         zs[e] = bl < nb ? to_f(z_t[(size_t)(b0 + bl) * R + r]) : 0.f;
     }
-    for (int e = tid; e < R * 4 * nq; e += kDcThreads) {
-        const int r = e / (4 * nq), j = e - r * 4 * nq;
-        us[e] = j < ncol ? to_f(U[(size_t)r * N + g0 * W + j]) : 0.f;
+    if (sizeof(T) == 2 && ncol % 8 == 0 && (g0 * W) % 8 == 0 && N % 8 == 0) {
+        // 8 columns per 16-byte load (the common case: the block's columns are aligned)
+        const int n8 = ncol / 8;
+        for (int e = tid; e < R * n8; e += kDcThreads) {
+            const int r = e / n8, j8 = e - r * n8;
+            const uint4 u = __ldg(reinterpret_cast<const uint4 *>(U + (size_t)r * N + g0 * W + 8 * j8));
+            float *d = us + r * 4 * nq + 8 * j8;
+            d[0] = bf16_lo(u.x); d[1] = bf16_hi(u.x); d[2] = bf16_lo(u.y); d[3] = bf16_hi(u.y);
+            d[4] = bf16_lo(u.z); d[5] = bf16_hi(u.z); d[6] = bf16_lo(u.w); d[7] = bf16_hi(u.w);
+        }
+        for (int e = tid; e < R * (4 * nq - ncol); e += kDcThreads) {
+            const int r = e / (4 * nq - ncol), j = ncol + e - r * (4 * nq - ncol);
+            us[r * 4 * nq + j] = 0.f;
+        }
+    } else {
+        for (int e = tid; e < R * 4 * nq; e += kDcThreads) {
+            const int r = e / (4 * nq), j = e - r * 4 * nq;
+            us[e] = j < ncol ? to_f(U[(size_t)r * N + g0 * W + j]) : 0.f;
+        }
     }
     __syncthreads();
     // w[b, j] = sum_r z[b, r] U[r, j] in 4 (sequences) x 4 (columns) tiles

@@ -80,6 +80,20 @@ size_t lowrank_ws(const Dims &d, bool bf16) {
 
 namespace dsc {
 void set_last_error(const char *msg) { snprintf(g_err, sizeof(g_err), "%s", msg); }
+
+// Armed wait limit of the test hook for the next tensor-core launch (0: not armed).
+thread_local unsigned long long g_test_wait_ns = 0;
+
+void take_wait_test(unsigned long long *wait_ns, int *withhold_cta) {
+    if (g_test_wait_ns) {
+        *wait_ns = g_test_wait_ns;
+        *withhold_cta = 0;
+        g_test_wait_ns = 0;
+    } else {
+        *wait_ns = 1000000000ull;     // one second, as the kernels' own default
+        *withhold_cta = -1;
+    }
+}
 }  // namespace dsc
 
 extern "C" {
@@ -239,6 +253,10 @@ DSC_API int dsc_lowrank_path(int B, int T, int D, int G, int W, int R, dsc_dtype
 }
 
 DSC_API unsigned dsc_device_fault(int reset) { return dsc::read_device_fault(reset != 0); }
+
+DSC_API void dsc_test_arm_wait_timeout(unsigned wait_limit_us) {
+    dsc::g_test_wait_ns = (unsigned long long)(wait_limit_us ? wait_limit_us : 1) * 1000ull;
+}
 
 DSC_API const char *dsc_status_string(dsc_status_t s) {
     switch (s) {

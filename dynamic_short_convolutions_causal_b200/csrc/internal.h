@@ -10,6 +10,11 @@ namespace dsc {
 // Records the detail string that dsc_last_error() returns on this host thread.
 void set_last_error(const char *msg);
 
+// Wait settings for the next tensor-core launch on this host thread: the normal limit
+// and no withheld loads, unless dsc_test_arm_wait_timeout() armed the test hook, which
+// this call then disarms.
+void take_wait_test(unsigned long long *wait_ns, int *withhold_cta);
+
 // Streaming CUDA-core kernels (stream.cu)
 void launch_conv_fwd(const void *x, const void *w, void *y, int B, int T, int D, int G, int W,
                      bool bf16, bool is_static, cudaStream_t s);

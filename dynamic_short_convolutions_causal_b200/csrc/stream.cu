@@ -9,10 +9,12 @@
 // These ops do 2-5 FLOP per byte; their bound is HBM bandwidth, and a kernel reaches it
 // only with enough bytes in flight.  So a thread owns V channels (4 to 16 bytes of a
 // token row) and walks a chunk of tokens of one sequence, keeping the W-1 rows it needs
-// from earlier (or later) tokens in registers, and it loads the rows of U tokens at
-// once before computing on them.  V shrinks as W grows, so that the filter taps and
-// the row windows stay in registers with room for many resident warps.  A warp reads
-// 32*V consecutive channels of a row, i.e. whole 128-byte lines.
+// from earlier (or later) tokens in registers.  Its rows arrive a batch of 8 or 16
+// tokens at a time through shared memory with cp.async, double-buffered: the next batch is in
+// flight while the current one is used, and the bytes in flight cost no registers.  A
+// warp reads 32*V consecutive channels of a row (whole 128-byte lines), and the
+// staging layout interleaves the threads so that their shared-memory reads do not
+// conflict.  V shrinks as W grows, so that the taps and row windows stay in registers.
 #include "common.cuh"
 #include "internal.h"
 
@@ -73,10 +75,57 @@ struct Lanes {
     static constexpr int V = sizeof(T) == 2 ? (W <= 4 ? 4 : 2) : (W <= 4 ? 4 : 2);
 };
 
-constexpr int kU = 8;              // token rows loaded at once per thread
 constexpr int kChunk = 128;        // tokens per thread (the W-1 row halo is re-read)
 constexpr int kBX = 32;            // threads along channels (one warp)
 constexpr int kBY = 8;             // chunks per block in the static backward
+
+__host__ __device__ inline int chunk_for(int T) { return T < kChunk ? T : kChunk; }
+__host__ __device__ inline int dw_partials(int B, int T) { return B * cdiv(cdiv(T, chunk_for(T)), kBY); }
+
+// cp.async of BYTES (4, 8 or 16) from global to shared memory; when `valid` is false the
+// destination is zero-filled and nothing is read.
+template <int BYTES>
+__device__ __forceinline__ void cp_async(uint32_t dst, const void *src, bool valid) {
+    const int n = valid ? BYTES : 0;
+    if constexpr (BYTES == 16)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(n) : "memory");
+    else
+        asm volatile("cp.async.ca.shared.global [%0], [%1], %2, %3;" ::"r"(dst), "l"(src), "n"(BYTES), "r"(n)
+                     : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <typename R>
+__device__ __forceinline__ R lds_raw(uint32_t addr) {
+    R r;
+    if constexpr (sizeof(R) == 4) {
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r) : "r"(addr));
+    } else if constexpr (sizeof(R) == 8) {
+        asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(addr));
+    } else {
+        asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(addr));
+    }
+    return r;
+}
+
+// Shared-memory staging of a thread's row batches: slot (stage, tensor, row u) of thread
+// `tid` is at ((stage * NT + tensor) * KU + u) * NTHREADS * BYTES + tid * BYTES.
+template <int BYTES, int NT, int KU, int NTHREADS = 256>
+struct Staging {
+    uint32_t base;            // this thread's slot 0: block base + tid * BYTES
+    __device__ Staging(uint32_t block_base, int tid) : base(block_base + (uint32_t)(tid * BYTES)) {}
+    __device__ uint32_t at(int stage, int tensor, int u) const {
+        return base + (uint32_t)(((stage * NT + tensor) * KU + u) * NTHREADS * BYTES);
+    }
+    static constexpr int bytes_per_thread() { return 2 * NT * KU * BYTES; }
+};
+
+// Rows per batch: 64 bytes of each staged tensor per thread and batch (16 rows of 4
+// bytes, 8 of 8, 4 of 16), which keeps a block's staging at or below 64 KB so that
+// several blocks share an SM.
+template <int SLOT> struct Batch { static constexpr int KU = 64 / SLOT; };
 
 // Explicit per-token taps of V channels: w [B*T, D/G, W], element (bt, g, k).
 template <typename T, int W, int V>
@@ -106,25 +155,36 @@ __device__ __forceinline__ void dyn_taps(const T *__restrict__ w, size_t bt, int
 
 // ------------------------------------------------------------------ forward
 // y[t] = x[t] + sum_k f_t[k] x[t-k] for V channels over a chunk of tokens; f is the
-// static w[c,k] (STATIC) or the explicit w[b,t,g(c),k].
+// static w[c,k] (STATIC) or the explicit w[b,t,g(c),k].  With explicit filters whose
+// group covers the thread's V channels (G % V == 0) and whose W taps make a 4-, 8- or
+// 16-byte aligned vector, the taps are staged with the rows; otherwise they are read
+// per token.
 template <typename T, int W, bool STATIC>
-__global__ void __launch_bounds__(256)
-k_stream_fwd(const T *__restrict__ x, const T *__restrict__ w, T *__restrict__ y, int B, int T_, int D,
-             int G, int chunk) {
+__device__ __forceinline__ void stream_fwd_item(const T *__restrict__ x, const T *__restrict__ w, T *__restrict__ y,
+                                                int B, int T_, int D, int G, int chunk, int bx, int by) {
     constexpr int V = Lanes<T, W>::V;
     using P = Pack<T, V>;
-    const int v = blockIdx.x * blockDim.x + threadIdx.x;
-    if (v >= D / V) return;
+    constexpr int TB = W * (int)sizeof(T);                         // bytes of one token's taps
+    constexpr bool kTapVec = !STATIC && (TB == 4 || TB == 8 || TB == 16);
+    constexpr int NT = kTapVec ? 2 : 1;
+    constexpr int SB = P::BYTES > TB || !kTapVec ? P::BYTES : TB;  // slot size
+    constexpr int KU = Batch<SB>::KU;
+    extern __shared__ __align__(16) uint8_t stg_raw[];
+    const Staging<SB, NT, KU> stg((uint32_t)__cvta_generic_to_shared(stg_raw), (int)threadIdx.x);
+    const int v = bx * 256 + threadIdx.x;
+    const bool active = v < D / V;
     const int nch = cdiv(T_, chunk);
-    const int b = blockIdx.y / nch;
-    const int t0 = (blockIdx.y - b * nch) * chunk;
+    const int b = by / nch;
+    const int t0 = (by - b * nch) * chunk;
     const int t1 = min(t0 + chunk, T_);
-    const int c0 = v * V;
+    const int c0 = active ? v * V : 0;
     const T *xb = x + (size_t)b * T_ * D + c0;
     T *yb = y + (size_t)b * T_ * D + c0;
+    const bool tap_stage = kTapVec && (G % V == 0);
+    const T *wb = STATIC ? w : w + ((size_t)b * T_ * (D / G) + c0 / G) * W;   // taps of token 0
 
     float f[W][V];
-    if (STATIC) {
+    if (STATIC && active) {
 #pragma unroll
         for (int i = 0; i < V; ++i)
 #pragma unroll
@@ -133,21 +193,62 @@ k_stream_fwd(const T *__restrict__ x, const T *__restrict__ w, T *__restrict__ y
     float win[W][V];   // win[k] = x[t-k]
 #pragma unroll
     for (int k = 1; k < W; ++k) {
-        if (t0 - k >= 0) P::unpack(P::load(xb + (size_t)(t0 - k) * D), win[k]);
+        if (active && t0 - k >= 0) P::unpack(P::load(xb + (size_t)(t0 - k) * D), win[k]);
         else
 #pragma unroll
             for (int i = 0; i < V; ++i) win[k][i] = 0.f;
     }
-    for (int tb = t0; tb < t1; tb += kU) {
-        typename P::raw_t raw[kU];
+    auto issue = [&](int tb, int stage) {
 #pragma unroll
-        for (int u = 0; u < kU; ++u) raw[u] = (tb + u < t1) ? P::load(xb + (size_t)(tb + u) * D) : P::zero();
+        for (int u = 0; u < KU; ++u) {
+            const bool ok = active && tb + u < t1;
+            const int t = ok ? tb + u : t0;
+            cp_async<P::BYTES>(stg.at(stage, 0, u), xb + (size_t)t * D, ok);
+            if constexpr (kTapVec)
+                if (tap_stage) cp_async<TB>(stg.at(stage, 1, u), wb + (size_t)t * (D / G) * W, ok);
+        }
+        cp_commit();
+    };
+    const int nb = cdiv(t1 - t0, KU);
+    issue(t0, 0);
+    for (int bi = 0; bi < nb; ++bi) {
+        const int tb = t0 + bi * KU, stage = bi & 1;
+        if (bi + 1 < nb) issue(tb + KU, stage ^ 1);
+        else cp_commit();
+        cp_wait<1>();
+        if (!active) continue;
 #pragma unroll
-        for (int u = 0; u < kU; ++u) {
+        for (int u = 0; u < KU; ++u) {
             const int t = tb + u;
             if (t >= t1) break;
-            P::unpack(raw[u], win[0]);
-            if (!STATIC) dyn_taps<T, W, V>(w, (size_t)b * T_ + t, c0, D, G, f);
+            P::unpack(lds_raw<typename P::raw_t>(stg.at(stage, 0, u)), win[0]);
+            if constexpr (!STATIC) {
+                bool staged = false;
+                if constexpr (kTapVec) {
+                    if (tap_stage) {
+                        staged = true;
+                        using TR = typename RawOf<TB>::type;
+                        const TR tr = lds_raw<TR>(stg.at(stage, 1, u));
+                        uint32_t tw[TB / 4];
+                        if constexpr (TB == 4) {
+                            tw[0] = tr;
+                        } else if constexpr (TB == 8) {
+                            tw[0] = tr.x; tw[1] = tr.y;
+                        } else {
+                            tw[0] = tr.x; tw[1] = tr.y; tw[2] = tr.z; tw[3] = tr.w;
+                        }
+#pragma unroll
+                        for (int k = 0; k < W; ++k) {
+                            float fk;
+                            if constexpr (sizeof(T) == 2) fk = (k & 1) ? bf16_hi(tw[k / 2]) : bf16_lo(tw[k / 2]);
+                            else fk = __uint_as_float(tw[k]);
+#pragma unroll
+                            for (int i = 0; i < V; ++i) f[k][i] = fk;
+                        }
+                    }
+                }
+                if (!staged) dyn_taps<T, W, V>(w, (size_t)b * T_ + t, c0, D, G, f);
+            }
             float out[V];
 #pragma unroll
             for (int i = 0; i < V; ++i) {
@@ -163,7 +264,22 @@ k_stream_fwd(const T *__restrict__ x, const T *__restrict__ w, T *__restrict__ y
                 for (int i = 0; i < V; ++i) win[k][i] = win[k - 1][i];
         }
     }
+    cp_wait<0>();
 }
+
+template <typename T, int W, bool STATIC>
+__global__ void __launch_bounds__(256)
+k_stream_fwd(const T *__restrict__ x, const T *__restrict__ w, T *__restrict__ y, int B, int T_, int D,
+             int G, int chunk) {
+    // persistent: the grid is sized to the resident blocks, each walks work items
+    // (256 thread-vectors of channels x one chunk of one sequence) with a stride
+    constexpr int V0 = Lanes<T, W>::V;
+    const int nbx = cdiv(D / V0, 256);
+    const int nitems = nbx * B * cdiv(T_, chunk);
+    for (int item = blockIdx.x; item < nitems; item += gridDim.x)
+        stream_fwd_item<T, W, STATIC>(x, w, y, B, T_, D, G, chunk, item % nbx, item / nbx);
+}
+
 
 // ------------------------------------------------------------------ static backward
 // One pass over x and dy per chunk of tokens:
@@ -174,18 +290,21 @@ k_stream_fwd(const T *__restrict__ x, const T *__restrict__ w, T *__restrict__ y
 // The block's kBY chunks sum their dw in shared memory in a fixed order and write one
 // partial row part[p, c, k]; a second kernel adds the partials in order.
 template <typename T, int W>
-__global__ void __launch_bounds__(kBX * kBY)
-k_static_bwd(const T *__restrict__ x, const T *__restrict__ ws, const T *__restrict__ dy, T *__restrict__ dx,
-             float *__restrict__ part, int B, int T_, int D, int chunk) {
+__device__ __forceinline__ void static_bwd_item(const T *__restrict__ x, const T *__restrict__ ws,
+                                                const T *__restrict__ dy, T *__restrict__ dx,
+                                                float *__restrict__ part, int B, int T_, int D, int chunk,
+                                                int bx, int by) {
     constexpr int V = Lanes<T, W>::V;
     using P = Pack<T, V>;
+    constexpr int kU = Batch<P::BYTES>::KU;
     __shared__ float red[kBY][kBX][V];
-    const int v = blockIdx.x * kBX + threadIdx.x;
+    extern __shared__ __align__(16) uint8_t stg_raw[];
+    const int v = bx * kBX + threadIdx.x;
     const bool active = v < D / V;
     const int nch = cdiv(T_, chunk);
     const int ngr = cdiv(nch, kBY);
-    const int b = blockIdx.y / ngr;
-    const int ci = (blockIdx.y - b * ngr) * kBY + threadIdx.y;
+    const int b = by / ngr;
+    const int ci = (by - b * ngr) * kBY + threadIdx.y;
     const int t0 = ci * chunk;
     const int t1 = min(t0 + chunk, T_);
     const int c0 = v * V;
@@ -241,22 +360,34 @@ k_static_bwd(const T *__restrict__ x, const T *__restrict__ ws, const T *__restr
                     xw[k][i] = xw[k - 1][i];
                 }
         };
-        for (int tb = t0; tb < t1; tb += kU) {
-            typename P::raw_t rx[kU], rg[kU];
+        const Staging<P::BYTES, 2, kU, kBX * kBY> stg((uint32_t)__cvta_generic_to_shared(stg_raw),
+                                                  (int)(threadIdx.y * kBX + threadIdx.x));
+        auto issue = [&](int tb, int stage) {
 #pragma unroll
             for (int u = 0; u < kU; ++u) {
                 const bool ok = tb + u < t1;
-                rx[u] = ok ? P::load(x + off + (size_t)(tb + u) * D) : P::zero();
-                rg[u] = ok ? P::load(dy + off + (size_t)(tb + u) * D) : P::zero();
+                const size_t r = (size_t)(ok ? tb + u : t0) * D;
+                cp_async<P::BYTES>(stg.at(stage, 0, u), x + off + r, ok);
+                cp_async<P::BYTES>(stg.at(stage, 1, u), dy + off + r, ok);
             }
+            cp_commit();
+        };
+        const int nb = cdiv(t1 - t0, kU);
+        issue(t0, 0);
+        for (int bi = 0; bi < nb; ++bi) {
+            const int tb = t0 + bi * kU, stage = bi & 1;
+            if (bi + 1 < nb) issue(tb + kU, stage ^ 1);
+            else cp_commit();
+            cp_wait<1>();
 #pragma unroll
             for (int u = 0; u < kU; ++u) {
                 if (tb + u >= t1) break;
-                P::unpack(rx[u], xw[0]);
-                P::unpack(rg[u], dyw[0]);
+                P::unpack(lds_raw<typename P::raw_t>(stg.at(stage, 0, u)), xw[0]);
+                P::unpack(lds_raw<typename P::raw_t>(stg.at(stage, 1, u)), dyw[0]);
                 step(tb + u, true);
             }
         }
+        cp_wait<0>();
         // rows t1-W+1 .. t1-1 need dy rows t1 .. t1+W-2 (zero past the sequence end)
 #pragma unroll
         for (int e = 0; e < W - 1; ++e) {
@@ -279,11 +410,23 @@ k_static_bwd(const T *__restrict__ x, const T *__restrict__ ws, const T *__restr
                 float s = 0.f;
 #pragma unroll
                 for (int yy = 0; yy < kBY; ++yy) s += red[yy][threadIdx.x][i];
-                part[((size_t)blockIdx.y * D + c0 + i) * W + k] = s;
+                part[((size_t)by * D + c0 + i) * W + k] = s;
             }
         }
         __syncthreads();
     }
+}
+
+template <typename T, int W>
+__global__ void __launch_bounds__(kBX * kBY)
+k_static_bwd(const T *__restrict__ x, const T *__restrict__ ws, const T *__restrict__ dy, T *__restrict__ dx,
+             float *__restrict__ part, int B, int T_, int D, int chunk) {
+    // persistent: work item = (kBX channel vectors, kBY chunks of one sequence)
+    constexpr int V = Lanes<T, W>::V;
+    const int nbx = cdiv(D / V, kBX);
+    const int nitems = nbx * dw_partials(B, T_);
+    for (int item = blockIdx.x; item < nitems; item += gridDim.x)
+        static_bwd_item<T, W>(x, ws, dy, dx, part, B, T_, D, chunk, item % nbx, item / nbx);
 }
 
 // out[e] = sum_{p < P} part[p * n + e], in order of p.
@@ -298,7 +441,31 @@ __global__ void k_sum_partials(const float *__restrict__ part, float *__restrict
 // ------------------------------------------------------------------ launchers
 namespace {
 
-int chunk_for(int T) { return T < kChunk ? T : kChunk; }
+
+// Blocks of `kern` that fit on the device at once (at least one per SM).
+template <typename K>
+int resident_blocks(K kern, int threads, int smem) {
+    int dev = 0, nsm = 148, per = 1;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per, kern, threads, smem) != cudaSuccess || per < 1) per = 1;
+    return nsm * per;
+}
+
+template <typename T, int W, bool STATIC>
+void launch_fwd_k(int nitems, const T *x, const T *w, T *y, int B, int T_, int D, int G, int chunk,
+                  cudaStream_t s) {
+    constexpr int V = Lanes<T, W>::V;
+    constexpr int PB = V * (int)sizeof(T);
+    constexpr int TB = W * (int)sizeof(T);
+    constexpr bool kTapVec = !STATIC && (TB == 4 || TB == 8 || TB == 16);
+    constexpr int SB = PB > TB || !kTapVec ? PB : TB;
+    constexpr int smem = 256 * Staging<SB, kTapVec ? 2 : 1, Batch<SB>::KU>::bytes_per_thread();
+    auto kern = k_stream_fwd<T, W, STATIC>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    const int grid = std::min(nitems, resident_blocks(kern, 256, smem));
+    kern<<<grid, 256, smem, s>>>(x, w, y, B, T_, D, G, chunk);
+}
 
 template <typename T, bool STATIC>
 void launch_stream_fwd_T(const void *x, const void *w, void *y, int B, int T_, int D, int G, int W,
@@ -311,8 +478,8 @@ void launch_stream_fwd_T(const void *x, const void *w, void *y, int B, int T_, i
 #define DSC_CASE(WW)                                                                                  \
     case WW: {                                                                                        \
         constexpr int V = Lanes<T, WW>::V;                                                            \
-        const dim3 grid(cdiv(D / V, 256), B * cdiv(T_, chunk));                                       \
-        k_stream_fwd<T, WW, STATIC><<<grid, 256, 0, s>>>(xp, wp, yp, B, T_, D, G, chunk);             \
+        launch_fwd_k<T, WW, STATIC>(cdiv(D / V, 256) * B * cdiv(T_, chunk), xp, wp, yp, B, T_, D, G,  \
+                                    chunk, s);                                                        \
         break;                                                                                        \
     }
         DSC_CASE(1) DSC_CASE(2) DSC_CASE(3) DSC_CASE(4) DSC_CASE(5) DSC_CASE(6) DSC_CASE(7) DSC_CASE(8)
@@ -333,8 +500,12 @@ void launch_static_bwd_T(const void *x, const void *w, const void *dy, void *dx,
 #define DSC_CASE(WW)                                                                                  \
     case WW: {                                                                                        \
         constexpr int V = Lanes<T, WW>::V;                                                            \
-        const dim3 grid(cdiv(D / V, kBX), P);                                                         \
-        k_static_bwd<T, WW><<<grid, dim3(kBX, kBY), 0, s>>>(xp, wp, gp, op, part, B, T_, D, chunk);   \
+        constexpr int SB = V * (int)sizeof(T);                                                        \
+        const int smem = kBX * kBY * Staging<SB, 2, Batch<SB>::KU, kBX * kBY>::bytes_per_thread();    \
+        auto kern = k_static_bwd<T, WW>;                                                              \
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);                \
+        const int grid = std::min(cdiv(D / V, kBX) * P, resident_blocks(kern, kBX * kBY, smem));      \
+        kern<<<grid, dim3(kBX, kBY), smem, s>>>(xp, wp, gp, op, part, B, T_, D, chunk);               \
         break;                                                                                        \
     }
         DSC_CASE(1) DSC_CASE(2) DSC_CASE(3) DSC_CASE(4) DSC_CASE(5) DSC_CASE(6) DSC_CASE(7) DSC_CASE(8)
@@ -347,7 +518,7 @@ void launch_static_bwd_T(const void *x, const void *w, const void *dy, void *dx,
 
 }  // namespace
 
-int static_dw_partials(int B, int T) { return B * cdiv(cdiv(T, chunk_for(T)), kBY); }
+int static_dw_partials(int B, int T) { return dw_partials(B, T); }
 
 void launch_conv_fwd(const void *x, const void *w, void *y, int B, int T, int D, int G, int W, bool bf16_,
                      bool is_static, cudaStream_t s) {

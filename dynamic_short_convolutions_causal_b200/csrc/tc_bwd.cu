@@ -99,6 +99,7 @@ struct BwdParams {
     unsigned *flag_du;        // [Bg]   dU partials written per slice group (16 per CTA)
     float *dz;                // [B*T][R]
     float *dU;                // [R][N]
+    WaitTest wt;
 };
 
 struct Bars {
@@ -154,7 +155,7 @@ __device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
 // Waits until *p >= target.  Gives up like mbar_wait: after kWaitLimitNs, or as soon
 // as another warp of the CTA has given up.
 __device__ __forceinline__ bool wait_count(const unsigned *p, unsigned target, volatile int *abort,
-                                           unsigned code) {
+                                           unsigned code, unsigned long long limit_ns) {
     if (ld_acquire(p) >= target) return true;
     const unsigned long long t0 = globaltimer();
     while (true) {
@@ -164,7 +165,7 @@ __device__ __forceinline__ bool wait_count(const unsigned *p, unsigned target, v
             if (ld_acquire(p) >= target) return true;
         }
         if (*abort) return false;
-        if (globaltimer() - t0 > kWaitLimitNs) {
+        if (globaltimer() - t0 > limit_ns) {
             *abort = 1;
             atomicOr(&g_fault_bwd, code);
             return false;
@@ -287,13 +288,13 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
                 const int b = m / p.tiles_per_seq, t0 = (m - b * p.tiles_per_seq) * kTt;
                 if (i >= NST) {
                     // the stage is free once tile i-NST's dx, written over its x tile, is stored
-                    if (!mbar_wait(bar.dxr(st), (n - 1) & 1, abort, 1u, &g_fault_bwd)) { ok = false; break; }
+                    if (!mbar_wait(bar.dxr(st), (n - 1) & 1, abort, 1u, &g_fault_bwd, p.wt.wait_ns)) { ok = false; break; }
                     store_dx(i - NST);
                     bulk_wait_read<0>();
                 }
                 if (j == 0) {
                     const int zb = mz & 1;
-                    if (!mbar_wait(bar.zempty(zb), ((mz >> 1) & 1) ^ 1, abort, 2u, &g_fault_bwd)) { ok = false; break; }
+                    if (!mbar_wait(bar.zempty(zb), ((mz >> 1) & 1) ^ 1, abort, 2u, &g_fault_bwd, p.wt.wait_ns)) { ok = false; break; }
                     mbar_arrive_expect_tx(bar.zfull(zb), tx_z);
                     const uint32_t zd = sb + p.off_z + zb * p.z_bytes;
                     for (int r8 = 0; r8 < p.R / 8; ++r8)
@@ -302,19 +303,20 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
                 }
                 if (!u_res) {
                     const int ub = i & 1;
-                    if (!mbar_wait(bar.uempty(ub), ((i >> 1) & 1) ^ 1, abort, 2u, &g_fault_bwd)) { ok = false; break; }
+                    if (!mbar_wait(bar.uempty(ub), ((i >> 1) & 1) ^ 1, abort, 2u, &g_fault_bwd, p.wt.wait_ns)) { ok = false; break; }
                     load_up(ub, slice);
                     ++uissued;
                 }
+                ++issued;
+                if (i == 0 && (int)blockIdx.x == p.wt.withhold_cta) continue;   // test hook: no loads
                 mbar_arrive_expect_tx(bar.full(st), tx_xy);
                 const uint32_t sd = sb + st * p.stage_bytes;
                 tma_load_3d(sd, &tm_dy, bar.full(st), slice * kDt, t0, b);
                 tma_load_3d(sd + p.xy_tile_bytes, &tm_x, bar.full(st), slice * kDt, t0 - (W - 1), b);
-                ++issued;
             }
             if (ok) {
                 for (int i = (nt > NST ? nt - NST : 0); i < nt; ++i) {
-                    if (!mbar_wait(bar.dxr(i % NST), (i / NST) & 1, abort, 1u, &g_fault_bwd)) break;
+                    if (!mbar_wait(bar.dxr(i % NST), (i / NST) & 1, abort, 1u, &g_fault_bwd, p.wt.wait_ns)) break;
                     store_dx(i);
                 }
             }
@@ -322,14 +324,14 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             // Let every load this warp issued land before the CTA can exit (matters only
             // when another warp gave up early; otherwise all of them were consumed).
             for (int i = (issued > NST ? issued - NST : 0); i < issued; ++i)
-                mbar_drain(bar.full(i % NST), (i / NST) & 1);
+                mbar_drain(bar.full(i % NST), (i / NST) & 1, p.wt.wait_ns);
             for (int z = (zissued > 2 ? zissued - 2 : 0); z < zissued; ++z)
-                mbar_drain(bar.zfull(z & 1), (z >> 1) & 1);
+                mbar_drain(bar.zfull(z & 1), (z >> 1) & 1, p.wt.wait_ns);
             if (u_res) {
-                for (int u = 0; u < uissued; ++u) mbar_drain(bar.ufull(u), 0);
+                for (int u = 0; u < uissued; ++u) mbar_drain(bar.ufull(u), 0, p.wt.wait_ns);
             } else {
                 for (int u = (uissued > 2 ? uissued - 2 : 0); u < uissued; ++u)
-                    mbar_drain(bar.ufull(u & 1), (u >> 1) & 1);
+                    mbar_drain(bar.ufull(u & 1), (u >> 1) & 1, p.wt.wait_ns);
             }
         }
         __syncwarp();
@@ -347,9 +349,9 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             const int j = i % S, mz = i / S, zb = mz & 1;
             const int ub = u_res ? j : (i & 1);
             const int upar = u_res ? 0 : ((i >> 1) & 1);
-            if (j == 0 && !warp_wait(bar.zfull(zb), (mz >> 1) & 1, abort, 4u, &g_fault_bwd)) break;
-            if (!warp_wait(bar.ufull(ub), upar, abort, 4u, &g_fault_bwd)) break;
-            if (!warp_wait(bar.wempty(), (i & 1) ^ 1, abort, 16u, &g_fault_bwd)) break;
+            if (j == 0 && !warp_wait(bar.zfull(zb), (mz >> 1) & 1, abort, 4u, &g_fault_bwd, p.wt.wait_ns)) break;
+            if (!warp_wait(bar.ufull(ub), upar, abort, 4u, &g_fault_bwd, p.wt.wait_ns)) break;
+            if (!warp_wait(bar.wempty(), (i & 1) ^ 1, abort, 16u, &g_fault_bwd, p.wt.wait_ns)) break;
             tc_fence_after();
             const uint32_t zs = sb + p.off_z + zb * p.z_bytes;
             const uint32_t us = sb + p.off_u + ub * p.u_bytes;
@@ -398,11 +400,20 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
         const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
         const int nc = p.R / 4;              // dz columns a warp reads out (its group's share)
 
-        // dz partial of token tile mz (this CTA's slices) -> global memory; count in.
+        // dz partial of token tile mz (this CTA's slices) -> global memory.  The count that
+        // tells the reducers the partial is complete is released one token tile later: the
+        // gpu-scope fence before it then covers stores issued long before, instead of
+        // stalling the warp for a round trip to L2 right after issuing them.
+        auto dz_signal = [&](int mz) {
+            fence_gpu();
+            __syncwarp();
+            if (lane == 0) red_release_add(p.flag_dz + sp.m0 + mz, 1u);
+        };
         auto dz_out = [&](int mz) -> bool {
             const int db = mz & 1;
-            if (!warp_wait(bar.dzfull(db), (mz >> 1) & 1, abort, 256u, &g_fault_bwd)) return false;
+            if (!warp_wait(bar.dzfull(db), (mz >> 1) & 1, abort, 256u, &g_fault_bwd, p.wt.wait_ns)) return false;
             tc_fence_after();
+            if (mz > 0) dz_signal(mz - 1);           // partial mz-1 was stored a token tile ago
             const int m = sp.m0 + mz;
             const int b = m / p.tiles_per_seq, t0 = (m - b * p.tiles_per_seq) * kTt;
             const int tok = t0 + row;
@@ -416,12 +427,8 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
                 if (tok < p.T) *reinterpret_cast<uint4 *>(dst + c0) = make_uint4(v[0], v[1], v[2], v[3]);
             }
             tc_fence_before();
-            fence_gpu();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(bar.dzempty(db));
-                red_release_add(p.flag_dz + m, 1u);
-            }
+            if (lane == 0) mbar_arrive(bar.dzempty(db));
             return true;
         };
 
@@ -429,7 +436,7 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
         for (int i = 0; i < nt; ++i) {
             const int j = i % S, mz = i / S;
             const int st = i % NST, n = i / NST;
-            if (!warp_wait(bar.full(st), n & 1, abort, 64u, &g_fault_bwd)) { ok = false; break; }
+            if (!warp_wait(bar.full(st), n & 1, abort, 64u, &g_fault_bwd, p.wt.wait_ns)) { ok = false; break; }
             const uint32_t dys = sb + st * p.stage_bytes, xs = dys + p.xy_tile_bytes;
 
             // ---- A2: dw[t,g,k] = sum_{c in g} dy[t,c] x[t-k,c], tap-major column k*NG + g.
@@ -488,11 +495,11 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
                 uint32_t pk[CH][W][NPK];
 #pragma unroll
                 for (int cq = 0; cq < CH; ++cq) a2_compute(cq, pk[cq]);
-                if (!warp_wait(bar.dwfree(), (i & 1) ^ 1, abort, 32u, &g_fault_bwd)) { ok = false; break; }
+                if (!warp_wait(bar.dwfree(), (i & 1) ^ 1, abort, 32u, &g_fault_bwd, p.wt.wait_ns)) { ok = false; break; }
 #pragma unroll
                 for (int cq = 0; cq < CH; ++cq) a2_store(cq, pk[cq]);
             } else {
-                if (!warp_wait(bar.dwfree(), (i & 1) ^ 1, abort, 32u, &g_fault_bwd)) { ok = false; break; }
+                if (!warp_wait(bar.dwfree(), (i & 1) ^ 1, abort, 32u, &g_fault_bwd, p.wt.wait_ns)) { ok = false; break; }
 #pragma unroll 1
                 for (int cq = 0; cq < CH; ++cq) {
                     uint32_t pk[W][NPK];
@@ -505,7 +512,7 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             if (lane == 0) mbar_arrive(bar.dwready());
 
             // ---- A1: dx[t,c] = dy[t,c] + sum_k w[t+k,g,k] dy[t+k,c]
-            if (!warp_wait(bar.wfull(), i & 1, abort, 128u, &g_fault_bwd)) { ok = false; break; }
+            if (!warp_wait(bar.wfull(), i & 1, abort, 128u, &g_fault_bwd, p.wt.wait_ns)) { ok = false; break; }
             tc_fence_after();
             constexpr int NGB = 8 / G;                      // filter groups of one chunk
             constexpr int KB = (W * (4 + NGB) <= 48) ? W : 4;   // taps per batch
@@ -567,7 +574,7 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             // once every epilogue warp is past A2 the x tile is dead, and dx goes there
             // (an mbarrier rather than a named barrier, so that the wait is bounded)
             if (lane == 0) mbar_arrive(bar.xdead());
-            if (!warp_wait(bar.xdead(), i & 1, abort, 4096u, &g_fault_bwd)) { ok = false; break; }
+            if (!warp_wait(bar.xdead(), i & 1, abort, 4096u, &g_fault_bwd, p.wt.wait_ns)) { ok = false; break; }
 #pragma unroll
             for (int cq = 0; cq < CH; ++cq) sts128(xs + (dxr0 ^ ((uint32_t)cq << 4)), dxo[cq]);
             fence_proxy_async_smem();
@@ -578,9 +585,10 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             if (j == 0 && mz > 0 && !dz_out(mz - 1)) { ok = false; break; }
         }
         if (ok && nt > 0) ok = dz_out(nt / S - 1);
+        if (ok && nt > 0) dz_signal(nt / S - 1);
 
         // ---- dU: this CTA's partial of each of its slices, then the slice group's sum
-        if (ok && warp_wait(bar.dufull(), 0, abort, 512u, &g_fault_bwd)) {
+        if (ok && warp_wait(bar.dufull(), 0, abort, 512u, &g_fault_bwd, p.wt.wait_ns)) {
             tc_fence_after();
             const int N = p.n_slices * p.SC;
             for (int j = 0; j < S; ++j) {
@@ -606,7 +614,7 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             fence_gpu();
             __syncwarp();
             if (lane == 0) red_release_add(p.flag_du + sp.b, 1u);
-            if (wait_count(p.flag_du + sp.b, (unsigned)(kEpiWarps * p.A), abort, 1024u)) {
+            if (wait_count(p.flag_du + sp.b, (unsigned)(kEpiWarps * p.A), abort, 1024u, p.wt.wait_ns)) {
                 // this CTA's share (of A) of the group's R x (S*SC) block, float4-wise
                 const int cols = S * p.SC;
                 const long long n4 = (long long)p.R * cols / 4;
@@ -650,10 +658,10 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             const int j = i % S, mz = i / S, db = mz & 1, zb = mz & 1;
             const int ub = u_res ? j : (i & 1);
             const int upar = u_res ? 0 : ((i >> 1) & 1);
-            if (!warp_wait(bar.ufull(ub), upar, abort, 4u, &g_fault_bwd)) break;
-            if (j == 0 && !warp_wait(bar.zfull(zb), (mz >> 1) & 1, abort, 4u, &g_fault_bwd)) break;
-            if (!warp_wait(bar.dwready(), i & 1, abort, 8u, &g_fault_bwd)) break;
-            if (j == 0 && !warp_wait(bar.dzempty(db), ((mz >> 1) & 1) ^ 1, abort, 8u, &g_fault_bwd)) break;
+            if (!warp_wait(bar.ufull(ub), upar, abort, 4u, &g_fault_bwd, p.wt.wait_ns)) break;
+            if (j == 0 && !warp_wait(bar.zfull(zb), (mz >> 1) & 1, abort, 4u, &g_fault_bwd, p.wt.wait_ns)) break;
+            if (!warp_wait(bar.dwready(), i & 1, abort, 8u, &g_fault_bwd, p.wt.wait_ns)) break;
+            if (j == 0 && !warp_wait(bar.dzempty(db), ((mz >> 1) & 1) ^ 1, abort, 8u, &g_fault_bwd, p.wt.wait_ns)) break;
             tc_fence_after();
             {
                 const uint32_t us = sb + p.off_u + ub * p.u_bytes;
@@ -708,7 +716,7 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
         const size_t part_stride = (size_t)p.B * p.T * p.R;
         const unsigned target = (unsigned)(kEpiWarps * p.Bg);
         for (int m = sp.m0; m < sp.m1; ++m) {
-            if (!wait_count(p.flag_dz + m, target, abort, 2048u)) break;
+            if (!wait_count(p.flag_dz + m, target, abort, 2048u, p.wt.wait_ns)) break;
             const int b = m / p.tiles_per_seq, t0 = (m - b * p.tiles_per_seq) * kTt;
             const int nrows = min(kTt, p.T - t0);
             const int lo = (int)((long long)nrows * sp.b / p.Bg), hi = (int)((long long)nrows * (sp.b + 1) / p.Bg);
@@ -739,7 +747,7 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
 
     __syncthreads();
     if (warp == kRecWarp) {
-        if (lane == 0) mbar_drain(bar.done(), 0);
+        if (lane == 0) mbar_drain(bar.done(), 0, p.wt.wait_ns);
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, p.tmem_cols);
@@ -953,6 +961,7 @@ cudaError_t launch_tc_lowrank_bwd(const void *x, const void *z, const void *U, c
     using namespace tcb;
     BwdParams p;
     if (!plan_bwd(B, T, D, G, W, R, num_sms(), p)) return cudaErrorNotSupported;
+    take_wait_test(&p.wt.wait_ns, &p.wt.withhold_cta);
     const WsLayout l = ws_layout(p);
     uint8_t *w8 = (uint8_t *)ws;
     bf16 *Up = (bf16 *)(w8 + l.up);

@@ -13,6 +13,14 @@ namespace tc {
 
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;   // 1 s: far beyond any real wait
 
+// Test hook of the bounded waits (set from the host for one launch): every wait of the
+// launch gives up after wait_ns, and CTA `withhold_cta` skips the loads of its first
+// tile, so that a consumer's wait runs out and the teardown path runs.
+struct WaitTest {
+    unsigned long long wait_ns;   // kWaitLimitNs normally
+    int withhold_cta;             // -1 normally
+};
+
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
@@ -72,7 +80,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // on giving up it records `code` in the device fault word and returns false.
 template <unsigned HintNs = 0>
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort,
-                                          unsigned code, unsigned *fault) {
+                                          unsigned code, unsigned *fault,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait<HintNs>(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     while (true) {
@@ -80,7 +89,7 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
         for (int i = 0; i < 32; ++i)
             if (mbar_try_wait<HintNs>(bar, parity)) return true;
         if (*abort) return false;
-        if (globaltimer() - t0 > kWaitLimitNs) {
+        if (globaltimer() - t0 > limit_ns) {
             *abort = 1;
             atomicOr(fault, code);
             return false;
@@ -91,18 +100,19 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 // Waits for a phase that is known to complete (a TMA load or MMAs already issued), even
 // after the CTA has given up on its other waits, so that nothing is still writing to
 // shared memory or TMEM when the CTA frees them and exits.  Bounded by kWaitLimitNs.
-__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity) {
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity,
+                                           unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return;
     const unsigned long long t0 = globaltimer();
     while (!mbar_try_wait(bar, parity))
-        if (globaltimer() - t0 > kWaitLimitNs) return;
+        if (globaltimer() - t0 > limit_ns) return;
 }
 
 // mbar_wait by every lane of a warp, with one warp-uniform outcome.
 template <unsigned HintNs = 0>
 __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity, volatile int *abort, unsigned code,
-                                          unsigned *fault) {
-    const bool ok = mbar_wait<HintNs>(bar, parity, abort, code, fault);
+                                          unsigned *fault, unsigned long long limit_ns = kWaitLimitNs) {
+    const bool ok = mbar_wait<HintNs>(bar, parity, abort, code, fault, limit_ns);
     return __all_sync(0xffffffffu, ok);
 }
 

@@ -66,6 +66,7 @@ struct FwdParams {
     uint32_t stage_bytes;     // one ring stage: x tile, z tile and the U slice
     uint32_t off_x, off_z, off_u, off_y, off_bar;   // off_x/z/u within a stage
     uint32_t z_layout;        // swizzle of the z tile (32/64/128-byte rows)
+    WaitTest wt;
 };
 
 // Barrier slots in shared memory (8 bytes each).
@@ -199,7 +200,8 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
                 const int slice = i % p.n_slices, tl_ = i / p.n_slices;
                 const int b = tl_ / p.tiles_per_seq, t0 = (tl_ % p.tiles_per_seq) * kTt;
                 const int s = it % S, n = it / S;
-                if (!mbar_wait<kWaitHint>(bar.empty(s), (n & 1) ^ 1, abort, 2u, &g_fault)) break;
+                if (!mbar_wait<kWaitHint>(bar.empty(s), (n & 1) ^ 1, abort, 2u, &g_fault, p.wt.wait_ns)) break;
+                if (it == 0 && (int)blockIdx.x == p.wt.withhold_cta) continue;   // test hook: no loads
                 mbar_arrive_expect_tx(bar.full(s), p.x_stage_tx + p.z_stage_bytes + p.u_bytes);
                 const uint32_t st = sb + s * p.stage_bytes;
                 tma_load_3d(st + p.off_x, &tm_x, bar.full(s), slice * kDt, t0 - (W - 1), b);
@@ -212,7 +214,7 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
             const int issued = it;
             for (int s = 0; s < S && s < issued; ++s) {
                 const int last = issued - 1 - ((issued - 1 - s) % S);   // last tile using stage s
-                mbar_drain(bar.full(s), (last / S) & 1);
+                mbar_drain(bar.full(s), (last / S) & 1, p.wt.wait_ns);
             }
         }
         __syncwarp();
@@ -231,8 +233,8 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
         for (int i = blockIdx.x; i < p.n_tiles; i += gridDim.x, ++it) {
             const int s = it % S, n = it / S;
             const int a = it % p.nbuf, m = it / p.nbuf;
-            if (!warp_wait<kWaitHint>(bar.full(s), n & 1, abort, 8u, &g_fault)) break;
-            if (!warp_wait<kWaitHint>(bar.acce(a), (m & 1) ^ 1, abort, 16u, &g_fault)) break;
+            if (!warp_wait<kWaitHint>(bar.full(s), n & 1, abort, 8u, &g_fault, p.wt.wait_ns)) break;
+            if (!warp_wait<kWaitHint>(bar.acce(a), (m & 1) ^ 1, abort, 16u, &g_fault, p.wt.wait_ns)) break;
             tc_fence_after();
             const uint32_t d = tmem + a * p.bufcols;
             const uint32_t za = sb + s * p.stage_bytes + p.off_z;
@@ -281,8 +283,8 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
             const int b = tlin / p.tiles_per_seq, t0 = (tlin - b * p.tiles_per_seq) * kTt;
             const int s = it % S, n = it / S;
             const int a = it % p.nbuf, m = it / p.nbuf;
-            if (!warp_wait<kWaitHint>(bar.full(s), n & 1, abort, 32u, &g_fault)) break;
-            if (!warp_wait<kWaitHint>(bar.accf(a), m & 1, abort, 64u, &g_fault)) break;
+            if (!warp_wait<kWaitHint>(bar.full(s), n & 1, abort, 32u, &g_fault, p.wt.wait_ns)) break;
+            if (!warp_wait<kWaitHint>(bar.accf(a), m & 1, abort, 64u, &g_fault, p.wt.wait_ns)) break;
             tc_fence_after();
             const int yb = yc & 1;
             if (lane == 0) bulk_wait_read<1>();
@@ -344,7 +346,7 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
 
     __syncthreads();
     if (warp == 1) {
-        if (lane == 0) mbar_drain(bar.done(), 0);
+        if (lane == 0) mbar_drain(bar.done(), 0, p.wt.wait_ns);
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, p.tmem_cols);
@@ -488,6 +490,7 @@ cudaError_t launch_tc_lowrank_fwd(const void *x, const void *z, const void *U, v
     using namespace tc;
     FwdParams p;
     if (!plan_fwd(B, T, D, G, W, R, p)) return cudaErrorNotSupported;
+    take_wait_test(&p.wt.wait_ns, &p.wt.withhold_cta);
     CUtensorMap mx, mz, mu, my;
     const uint64_t dx[3] = {(uint64_t)D, (uint64_t)T, (uint64_t)B};
     const uint32_t bx[3] = {(uint32_t)kDt, (uint32_t)(kTt + W - 1), 1};

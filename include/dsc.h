@@ -197,6 +197,15 @@ DSC_API int dsc_lowrank_path(int B, int T, int D, int G, int W, int R, dsc_dtype
  * clears the word afterwards. */
 DSC_API unsigned dsc_device_fault(int reset);
 
+/* Test hook for the tensor-core kernels' bounded waits; not for production use.  Arms
+ * the next dsc_fwd_lowrank or dsc_bwd_lowrank call on this host thread that runs on the
+ * tensor-core kernels: in that launch every wait gives up after wait_limit_us
+ * microseconds, and one CTA withholds the loads of its first tile, so that a wait does
+ * run out.  The call returns DSC_OK, its outputs are undefined, and dsc_device_fault()
+ * then reports a nonzero code; nothing faults or hangs, and later calls run normally.
+ * The hook exists so that the give-up-and-clean-up path can be tested. */
+DSC_API void dsc_test_arm_wait_timeout(unsigned wait_limit_us);
+
 /* Static description of a status code. */
 DSC_API const char *dsc_status_string(dsc_status_t status);
 
