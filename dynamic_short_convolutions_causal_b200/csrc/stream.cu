@@ -75,11 +75,13 @@ struct Lanes {
     static constexpr int V = sizeof(T) == 2 ? (W <= 4 ? 4 : 2) : (W <= 4 ? 4 : 2);
 };
 
-constexpr int kChunk = 128;        // tokens per thread (the W-1 row halo is re-read)
+constexpr int kChunk = 128;        // tokens per thread in the backward (the W-1 row halos are re-read)
+constexpr int kChunkFwd = 32;      // in the forward: more, shorter token walks in parallel
 constexpr int kBX = 32;            // threads along channels (one warp)
 constexpr int kBY = 8;             // chunks per block in the static backward
 
 __host__ __device__ inline int chunk_for(int T) { return T < kChunk ? T : kChunk; }
+inline int chunk_fwd(int T) { return T < kChunkFwd ? T : kChunkFwd; }
 __host__ __device__ inline int dw_partials(int B, int T) { return B * cdiv(cdiv(T, chunk_for(T)), kBY); }
 
 // cp.async of BYTES (4, 8 or 16) from global to shared memory; when `valid` is false the
@@ -271,8 +273,8 @@ template <typename T, int W, bool STATIC>
 __global__ void __launch_bounds__(256)
 k_stream_fwd(const T *__restrict__ x, const T *__restrict__ w, T *__restrict__ y, int B, int T_, int D,
              int G, int chunk) {
-    // persistent: the grid is sized to the resident blocks, each walks work items
-    // (256 thread-vectors of channels x one chunk of one sequence) with a stride
+    // work item = 256 thread-vectors of channels x one chunk of one sequence; the grid
+    // has one block per item (the loop also serves smaller grids)
     constexpr int V0 = Lanes<T, W>::V;
     const int nbx = cdiv(D / V0, 256);
     const int nitems = nbx * B * cdiv(T_, chunk);
@@ -463,14 +465,14 @@ void launch_fwd_k(int nitems, const T *x, const T *w, T *y, int B, int T_, int D
     constexpr int smem = 256 * Staging<SB, kTapVec ? 2 : 1, Batch<SB>::KU>::bytes_per_thread();
     auto kern = k_stream_fwd<T, W, STATIC>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    const int grid = std::min(nitems, resident_blocks(kern, 256, smem));
-    kern<<<grid, 256, smem, s>>>(x, w, y, B, T_, D, G, chunk);
+    // one work item per block: short-lived blocks overlap each other's first loads
+    kern<<<nitems, 256, smem, s>>>(x, w, y, B, T_, D, G, chunk);
 }
 
 template <typename T, bool STATIC>
 void launch_stream_fwd_T(const void *x, const void *w, void *y, int B, int T_, int D, int G, int W,
                          cudaStream_t s) {
-    const int chunk = chunk_for(T_);
+    const int chunk = chunk_fwd(T_);
     const T *xp = (const T *)x;
     const T *wp = (const T *)w;
     T *yp = (T *)y;

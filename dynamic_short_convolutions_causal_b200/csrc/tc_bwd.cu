@@ -34,9 +34,10 @@
 //               TMA store of dx from the stage once the epilogue has written it there
 //   warp 1      recompute: one MMA per tap k with the z tile shifted by k rows,
 //                 Wk[t, g] = sum_r z[t0+t+k, r] Up[r, k*NG+g],
-//               so TMEM lane t holds w[t+k, g, k] for every k
-//   warp 2      dz[m] += dw Up^T  (A = dw tile, B = Up slice; M=128 tokens, N=R) and
-//               dU^T[s] += dw^T z  (A = dw tile read MN-major, B = z; M=128 columns)
+//               so TMEM lane t holds w[t+k, g, k] for every k; and
+//               dz[m] += dw Up^T  (A = dw tile, B = Up slice; M=128 tokens, N=R)
+//   warp 2      dU^T[s] += dw^T z  (A = dw tile read MN-major, B = z; M=128 columns),
+//               and the gpu-scope publication of each finished dz partial
 //   warp 3      reducer: sums the dz partials of its rows of each token tile
 //   warps 4-19  epilogue, one token row per thread, 16 channels per warp:
 //                 A2: dw (bf16) into the shared-memory dw tile;
@@ -69,7 +70,7 @@ constexpr int kCPW = kDt / 4;                   // channels per epilogue warp
 // Warp roles.  Warps 0-3 sit on the SM's four sub-partitions, one each, and the
 // epilogue warps 4-19 four to a sub-partition; 20 warps keep 96 registers a thread.
 constexpr int kRecWarp = 1;
-constexpr int kMmaWarp = 2;                     // dz and dU MMAs
+constexpr int kMmaWarp = 2;                     // dU MMAs, dz partial publication
 constexpr int kRedWarp = 3;
 constexpr int kEpi0 = 4;
 constexpr int kThreads = 32 * (kEpi0 + kEpiWarps);
@@ -119,8 +120,9 @@ struct Bars {
     __device__ uint32_t dufull() const { return base + 8 * 22; }
     __device__ uint32_t done() const { return base + 8 * 23; }
     __device__ uint32_t xdead() const { return base + 8 * 24; }
+    __device__ uint32_t dzdone(int d) const { return base + 8 * (25 + d); }
 };
-constexpr uint32_t kBarBytes = 8 * 25;
+constexpr uint32_t kBarBytes = 8 * 29;
 
 __device__ __forceinline__ void unpack8(const uint4 &u, float (&v)[8]) {
     v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x);
@@ -221,14 +223,15 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             mbar_init(bar.zfull(z), 1);
             mbar_init(bar.zempty(z), 2);        // recompute and dz/dU streams
             mbar_init(bar.ufull(z), 1);
-            mbar_init(bar.uempty(z), 2);        // recompute and dz/dU streams
+            mbar_init(bar.uempty(z), 1);        // the recompute/dz stream (commit after dz)
             mbar_init(bar.dzfull(z), 1);
             mbar_init(bar.dzempty(z), kEpiWarps);
         }
+        for (int z = 0; z < 4; ++z) mbar_init(bar.dzdone(z), kEpiWarps);
         mbar_init(bar.wfull(), 1);
         mbar_init(bar.wempty(), kEpiWarps);
         mbar_init(bar.dwready(), kEpiWarps);
-        mbar_init(bar.dwfree(), 1);
+        mbar_init(bar.dwfree(), 2);             // dz and dU streams
         mbar_init(bar.dufull(), 1);
         mbar_init(bar.done(), 2);               // recompute and dz/dU streams
         mbar_init(bar.xdead(), kEpiWarps);      // every epilogue warp is past A2
@@ -336,22 +339,35 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
         }
         __syncwarp();
     } else if (warp == kRecWarp) {
-        // ---------------------------------------------------------- MMA issuer: recompute
+        // ---------------------------------------------------------- MMA issuer: recompute, dz
         // Each MMA warp runs its schedule warp-uniformly; one elected lane issues each
         // tcgen05 instruction, and descriptors advance by adding to their start field.
-        const uint64_t t_zk = desc_tmpl(p.z_slab, 128, kSwNone);               // z, K-major, no swizzle
-        const uint64_t t_u_mn = desc_tmpl((uint32_t)(p.R * 128), 1024, kSw128);  // Up as MN-major B
+        // Order: recompute(0); then per tile i: dz(i) once its dw is written, and
+        // recompute(i+1) once the epilogue has read the filters of tile i.
+        //   recompute: Wk[t, g] = sum_r z[t0+t+k, r] Up[r, k*NG+g], one MMA chain per tap
+        //     with the z tile shifted by k rows (A: z, K-major; B: Up, MN-major);
+        //   dz[m] (+)= dw Up^T: A = dw tile (K-major view), B = Up slice (K-major), 16
+        //     columns per step; accumulates over the token tile's slices.
+        constexpr int SC = (kDt / G) * W;
+        constexpr int KSC = SC / 16;
+        const uint64_t t_zk = desc_tmpl(p.z_slab, 128, kSwNone);
+        const uint64_t t_u_mn = desc_tmpl((uint32_t)(p.R * 128), 1024, kSw128);
+        const uint64_t t_k128 = desc_tmpl(16, 1024, kSw128);
         const uint32_t i_rec = idesc_bf16(128, p.NGp, false, true);
+        const uint32_t i_dz = idesc_bf16(128, p.R, false, false);
         const int ksr = p.R / 16;
         const uint32_t ubox = (uint32_t)(p.R * 128);
-        const uint64_t st_zk = (2 * p.z_slab) >> 4;   // 16 more z columns (start field units)
-        for (int i = 0; i < nt; ++i) {
+        const uint64_t st_zk = (2 * p.z_slab) >> 4;       // 16 more z columns (start field units)
+        const uint64_t st_wrap_a = (16384u - 96u) >> 4;   // next 64-column dw atom
+        const uint64_t st_wrap_b = (ubox - 96u) >> 4;     // next 64-column Up box
+        const uint32_t dw0 = sb + p.off_dw;
+        auto recompute = [&](int i) -> bool {
             const int j = i % S, mz = i / S, zb = mz & 1;
             const int ub = u_res ? j : (i & 1);
             const int upar = u_res ? 0 : ((i >> 1) & 1);
-            if (j == 0 && !warp_wait(bar.zfull(zb), (mz >> 1) & 1, abort, 4u, &g_fault_bwd, p.wt.wait_ns)) break;
-            if (!warp_wait(bar.ufull(ub), upar, abort, 4u, &g_fault_bwd, p.wt.wait_ns)) break;
-            if (!warp_wait(bar.wempty(), (i & 1) ^ 1, abort, 16u, &g_fault_bwd, p.wt.wait_ns)) break;
+            if (j == 0 && !warp_wait(bar.zfull(zb), (mz >> 1) & 1, abort, 4u, &g_fault_bwd, p.wt.wait_ns)) return false;
+            if (!warp_wait(bar.ufull(ub), upar, abort, 4u, &g_fault_bwd, p.wt.wait_ns)) return false;
+            if (!warp_wait(bar.wempty(), (i & 1) ^ 1, abort, 16u, &g_fault_bwd, p.wt.wait_ns)) return false;
             tc_fence_after();
             const uint32_t zs = sb + p.off_z + zb * p.z_bytes;
             const uint32_t us = sb + p.off_u + ub * p.u_bytes;
@@ -371,9 +387,41 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             if (elect_one()) {
                 mma_commit(bar.wfull());
                 if (j == S - 1) mma_commit(bar.zempty(zb));
-                if (!u_res) mma_commit(bar.uempty(ub));
             }
             __syncwarp();
+            return true;
+        };
+        auto dz_mma = [&](int i) -> bool {
+            const int j = i % S, mz = i / S, db = mz & 1;
+            const int ub = u_res ? j : (i & 1);
+            if (!warp_wait(bar.dwready(), i & 1, abort, 8u, &g_fault_bwd, p.wt.wait_ns)) return false;
+            if (j == 0 && !warp_wait(bar.dzempty(db), ((mz >> 1) & 1) ^ 1, abort, 8u, &g_fault_bwd, p.wt.wait_ns))
+                return false;
+            tc_fence_after();
+            const uint32_t us = sb + p.off_u + ub * p.u_bytes;
+            uint64_t da = desc_at(t_k128, dw0), dbd = desc_at(t_k128, us);
+            const uint32_t d = tmem + p.tm_dz + db * p.R;
+#pragma unroll
+            for (int kk = 0; kk < KSC; ++kk) {
+                if (elect_one()) mma_bf16_ss(d, da, dbd, i_dz, (j > 0 || kk > 0) ? 1u : 0u);
+                __syncwarp();
+                const bool wrap = (kk & 3) == 3;
+                da += wrap ? st_wrap_a : 2u;
+                dbd += wrap ? st_wrap_b : 2u;
+            }
+            if (elect_one()) {
+                mma_commit(bar.dwfree());
+                if (!u_res) mma_commit(bar.uempty(ub));   // recompute(i) and dz(i) read Up
+                if (j == S - 1) mma_commit(bar.dzfull(db));
+            }
+            __syncwarp();
+            return true;
+        };
+        if (nt > 0 && recompute(0)) {
+            for (int i = 0; i < nt; ++i) {
+                if (!dz_mma(i)) break;
+                if (i + 1 < nt && !recompute(i + 1)) break;
+            }
         }
         if (elect_one()) mma_commit(bar.done());
         __syncwarp();
@@ -400,20 +448,13 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
         const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
         const int nc = p.R / 4;              // dz columns a warp reads out (its group's share)
 
-        // dz partial of token tile mz (this CTA's slices) -> global memory.  The count that
-        // tells the reducers the partial is complete is released one token tile later: the
-        // gpu-scope fence before it then covers stores issued long before, instead of
-        // stalling the warp for a round trip to L2 right after issuing them.
-        auto dz_signal = [&](int mz) {
-            fence_gpu();
-            __syncwarp();
-            if (lane == 0) red_release_add(p.flag_dz + sp.m0 + mz, 1u);
-        };
+        // dz partial of token tile mz (this CTA's slices) -> global memory.  The warps then
+        // arrive on a CTA barrier; the reducer warp, off the epilogue's critical path, makes
+        // the partial visible to the other CTAs (gpu-scope release of the tile's count).
         auto dz_out = [&](int mz) -> bool {
             const int db = mz & 1;
             if (!warp_wait(bar.dzfull(db), (mz >> 1) & 1, abort, 256u, &g_fault_bwd, p.wt.wait_ns)) return false;
             tc_fence_after();
-            if (mz > 0) dz_signal(mz - 1);           // partial mz-1 was stored a token tile ago
             const int m = sp.m0 + mz;
             const int b = m / p.tiles_per_seq, t0 = (m - b * p.tiles_per_seq) * kTt;
             const int tok = t0 + row;
@@ -428,7 +469,10 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar.dzempty(db));
+            if (lane == 0) {
+                mbar_arrive(bar.dzempty(db));
+                mbar_arrive(bar.dzdone(mz & 3));
+            }
             return true;
         };
 
@@ -585,7 +629,6 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             if (j == 0 && mz > 0 && !dz_out(mz - 1)) { ok = false; break; }
         }
         if (ok && nt > 0) ok = dz_out(nt / S - 1);
-        if (ok && nt > 0) dz_signal(nt / S - 1);
 
         // ---- dU: this CTA's partial of each of its slices, then the slice group's sum
         if (ok && warp_wait(bar.dufull(), 0, abort, 512u, &g_fault_bwd, p.wt.wait_ns)) {
@@ -634,78 +677,67 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
-        // ---------------------------------------------------------- MMA issuer: dz and dU
-        // Once tile i's dw is written:
-        //   dz[m] (+)= dw Up^T: A = dw tile (K-major view), B = Up slice (K-major), 16
-        //     columns per step (+32 bytes within a 64-column atom, the next atom every 4
-        //     steps); accumulates over the token tile's slices;
-        //   dU^T[slice] (+)= dw^T z: A = dw^T (MN-major), B = z tile rows 0..127
-        //     (MN-major), 16 tokens per step; accumulates over the CTA's token tiles.
-        // The step counts are compile-time, so the issue loops unroll fully.
+        // ---------------------------------------------------------- MMA issuer: dU
+        // dU^T[slice] (+)= dw^T z once tile i's dw is written: A = dw^T (MN-major), B = z
+        // tile rows 0..127 (MN-major), 16 tokens per step; accumulates over the CTA's
+        // token tiles.  After issuing a tile, the warp also publishes a finished dz
+        // partial (see dz_publish): its wait there is already satisfied, and the fence it
+        // takes overlaps the next tile's epilogue work instead of holding up the epilogue.
         constexpr int SC = (kDt / G) * W;
-        constexpr int KSC = SC / 16;
         constexpr int NMB = (SC + 127) / 128;
-        const uint64_t t_k128 = desc_tmpl(16, 1024, kSw128);
         const uint64_t t_dwt = desc_tmpl(16384, 1024, kSw128);
         const uint64_t t_zmn = desc_tmpl(128, p.z_slab, kSwNone);
-        const uint32_t i_dz = idesc_bf16(128, p.R, false, false);
         const uint32_t i_du = idesc_bf16(128, p.R, true, true);
-        const uint32_t ubox = (uint32_t)(p.R * 128);
-        const uint64_t st_wrap_a = (16384u - 96u) >> 4;   // next 64-column dw atom
-        const uint64_t st_wrap_b = (ubox - 96u) >> 4;     // next 64-column Up box
         const uint32_t dw0 = sb + p.off_dw;
-        for (int i = 0; i < nt; ++i) {
-            const int j = i % S, mz = i / S, db = mz & 1, zb = mz & 1;
-            const int ub = u_res ? j : (i & 1);
-            const int upar = u_res ? 0 : ((i >> 1) & 1);
-            if (!warp_wait(bar.ufull(ub), upar, abort, 4u, &g_fault_bwd, p.wt.wait_ns)) break;
+        int published = 0;                 // token tiles whose dz partial has been published
+        // The epilogue arrives on dzdone[mz % 4] once token tile mz's partial is stored; a
+        // gpu-scope fence, then one add of 16 to the tile's counter, make it visible.
+        auto dz_publish = [&](int upto) -> bool {   // publish token tiles [published, upto)
+            for (; published < upto; ++published) {
+                const int mz = published;
+                if (!warp_wait(bar.dzdone(mz & 3), (mz >> 2) & 1, abort, 2048u, &g_fault_bwd, p.wt.wait_ns))
+                    return false;
+                fence_gpu();
+                __syncwarp();
+                if (lane == 0) red_release_add(p.flag_dz + sp.m0 + mz, (unsigned)kEpiWarps);
+                __syncwarp();
+            }
+            return true;
+        };
+        bool ok = true;
+        for (int i = 0; i < nt && ok; ++i) {
+            const int j = i % S, mz = i / S, zb = mz & 1;
             if (j == 0 && !warp_wait(bar.zfull(zb), (mz >> 1) & 1, abort, 4u, &g_fault_bwd, p.wt.wait_ns)) break;
             if (!warp_wait(bar.dwready(), i & 1, abort, 8u, &g_fault_bwd, p.wt.wait_ns)) break;
-            if (j == 0 && !warp_wait(bar.dzempty(db), ((mz >> 1) & 1) ^ 1, abort, 8u, &g_fault_bwd, p.wt.wait_ns)) break;
             tc_fence_after();
-            {
-                const uint32_t us = sb + p.off_u + ub * p.u_bytes;
-                uint64_t da = desc_at(t_k128, dw0), dbd = desc_at(t_k128, us);
-                const uint32_t d = tmem + p.tm_dz + db * p.R;
+            const uint32_t zs = sb + p.off_z + zb * p.z_bytes;
 #pragma unroll
-                for (int kk = 0; kk < KSC; ++kk) {
-                    if (elect_one()) mma_bf16_ss(d, da, dbd, i_dz, (j > 0 || kk > 0) ? 1u : 0u);
+            for (int mb = 0; mb < NMB; ++mb) {
+                const uint32_t d = tmem + p.tm_du + (j * NMB + mb) * p.R;
+                uint64_t da = desc_at(t_dwt, dw0 + mb * 32768u), dbd = desc_at(t_zmn, zs);
+#pragma unroll
+                for (int kk = 0; kk < kTt / 16; ++kk) {
+                    if (elect_one()) mma_bf16_ss(d, da, dbd, i_du, (mz == 0 && kk == 0) ? 0u : 1u);
                     __syncwarp();
-                    const bool wrap = (kk & 3) == 3;
-                    da += wrap ? st_wrap_a : 2u;
-                    dbd += wrap ? st_wrap_b : 2u;
-                }
-            }
-            {
-                const uint32_t zs = sb + p.off_z + zb * p.z_bytes;
-#pragma unroll
-                for (int mb = 0; mb < NMB; ++mb) {
-                    const uint32_t d = tmem + p.tm_du + (j * NMB + mb) * p.R;
-                    uint64_t da = desc_at(t_dwt, dw0 + mb * 32768u), dbd = desc_at(t_zmn, zs);
-#pragma unroll
-                    for (int kk = 0; kk < kTt / 16; ++kk) {
-                        if (elect_one()) mma_bf16_ss(d, da, dbd, i_du, (mz == 0 && kk == 0) ? 0u : 1u);
-                        __syncwarp();
-                        da += 2048u >> 4;
-                        dbd += 256u >> 4;
-                    }
+                    da += 2048u >> 4;
+                    dbd += 256u >> 4;
                 }
             }
             if (elect_one()) {
                 mma_commit(bar.dwfree());
-                if (!u_res) mma_commit(bar.uempty(ub));
-                if (j == S - 1) {
-                    mma_commit(bar.dzfull(db));
-                    mma_commit(bar.zempty(zb));
-                }
+                if (j == S - 1) mma_commit(bar.zempty(zb));
             }
             __syncwarp();
+            // tile i-1 being the first of a token tile mz' means the partial of mz'-1 was
+            // stored (in that tile's epilogue, before the dw of tile i)
+            if (i >= 1 && (i - 1) % S == 0) ok = dz_publish((i - 1) / S);
         }
         if (elect_one()) {
             mma_commit(bar.dufull());
             mma_commit(bar.done());
         }
         __syncwarp();
+        if (ok) dz_publish(nt / S);        // the last token tiles
     } else if (warp == kRedWarp) {
         // ---------------------------------------------------------- dz reducer
         // Once all Bg slice groups have written their partial of token tile m, sum this

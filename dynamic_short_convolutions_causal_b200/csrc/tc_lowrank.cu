@@ -12,12 +12,16 @@
 // The x tile (plus its W-1 row causal halo; TMA fills rows before t=0 with zeros),
 // the z tile and the U slice arrive by TMA; y leaves through shared memory by TMA.
 //
-// Warp roles (persistent CTAs, one per SM, each owning a contiguous range of tiles in
-// slice-major order so that the U slice changes rarely):
-//   warp 0  TMA producer (x, z per tile; U per slice), 4-stage ring
-//   warp 1  TMEM allocator and MMA issuer (one thread), double-buffered accumulator
-//   warps 2-9  epilogue: warp w reads TMEM lanes 32*(w%4).. (its 32 tokens) and handles
-//              32 channels (half the slice); one token row per thread.
+// Warp roles (persistent CTAs, one per SM, tiles in token-major round-robin order):
+//   warp 0  TMA producer: the MMA operands of a tile (z tile, U slice) into a 2-deep
+//           operand ring that the MMA releases as soon as its MMAs complete, and the x
+//           tile into a deeper x ring that the epilogue releases.  Splitting the two keeps
+//           the x loads several tiles ahead of the epilogue, which both epilogue sets
+//           need: each holds one x stage while it works.
+//   warp 1  TMEM allocator and MMA issuer (one elected lane), double-buffered accumulator
+//   warps 2-17  two epilogue sets of 8 warps taking alternating tiles: warp w reads TMEM
+//              lanes 32*(w%4).. (its 32 tokens) and handles 32 channels (half the slice);
+//              one token row per thread.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -61,24 +65,31 @@ struct FwdParams {
     int n_pad;                // slice_cols rounded up to 16
     int u_boxes;              // ceil(n_pad / 64) TMA boxes of 64 columns
     int bufcols, nbuf, tmem_cols;
-    int stages, nwg;          // nwg: epilogue warp sets (1 or 2)
+    int stages, nwg;          // x ring depth; nwg: epilogue warp sets (1 or 2)
+    int op_stages;            // operand (z, U) ring depth
     uint32_t x_stage_tx, x_stage_bytes, z_stage_bytes, u_bytes, y_buf_bytes;
-    uint32_t stage_bytes;     // one ring stage: x tile, z tile and the U slice
-    uint32_t off_x, off_z, off_u, off_y, off_bar;   // off_x/z/u within a stage
+    uint32_t op_bytes;        // one operand stage: z tile and U slice
+    uint32_t off_x, off_op, off_y, off_bar;   // ring bases
+    uint32_t off_z, off_u;    // within an operand stage
     uint32_t z_layout;        // swizzle of the z tile (32/64/128-byte rows)
     WaitTest wt;
 };
 
 // Barrier slots in shared memory (8 bytes each).
+constexpr int kMaxXStages = 8;
+constexpr int kOpStages = 2;
+
 struct Bars {
     uint32_t base;
     __device__ uint32_t full(int s) const { return base + 8 * s; }
-    __device__ uint32_t empty(int s) const { return base + 8 * (4 + s); }
-    __device__ uint32_t accf(int a) const { return base + 8 * (8 + a); }
-    __device__ uint32_t acce(int a) const { return base + 8 * (10 + a); }
-    __device__ uint32_t done() const { return base + 8 * 12; }
+    __device__ uint32_t empty(int s) const { return base + 8 * (kMaxXStages + s); }
+    __device__ uint32_t ofull(int o) const { return base + 8 * (2 * kMaxXStages + o); }
+    __device__ uint32_t oempty(int o) const { return base + 8 * (2 * kMaxXStages + kOpStages + o); }
+    __device__ uint32_t accf(int a) const { return base + 8 * (2 * kMaxXStages + 2 * kOpStages + a); }
+    __device__ uint32_t acce(int a) const { return base + 8 * (2 * kMaxXStages + 2 * kOpStages + 2 + a); }
+    __device__ uint32_t done() const { return base + 8 * (2 * kMaxXStages + 2 * kOpStages + 4); }
 };
-constexpr uint32_t kBarBytes = 8 * 13;
+constexpr uint32_t kBarBytes = 8 * (2 * kMaxXStages + 2 * kOpStages + 5);
 
 __device__ __forceinline__ void unpack8(const uint4 &u, float (&v)[8]) {
     v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x);
@@ -167,6 +178,10 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
             mbar_init(bar.full(s), 1);
             mbar_init(bar.empty(s), 8);
         }
+        for (int o = 0; o < p.op_stages; ++o) {
+            mbar_init(bar.ofull(o), 1);
+            mbar_init(bar.oempty(o), 1);
+        }
         for (int a = 0; a < 2; ++a) {
             mbar_init(bar.accf(a), 1);
             mbar_init(bar.acce(a), 8);
@@ -200,21 +215,28 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
                 const int slice = i % p.n_slices, tl_ = i / p.n_slices;
                 const int b = tl_ / p.tiles_per_seq, t0 = (tl_ % p.tiles_per_seq) * kTt;
                 const int s = it % S, n = it / S;
+                const int o = it % p.op_stages, on = it / p.op_stages;
+                if (!mbar_wait<kWaitHint>(bar.oempty(o), (on & 1) ^ 1, abort, 2u, &g_fault, p.wt.wait_ns)) break;
                 if (!mbar_wait<kWaitHint>(bar.empty(s), (n & 1) ^ 1, abort, 2u, &g_fault, p.wt.wait_ns)) break;
                 if (it == 0 && (int)blockIdx.x == p.wt.withhold_cta) continue;   // test hook: no loads
-                mbar_arrive_expect_tx(bar.full(s), p.x_stage_tx + p.z_stage_bytes + p.u_bytes);
-                const uint32_t st = sb + s * p.stage_bytes;
-                tma_load_3d(st + p.off_x, &tm_x, bar.full(s), slice * kDt, t0 - (W - 1), b);
-                tma_load_3d(st + p.off_z, &tm_z, bar.full(s), 0, t0, b);
+                const uint32_t os = sb + p.off_op + o * p.op_bytes;
+                mbar_arrive_expect_tx(bar.ofull(o), p.z_stage_bytes + p.u_bytes);
+                tma_load_3d(os + p.off_z, &tm_z, bar.ofull(o), 0, t0, b);
                 for (int bx = 0; bx < p.u_boxes; ++bx)
-                    tma_load_2d(st + p.off_u + bx * (uint32_t)(p.R * 128), &tm_u, bar.full(s),
+                    tma_load_2d(os + p.off_u + bx * (uint32_t)(p.R * 128), &tm_u, bar.ofull(o),
                                 slice * p.slice_cols + 64 * bx, 0);
+                mbar_arrive_expect_tx(bar.full(s), p.x_stage_tx);
+                tma_load_3d(sb + p.off_x + s * p.x_stage_bytes, &tm_x, bar.full(s), slice * kDt, t0 - (W - 1), b);
             }
             // Let every load this warp issued land before the CTA can exit.
             const int issued = it;
             for (int s = 0; s < S && s < issued; ++s) {
                 const int last = issued - 1 - ((issued - 1 - s) % S);   // last tile using stage s
                 mbar_drain(bar.full(s), (last / S) & 1, p.wt.wait_ns);
+            }
+            for (int o = 0; o < p.op_stages && o < issued; ++o) {
+                const int last = issued - 1 - ((issued - 1 - o) % p.op_stages);
+                mbar_drain(bar.ofull(o), (last / p.op_stages) & 1, p.wt.wait_ns);
             }
         }
         __syncwarp();
@@ -231,14 +253,14 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
         const uint32_t i_last = idesc_bf16(128, p.n_pad - 256 * (nchunks - 1), false, true);
         int it = 0;
         for (int i = blockIdx.x; i < p.n_tiles; i += gridDim.x, ++it) {
-            const int s = it % S, n = it / S;
+            const int o = it % p.op_stages, on = it / p.op_stages;
             const int a = it % p.nbuf, m = it / p.nbuf;
-            if (!warp_wait<kWaitHint>(bar.full(s), n & 1, abort, 8u, &g_fault, p.wt.wait_ns)) break;
+            if (!warp_wait<kWaitHint>(bar.ofull(o), on & 1, abort, 8u, &g_fault, p.wt.wait_ns)) break;
             if (!warp_wait<kWaitHint>(bar.acce(a), (m & 1) ^ 1, abort, 16u, &g_fault, p.wt.wait_ns)) break;
             tc_fence_after();
             const uint32_t d = tmem + a * p.bufcols;
-            const uint32_t za = sb + s * p.stage_bytes + p.off_z;
-            const uint32_t ua = sb + s * p.stage_bytes + p.off_u;
+            const uint32_t za = sb + p.off_op + o * p.op_bytes + p.off_z;
+            const uint32_t ua = sb + p.off_op + o * p.op_bytes + p.off_u;
             for (int nc = 0; nc < nchunks; ++nc) {
                 const uint32_t idesc = nc + 1 < nchunks ? i_full : i_last;
                 uint64_t dz = desc_at(t_z, za), du = desc_at(t_u, ua + nc * 4 * ubox);
@@ -249,7 +271,10 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
                     du += 2048u >> 4;
                 }
             }
-            if (elect_one()) mma_commit(bar.accf(a));
+            if (elect_one()) {
+                mma_commit(bar.accf(a));
+                mma_commit(bar.oempty(o));
+            }
             __syncwarp();
         }
         if (elect_one()) mma_commit(bar.done());
@@ -289,7 +314,7 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
             const int yb = yc & 1;
             if (lane == 0) bulk_wait_read<1>();
             __syncwarp();
-            const uint32_t xs = sb + s * p.stage_bytes + p.off_x;
+            const uint32_t xs = sb + p.off_x + s * p.x_stage_bytes;
             const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16) + a * p.bufcols;
             const uint32_t yw = yrow + yb * ES::YBUF;
             uint32_t wr[2][TP::NCOL];
@@ -431,12 +456,15 @@ bool plan_fwd(int B, int T, int D, int G, int W, int R, FwdParams &p) {
     p.nwg = (ncol <= 32 && DSC_FWD_SETS >= 2) ? 2 : 1;   // epilogue warp sets
     if (p.nbuf < p.nwg) p.nwg = p.nbuf;
     p.y_buf_bytes = (uint32_t)(32 * 32 * 2);
-    p.off_x = 0;
-    p.off_z = p.x_stage_bytes;
-    p.off_u = p.off_z + p.z_stage_bytes;
-    p.stage_bytes = (p.off_u + p.u_bytes + 1023) / 1024 * 1024;
-    for (int st = 4; st >= 2; --st) {
-        const uint32_t off_y = st * p.stage_bytes;
+    p.off_z = 0;
+    p.off_u = p.z_stage_bytes;
+    p.op_bytes = (p.off_u + p.u_bytes + 1023) / 1024 * 1024;
+    p.op_stages = kOpStages;
+    p.off_op = 0;
+    p.off_x = p.op_stages * p.op_bytes;
+    // as deep an x ring as fits next to the operand ring and the y staging
+    for (int st = kMaxXStages; st >= 2; --st) {
+        const uint32_t off_y = p.off_x + st * p.x_stage_bytes;
         const uint32_t off_bar = off_y + 8 * p.nwg * 2 * p.y_buf_bytes;
         const uint32_t total = off_bar + kBarBytes + 16 + 1024;
         if (total <= kSmemLimit) {
