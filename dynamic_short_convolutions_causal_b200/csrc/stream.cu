@@ -81,7 +81,12 @@ constexpr int kBX = 32;            // threads along channels (one warp)
 constexpr int kBY = 8;             // chunks per block in the static backward
 
 __host__ __device__ inline int chunk_for(int T) { return T < kChunk ? T : kChunk; }
-inline int chunk_fwd(int T) { return T < kChunkFwd ? T : kChunkFwd; }
+// tokens per thread in the forward: short walks for few taps (more walks in parallel),
+// long ones for many taps (the W-1 halo rows each walk re-reads)
+inline int chunk_fwd(int T, int W) {
+    const int c = W <= 4 ? kChunkFwd : kChunk;
+    return T < c ? T : c;
+}
 __host__ __device__ inline int dw_partials(int B, int T) { return B * cdiv(cdiv(T, chunk_for(T)), kBY); }
 
 // cp.async of BYTES (4, 8 or 16) from global to shared memory; when `valid` is false the
@@ -472,7 +477,7 @@ void launch_fwd_k(int nitems, const T *x, const T *w, T *y, int B, int T_, int D
 template <typename T, bool STATIC>
 void launch_stream_fwd_T(const void *x, const void *w, void *y, int B, int T_, int D, int G, int W,
                          cudaStream_t s) {
-    const int chunk = chunk_fwd(T_);
+    const int chunk = chunk_fwd(T_, W);
     const T *xp = (const T *)x;
     const T *wp = (const T *)w;
     T *yp = (T *)y;

@@ -34,10 +34,10 @@
 //               TMA store of dx from the stage once the epilogue has written it there
 //   warp 1      recompute: one MMA per tap k with the z tile shifted by k rows,
 //                 Wk[t, g] = sum_r z[t0+t+k, r] Up[r, k*NG+g],
-//               so TMEM lane t holds w[t+k, g, k] for every k; and
-//               dz[m] += dw Up^T  (A = dw tile, B = Up slice; M=128 tokens, N=R)
-//   warp 2      dU^T[s] += dw^T z  (A = dw tile read MN-major, B = z; M=128 columns),
-//               and the gpu-scope publication of each finished dz partial
+//               so TMEM lane t holds w[t+k, g, k] for every k; between tiles, the
+//               gpu-scope publication of each finished dz partial
+//   warp 2      dz[m] += dw Up^T  (A = dw tile, B = Up slice; M=128 tokens, N=R) and
+//               dU^T[s] += dw^T z  (A = dw tile read MN-major, B = z; M=128 columns)
 //   warp 3      reducer: sums the dz partials of its rows of each token tile
 //   warps 4-19  epilogue, one token row per thread, 16 channels per warp:
 //                 A2: dw (bf16) into the shared-memory dw tile;
@@ -70,7 +70,7 @@ constexpr int kCPW = kDt / 4;                   // channels per epilogue warp
 // Warp roles.  Warps 0-3 sit on the SM's four sub-partitions, one each, and the
 // epilogue warps 4-19 four to a sub-partition; 20 warps keep 96 registers a thread.
 constexpr int kRecWarp = 1;
-constexpr int kMmaWarp = 2;                     // dU MMAs, dz partial publication
+constexpr int kMmaWarp = 2;                     // dz and dU MMAs
 constexpr int kRedWarp = 3;
 constexpr int kEpi0 = 4;
 constexpr int kThreads = 32 * (kEpi0 + kEpiWarps);
@@ -79,9 +79,10 @@ constexpr int kMaxStages = 3;
 struct BwdParams {
     int B, T, D, G, W, R;
     int NGs;                  // filter groups per slice (64/G)
-    int NGp;                  // TMEM columns per tap block (NGs rounded up to 16)
-    int SC;                   // filter columns per slice (NGs*W)
-    int SCp;                  // SC rounded up to 128 (dU^T M-blocks)
+    int NGp;                  // columns per tap block in Up, the dw tile and TMEM (Cols::NB)
+    int SC;                   // filter columns of U per slice (NGs*W)
+    int SCq;                  // columns per slice in the tap-major layout (Cols::SCQ)
+    int SCp;                  // SCq rounded up to 128 (dU^T M-blocks)
     int n_slices, tiles_per_seq, n_tt;
     int A, Bg;                // token ranges x slice groups = grid
     int u_boxes;              // TMA boxes of 64 Up columns per slice
@@ -131,6 +132,26 @@ __device__ __forceinline__ void unpack8(const uint4 &u, float (&v)[8]) {
     v[6] = bf16_lo(u.w); v[7] = bf16_hi(u.w);
 }
 
+// Column layout of the tap-major filter blocks (the Up copy of U, the dw tile and the
+// recomputed filters in TMEM).  For G <= 4 a tap block has one column per filter group
+// of the slice (64/G >= 16).  For G >= 8 the block is padded to 16 columns, the MMA's
+// smallest N and a 32-byte descriptor step; and for G >= 32, where a group would span
+// several epilogue warps, each warp's 16 channels form a "virtual group" with a copy of
+// the group's U column: dz = dw Up^T sums the virtual groups by itself, and the dU
+// columns of a group's virtual groups are added when dU is read out.
+template <int W, int G>
+struct Cols {
+    static constexpr int GV = G < 16 ? G : 16;       // channels per (virtual) group
+    static constexpr int NGV = 64 / GV;              // (virtual) groups per slice
+    static constexpr int NB = NGV < 16 ? 16 : NGV;   // columns per tap block
+    static constexpr int SCQ = NB * W;               // columns per slice
+    static constexpr int NMB = (SCQ + 127) / 128;    // dU^T M-blocks per slice
+    static constexpr int VPR = G / GV;               // virtual groups per real group
+};
+
+__device__ __forceinline__ void sts16(uint32_t addr, uint16_t v) {
+    asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory");
+}
 __device__ __forceinline__ void sts32(uint32_t addr, uint32_t v) {
     asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
 }
@@ -198,7 +219,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ CUtensorMap tm_x,
                  const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_u,
                  const __grid_constant__ CUtensorMap tm_dx, const BwdParams p) {
-    constexpr int NG8 = 8 / G;          // filter groups in one 8-channel chunk
+    using CL = Cols<W, G>;
+    constexpr int GV = CL::GV;
+    constexpr int NG8 = GV <= 8 ? 8 / GV : 1;   // (virtual) groups in one 8-channel chunk
     constexpr int CH = kCPW / 8;        // 16-byte chunks of a warp's channels in a row
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -223,7 +246,7 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             mbar_init(bar.zfull(z), 1);
             mbar_init(bar.zempty(z), 2);        // recompute and dz/dU streams
             mbar_init(bar.ufull(z), 1);
-            mbar_init(bar.uempty(z), 1);        // the recompute/dz stream (commit after dz)
+            mbar_init(bar.uempty(z), 2);        // recompute and dz/dU streams
             mbar_init(bar.dzfull(z), 1);
             mbar_init(bar.dzempty(z), kEpiWarps);
         }
@@ -231,18 +254,19 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
         mbar_init(bar.wfull(), 1);
         mbar_init(bar.wempty(), kEpiWarps);
         mbar_init(bar.dwready(), kEpiWarps);
-        mbar_init(bar.dwfree(), 2);             // dz and dU streams
+        mbar_init(bar.dwfree(), 1);
         mbar_init(bar.dufull(), 1);
         mbar_init(bar.done(), 2);               // recompute and dz/dU streams
         mbar_init(bar.xdead(), kEpiWarps);      // every epilogue warp is past A2
         *abort = 0;
         fence_barrier_init();
     }
-    // dw^T rows beyond SC (padding of the last 128-column M-block) must read as zero.
-    if (p.SCp > p.SC) {
+    // Columns of the dw tile that no epilogue warp writes (the padding of the last
+    // 128-column M-block, and the padding of each tap block when G >= 8) must read as zero.
+    if (G >= 8 || p.SCp > p.SCq) {
         for (uint32_t o = threadIdx.x * 16; o < (uint32_t)(p.SCp / 64) * 16384u; o += kThreads * 16) {
             const uint32_t atom = o / 16384u;
-            if ((int)(atom * 64) + 64 > p.SC) sts128(sb + p.off_dw + o, make_uint4(0, 0, 0, 0));
+            if (G >= 8 || (int)(atom * 64) + 64 > p.SCq) sts128(sb + p.off_dw + o, make_uint4(0, 0, 0, 0));
         }
         fence_proxy_async_smem();
     }
@@ -261,7 +285,6 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    const int nmb = p.SCp / 128;        // dU^T M-blocks per slice
 
     if (warp == 0) {
         // ---------------------------------------------------------- TMA producer
@@ -272,7 +295,7 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
                 mbar_arrive_expect_tx(bar.ufull(ub), p.u_bytes);
                 const uint32_t ud = sb + p.off_u + ub * p.u_bytes;
                 for (int bx = 0; bx < p.u_boxes; ++bx)
-                    tma_load_2d(ud + bx * (uint32_t)(p.R * 128), &tm_u, bar.ufull(ub), slice * p.SC + 64 * bx, 0);
+                    tma_load_2d(ud + bx * (uint32_t)(p.R * 128), &tm_u, bar.ufull(ub), slice * p.SCq + 64 * bx, 0);
             };
             auto store_dx = [&](int i) {      // dx of tile i, from its stage's x region
                 const int m = sp.m0 + i / S, slice = sp.s0 + i % S;
@@ -339,41 +362,51 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
         }
         __syncwarp();
     } else if (warp == kRecWarp) {
-        // ---------------------------------------------------------- MMA issuer: recompute, dz
+        // ---------------------------------------------------------- MMA issuer: recompute
         // Each MMA warp runs its schedule warp-uniformly; one elected lane issues each
         // tcgen05 instruction, and descriptors advance by adding to their start field.
-        // Order: recompute(0); then per tile i: dz(i) once its dw is written, and
-        // recompute(i+1) once the epilogue has read the filters of tile i.
-        //   recompute: Wk[t, g] = sum_r z[t0+t+k, r] Up[r, k*NG+g], one MMA chain per tap
-        //     with the z tile shifted by k rows (A: z, K-major; B: Up, MN-major);
-        //   dz[m] (+)= dw Up^T: A = dw tile (K-major view), B = Up slice (K-major), 16
-        //     columns per step; accumulates over the token tile's slices.
-        constexpr int SC = (kDt / G) * W;
-        constexpr int KSC = SC / 16;
-        const uint64_t t_zk = desc_tmpl(p.z_slab, 128, kSwNone);
-        const uint64_t t_u_mn = desc_tmpl((uint32_t)(p.R * 128), 1024, kSw128);
-        const uint64_t t_k128 = desc_tmpl(16, 1024, kSw128);
+        // Tile i's filters are recomputed once the epilogue has read those of tile i-1:
+        //   Wk[t, g] = sum_r z[t0+t+k, r] Up[r, k*NB+g], one MMA chain per tap with the z
+        //   tile shifted by k rows (A: z, K-major; B: Up, MN-major).
+        // Between tiles the warp, otherwise idle, publishes each finished dz partial: the
+        // epilogue arrives on dzdone[mz % 4] once token tile mz's partial is stored, and a
+        // gpu-scope fence, then one add of 16 to the tile's counter, make it visible to the
+        // other CTAs.  The epilogue never waits for that fence.
+        const uint64_t t_zk = desc_tmpl(p.z_slab, 128, kSwNone);               // z, K-major, no swizzle
+        const uint64_t t_u_mn = desc_tmpl((uint32_t)(p.R * 128), 1024, kSw128);  // Up as MN-major B
         const uint32_t i_rec = idesc_bf16(128, p.NGp, false, true);
-        const uint32_t i_dz = idesc_bf16(128, p.R, false, false);
         const int ksr = p.R / 16;
         const uint32_t ubox = (uint32_t)(p.R * 128);
-        const uint64_t st_zk = (2 * p.z_slab) >> 4;       // 16 more z columns (start field units)
-        const uint64_t st_wrap_a = (16384u - 96u) >> 4;   // next 64-column dw atom
-        const uint64_t st_wrap_b = (ubox - 96u) >> 4;     // next 64-column Up box
-        const uint32_t dw0 = sb + p.off_dw;
-        auto recompute = [&](int i) -> bool {
+        const uint64_t st_zk = (2 * p.z_slab) >> 4;   // 16 more z columns (start field units)
+        int published = 0;                            // token tiles published so far
+        auto dz_publish = [&](int upto, bool block) -> bool {   // publish [published, upto)
+            for (; published < upto; ++published) {
+                const int mz = published;
+                if (!block && !__all_sync(0xffffffffu, mbar_try_wait(bar.dzdone(mz & 3), (mz >> 2) & 1)))
+                    return true;   // not stored yet: try again after the next tile
+                if (!warp_wait(bar.dzdone(mz & 3), (mz >> 2) & 1, abort, 2048u, &g_fault_bwd, p.wt.wait_ns))
+                    return false;
+                fence_gpu();
+                __syncwarp();
+                if (lane == 0) red_release_add(p.flag_dz + sp.m0 + mz, (unsigned)kEpiWarps);
+                __syncwarp();
+            }
+            return true;
+        };
+        bool ok = true;
+        for (int i = 0; i < nt; ++i) {
             const int j = i % S, mz = i / S, zb = mz & 1;
             const int ub = u_res ? j : (i & 1);
             const int upar = u_res ? 0 : ((i >> 1) & 1);
-            if (j == 0 && !warp_wait(bar.zfull(zb), (mz >> 1) & 1, abort, 4u, &g_fault_bwd, p.wt.wait_ns)) return false;
-            if (!warp_wait(bar.ufull(ub), upar, abort, 4u, &g_fault_bwd, p.wt.wait_ns)) return false;
-            if (!warp_wait(bar.wempty(), (i & 1) ^ 1, abort, 16u, &g_fault_bwd, p.wt.wait_ns)) return false;
+            if (j == 0 && !warp_wait(bar.zfull(zb), (mz >> 1) & 1, abort, 4u, &g_fault_bwd, p.wt.wait_ns)) break;
+            if (!warp_wait(bar.ufull(ub), upar, abort, 4u, &g_fault_bwd, p.wt.wait_ns)) break;
+            if (!warp_wait(bar.wempty(), (i & 1) ^ 1, abort, 16u, &g_fault_bwd, p.wt.wait_ns)) break;
             tc_fence_after();
             const uint32_t zs = sb + p.off_z + zb * p.z_bytes;
             const uint32_t us = sb + p.off_u + ub * p.u_bytes;
 #pragma unroll
             for (int k = 0; k < W; ++k) {
-                const int col0 = k * (kDt / G);
+                const int col0 = k * CL::NB;
                 uint64_t da = desc_at(t_zk, zs + 16 * k);
                 uint64_t db = desc_at(t_u_mn, us + (col0 / 64) * ubox + (col0 % 64) * 2);
                 const uint32_t d = tmem + p.tm_w + k * p.NGp;
@@ -387,44 +420,16 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             if (elect_one()) {
                 mma_commit(bar.wfull());
                 if (j == S - 1) mma_commit(bar.zempty(zb));
+                if (!u_res) mma_commit(bar.uempty(ub));
             }
             __syncwarp();
-            return true;
-        };
-        auto dz_mma = [&](int i) -> bool {
-            const int j = i % S, mz = i / S, db = mz & 1;
-            const int ub = u_res ? j : (i & 1);
-            if (!warp_wait(bar.dwready(), i & 1, abort, 8u, &g_fault_bwd, p.wt.wait_ns)) return false;
-            if (j == 0 && !warp_wait(bar.dzempty(db), ((mz >> 1) & 1) ^ 1, abort, 8u, &g_fault_bwd, p.wt.wait_ns))
-                return false;
-            tc_fence_after();
-            const uint32_t us = sb + p.off_u + ub * p.u_bytes;
-            uint64_t da = desc_at(t_k128, dw0), dbd = desc_at(t_k128, us);
-            const uint32_t d = tmem + p.tm_dz + db * p.R;
-#pragma unroll
-            for (int kk = 0; kk < KSC; ++kk) {
-                if (elect_one()) mma_bf16_ss(d, da, dbd, i_dz, (j > 0 || kk > 0) ? 1u : 0u);
-                __syncwarp();
-                const bool wrap = (kk & 3) == 3;
-                da += wrap ? st_wrap_a : 2u;
-                dbd += wrap ? st_wrap_b : 2u;
-            }
-            if (elect_one()) {
-                mma_commit(bar.dwfree());
-                if (!u_res) mma_commit(bar.uempty(ub));   // recompute(i) and dz(i) read Up
-                if (j == S - 1) mma_commit(bar.dzfull(db));
-            }
-            __syncwarp();
-            return true;
-        };
-        if (nt > 0 && recompute(0)) {
-            for (int i = 0; i < nt; ++i) {
-                if (!dz_mma(i)) break;
-                if (i + 1 < nt && !recompute(i + 1)) break;
-            }
+            // partials of the token tiles before this one are stored by now or soon;
+            // publish those that are (without waiting), the rest at a later tile
+            if (!(ok = dz_publish(mz, false))) break;
         }
         if (elect_one()) mma_commit(bar.done());
         __syncwarp();
+        if (ok) dz_publish(nt / S, true);   // the remaining token tiles, the last one included
     } else if (warp >= kEpi0) {
         // ---------------------------------------------------------- epilogue
         const int ew = warp - kEpi0;
@@ -503,7 +508,7 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
                         pk[k][1] = bf16x2_mul(d0.y, xu[k].y);
                         pk[k][2] = bf16x2_mul(d0.z, xu[k].z);
                         pk[k][3] = bf16x2_mul(d0.w, xu[k].w);
-                    } else {
+                    } else if constexpr (G <= 4) {
                         float dv[8], xv[8], dw[NG8];
                         unpack8(d0, dv);
                         unpack8(xu[k], xv);
@@ -535,7 +540,38 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
                     }
                 }
             };
-            if constexpr (kPre) {
+            if constexpr (G >= 8) {
+                // one value per (virtual group, tap): GV = 8 gives one per chunk, and the
+                // two chunks' groups are adjacent columns; GV = 16 gives one per warp
+                float sv[CH][W];
+#pragma unroll
+                for (int cq = 0; cq < CH; ++cq) {
+                    float dv[8];
+                    unpack8(lds128(dys + (dyr[0] ^ ((uint32_t)cq << 4))), dv);
+#pragma unroll
+                    for (int k = 0; k < W; ++k) {
+                        float xv[8];
+                        unpack8(lds128(xs + (xr[k] ^ ((uint32_t)cq << 4))), xv);
+                        float acc = 0.f;
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) acc = fmaf(dv[e], xv[e], acc);
+                        sv[cq][k] = acc;
+                    }
+                }
+                if (!warp_wait(bar.dwfree(), (i & 1) ^ 1, abort, 32u, &g_fault_bwd, p.wt.wait_ns)) { ok = false; break; }
+#pragma unroll
+                for (int k = 0; k < W; ++k) {
+                    const int jp = k * CL::NB + (GV == 8 ? 2 * h : h);
+                    const uint32_t atom = (uint32_t)(jp >> 6), within = (uint32_t)(jp & 63);
+                    const uint32_t a = dwrow + atom * 16384u + ((((within >> 3) << 4) ^ dwsw) | ((within & 7) * 2));
+                    if constexpr (GV == 8) {
+                        sts32(a, pack_bf16x2(sv[0][k], sv[1][k]));
+                    } else {
+                        const uint32_t pr = pack_bf16x2(sv[0][k] + sv[1][k], 0.f);
+                        sts16(a, (uint16_t)(pr & 0xffffu));
+                    }
+                }
+            } else if constexpr (kPre) {
                 uint32_t pk[CH][W][NPK];
 #pragma unroll
                 for (int cq = 0; cq < CH; ++cq) a2_compute(cq, pk[cq]);
@@ -558,7 +594,7 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             // ---- A1: dx[t,c] = dy[t,c] + sum_k w[t+k,g,k] dy[t+k,c]
             if (!warp_wait(bar.wfull(), i & 1, abort, 128u, &g_fault_bwd, p.wt.wait_ns)) { ok = false; break; }
             tc_fence_after();
-            constexpr int NGB = 8 / G;                      // filter groups of one chunk
+            constexpr int NGB = NG8;                        // (virtual) groups of one chunk
             constexpr int KB = (W * (4 + NGB) <= 48) ? W : 4;   // taps per batch
             uint4 dxo[CH];
 #pragma unroll
@@ -575,7 +611,7 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
 #pragma unroll
                     for (int kb = 0; kb < KB; ++kb)
                         if (k0 + kb < W)
-                            tmem_ld<NGB>(tl + p.tm_w + (k0 + kb) * p.NGp + (kCPW * h + 8 * cq) / G, wr[kb]);
+                            tmem_ld<NGB>(tl + p.tm_w + (k0 + kb) * p.NGp + (kCPW * h + 8 * cq) / GV, wr[kb]);
                     tmem_wait_ld();
 #pragma unroll
                     for (int kb = 0; kb < KB; ++kb)
@@ -599,7 +635,7 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
                             unpack8(du[kb], dk);
 #pragma unroll
                             for (int e = 0; e < 8; ++e)
-                                dx[e] = fmaf(__uint_as_float(wr[kb][e / G]), dk[e], k == 0 ? dk[e] : dx[e]);
+                                dx[e] = fmaf(__uint_as_float(wr[kb][e / GV]), dk[e], k == 0 ? dk[e] : dx[e]);
                         }
                     }
                 }
@@ -636,19 +672,33 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             const int N = p.n_slices * p.SC;
             for (int j = 0; j < S; ++j) {
                 const int slice = sp.s0 + j;
-                if (h < nmb) {
-                    // lane j' of dU^T M-block h -> natural column g*W + k
+                if (h < CL::NMB) {
+                    // lane j' of dU^T M-block h is tap-major column k*NB + gv; the real
+                    // column of U is g*W + k with g the (virtual) group's real group
                     const int jp = 128 * h + row;
-                    const int jn = (jp % p.NGs) * W + jp / p.NGs;
+                    const int k = jp / CL::NB, gv = jp % CL::NB;
+                    const bool valid = k < W && gv < CL::NGV && gv % CL::VPR == 0;
+                    const int jn = (gv * GV / G) * W + k;
                     float *dst = p.du_part + (size_t)sp.a * p.R * N + (size_t)slice * p.SC + jn;
 #pragma unroll 1
                     for (int c0 = 0; c0 < p.R; c0 += 16) {
                         uint32_t v[16];
-                        tmem_ld<16>(tl + p.tm_du + (j * nmb + h) * p.R + c0, v);   // warp-collective
+                        tmem_ld<16>(tl + p.tm_du + (j * CL::NMB + h) * p.R + c0, v);   // warp-collective
                         tmem_wait_ld_regs(v);
-                        if (jp < p.SC) {
+                        float f[16];
 #pragma unroll
-                            for (int m2 = 0; m2 < 16; ++m2) dst[(size_t)(c0 + m2) * N] = __uint_as_float(v[m2]);
+                        for (int m2 = 0; m2 < 16; ++m2) f[m2] = __uint_as_float(v[m2]);
+                        if constexpr (CL::VPR >= 2) {
+#pragma unroll
+                            for (int m2 = 0; m2 < 16; ++m2) f[m2] += __shfl_xor_sync(0xffffffffu, f[m2], 1);
+                        }
+                        if constexpr (CL::VPR >= 4) {
+#pragma unroll
+                            for (int m2 = 0; m2 < 16; ++m2) f[m2] += __shfl_xor_sync(0xffffffffu, f[m2], 2);
+                        }
+                        if (valid) {
+#pragma unroll
+                            for (int m2 = 0; m2 < 16; ++m2) dst[(size_t)(c0 + m2) * N] = f[m2];
                         }
                     }
                 }
@@ -658,86 +708,93 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             __syncwarp();
             if (lane == 0) red_release_add(p.flag_du + sp.b, 1u);
             if (wait_count(p.flag_du + sp.b, (unsigned)(kEpiWarps * p.A), abort, 1024u, p.wt.wait_ns)) {
-                // this CTA's share (of A) of the group's R x (S*SC) block, float4-wise
+                // this CTA's share (of A) of the group's R x (S*SC) block
                 const int cols = S * p.SC;
-                const long long n4 = (long long)p.R * cols / 4;
-                const long long e0 = n4 * sp.a / p.A, e1 = n4 * (sp.a + 1) / p.A;
+                const long long n = (long long)p.R * cols;
+                const long long e0 = n * sp.a / p.A, e1 = n * (sp.a + 1) / p.A;
                 const int et = threadIdx.x - 32 * kEpi0;
                 for (long long e = e0 + et; e < e1; e += 32 * kEpiWarps) {
-                    const int r = (int)(4 * e / cols), c = (int)(4 * e - (long long)r * cols);
+                    const int r = (int)(e / cols), c = (int)(e - (long long)r * cols);
                     const size_t off = (size_t)r * N + (size_t)sp.s0 * p.SC + c;
-                    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                    for (int a = 0; a < p.A; ++a) {
-                        const float4 v = __ldcg(reinterpret_cast<const float4 *>(p.du_part + (size_t)a * p.R * N + off));
-                        acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-                    }
-                    *reinterpret_cast<float4 *>(p.dU + off) = acc;
+                    float acc = 0.f;
+                    for (int a = 0; a < p.A; ++a) acc += __ldcg(p.du_part + (size_t)a * p.R * N + off);
+                    p.dU[off] = acc;
                 }
             }
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
-        // ---------------------------------------------------------- MMA issuer: dU
-        // dU^T[slice] (+)= dw^T z once tile i's dw is written: A = dw^T (MN-major), B = z
-        // tile rows 0..127 (MN-major), 16 tokens per step; accumulates over the CTA's
-        // token tiles.  After issuing a tile, the warp also publishes a finished dz
-        // partial (see dz_publish): its wait there is already satisfied, and the fence it
-        // takes overlaps the next tile's epilogue work instead of holding up the epilogue.
-        constexpr int SC = (kDt / G) * W;
-        constexpr int NMB = (SC + 127) / 128;
+        // ---------------------------------------------------------- MMA issuer: dz and dU
+        // Once tile i's dw is written:
+        //   dz[m] (+)= dw Up^T: A = dw tile (K-major view), B = Up slice (K-major), 16
+        //     columns per step (+32 bytes within a 64-column atom, the next atom every 4
+        //     steps); accumulates over the token tile's slices;
+        //   dU^T[slice] (+)= dw^T z: A = dw^T (MN-major), B = z tile rows 0..127
+        //     (MN-major), 16 tokens per step; accumulates over the CTA's token tiles.
+        // The step counts are compile-time, so the issue loops unroll fully.
+        constexpr int KSC = CL::SCQ / 16;
+        constexpr int NMB = CL::NMB;
+        const uint64_t t_k128 = desc_tmpl(16, 1024, kSw128);
         const uint64_t t_dwt = desc_tmpl(16384, 1024, kSw128);
         const uint64_t t_zmn = desc_tmpl(128, p.z_slab, kSwNone);
+        const uint32_t i_dz = idesc_bf16(128, p.R, false, false);
         const uint32_t i_du = idesc_bf16(128, p.R, true, true);
+        const uint32_t ubox = (uint32_t)(p.R * 128);
+        const uint64_t st_wrap_a = (16384u - 96u) >> 4;   // next 64-column dw atom
+        const uint64_t st_wrap_b = (ubox - 96u) >> 4;     // next 64-column Up box
         const uint32_t dw0 = sb + p.off_dw;
-        int published = 0;                 // token tiles whose dz partial has been published
-        // The epilogue arrives on dzdone[mz % 4] once token tile mz's partial is stored; a
-        // gpu-scope fence, then one add of 16 to the tile's counter, make it visible.
-        auto dz_publish = [&](int upto) -> bool {   // publish token tiles [published, upto)
-            for (; published < upto; ++published) {
-                const int mz = published;
-                if (!warp_wait(bar.dzdone(mz & 3), (mz >> 2) & 1, abort, 2048u, &g_fault_bwd, p.wt.wait_ns))
-                    return false;
-                fence_gpu();
-                __syncwarp();
-                if (lane == 0) red_release_add(p.flag_dz + sp.m0 + mz, (unsigned)kEpiWarps);
-                __syncwarp();
-            }
-            return true;
-        };
-        bool ok = true;
-        for (int i = 0; i < nt && ok; ++i) {
-            const int j = i % S, mz = i / S, zb = mz & 1;
+        for (int i = 0; i < nt; ++i) {
+            const int j = i % S, mz = i / S, db = mz & 1, zb = mz & 1;
+            const int ub = u_res ? j : (i & 1);
+            const int upar = u_res ? 0 : ((i >> 1) & 1);
+            if (!warp_wait(bar.ufull(ub), upar, abort, 4u, &g_fault_bwd, p.wt.wait_ns)) break;
             if (j == 0 && !warp_wait(bar.zfull(zb), (mz >> 1) & 1, abort, 4u, &g_fault_bwd, p.wt.wait_ns)) break;
             if (!warp_wait(bar.dwready(), i & 1, abort, 8u, &g_fault_bwd, p.wt.wait_ns)) break;
+            if (j == 0 && !warp_wait(bar.dzempty(db), ((mz >> 1) & 1) ^ 1, abort, 8u, &g_fault_bwd, p.wt.wait_ns)) break;
             tc_fence_after();
-            const uint32_t zs = sb + p.off_z + zb * p.z_bytes;
+            {
+                const uint32_t us = sb + p.off_u + ub * p.u_bytes;
+                uint64_t da = desc_at(t_k128, dw0), dbd = desc_at(t_k128, us);
+                const uint32_t d = tmem + p.tm_dz + db * p.R;
 #pragma unroll
-            for (int mb = 0; mb < NMB; ++mb) {
-                const uint32_t d = tmem + p.tm_du + (j * NMB + mb) * p.R;
-                uint64_t da = desc_at(t_dwt, dw0 + mb * 32768u), dbd = desc_at(t_zmn, zs);
-#pragma unroll
-                for (int kk = 0; kk < kTt / 16; ++kk) {
-                    if (elect_one()) mma_bf16_ss(d, da, dbd, i_du, (mz == 0 && kk == 0) ? 0u : 1u);
+                for (int kk = 0; kk < KSC; ++kk) {
+                    if (elect_one()) mma_bf16_ss(d, da, dbd, i_dz, (j > 0 || kk > 0) ? 1u : 0u);
                     __syncwarp();
-                    da += 2048u >> 4;
-                    dbd += 256u >> 4;
+                    const bool wrap = (kk & 3) == 3;
+                    da += wrap ? st_wrap_a : 2u;
+                    dbd += wrap ? st_wrap_b : 2u;
+                }
+            }
+            {
+                const uint32_t zs = sb + p.off_z + zb * p.z_bytes;
+#pragma unroll
+                for (int mb = 0; mb < NMB; ++mb) {
+                    const uint32_t d = tmem + p.tm_du + (j * NMB + mb) * p.R;
+                    uint64_t da = desc_at(t_dwt, dw0 + mb * 32768u), dbd = desc_at(t_zmn, zs);
+#pragma unroll
+                    for (int kk = 0; kk < kTt / 16; ++kk) {
+                        if (elect_one()) mma_bf16_ss(d, da, dbd, i_du, (mz == 0 && kk == 0) ? 0u : 1u);
+                        __syncwarp();
+                        da += 2048u >> 4;
+                        dbd += 256u >> 4;
+                    }
                 }
             }
             if (elect_one()) {
                 mma_commit(bar.dwfree());
-                if (j == S - 1) mma_commit(bar.zempty(zb));
+                if (!u_res) mma_commit(bar.uempty(ub));
+                if (j == S - 1) {
+                    mma_commit(bar.dzfull(db));
+                    mma_commit(bar.zempty(zb));
+                }
             }
             __syncwarp();
-            // tile i-1 being the first of a token tile mz' means the partial of mz'-1 was
-            // stored (in that tile's epilogue, before the dw of tile i)
-            if (i >= 1 && (i - 1) % S == 0) ok = dz_publish((i - 1) / S);
         }
         if (elect_one()) {
             mma_commit(bar.dufull());
             mma_commit(bar.done());
         }
         __syncwarp();
-        if (ok) dz_publish(nt / S);        // the last token tiles
     } else if (warp == kRedWarp) {
         // ---------------------------------------------------------- dz reducer
         // Once all Bg slice groups have written their partial of token tile m, sum this
@@ -786,24 +843,34 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
     }
 }
 
-// Up[r, s*SC + k*NG + g] = U[r, s*SC + g*W + k]  (tap-major columns within each slice).
-// Grid (ceil(N/2048), R): one row r per grid row; each thread writes 8 consecutive output
-// columns with one 16-byte store (NG is a multiple of 8, so the 8 share one tap k and read
-// source columns W apart).  Block (0, 0) also clears the main kernel's counters.
-__global__ void k_permute_u(const bf16 *__restrict__ U, bf16 *__restrict__ Up, int R, int N, int SC, int NG,
-                            int W, unsigned *__restrict__ flags, int nflags) {
+// Up[r, s*SCq + k*NB + gv] = U[r, (real group of virtual group gv of slice s)*W + k], and
+// 0 for padding columns gv >= NGV (see Cols).  For G <= 4 that is the tap-major
+// reordering Up[r, s*SC + k*NG + g] = U[r, s*SC + g*W + k].
+// Grid (ceil(N'/2048), R): one row r per grid row; each thread writes 8 consecutive output
+// columns (one tap, 8 consecutive (virtual) groups) with one 16-byte store.  Block (0, 0)
+// also clears the main kernel's counters.
+__global__ void k_permute_u(const bf16 *__restrict__ U, bf16 *__restrict__ Up, int R, int N, int Nq, int SCq,
+                            int NB, int NGV, int GV, int G, int W, unsigned *__restrict__ flags, int nflags) {
     if (blockIdx.x == 0 && blockIdx.y == 0)
         for (int f = threadIdx.x; f < nflags; f += blockDim.x) flags[f] = 0u;
     const int r = blockIdx.y;
     const int j = 8 * (blockIdx.x * blockDim.x + threadIdx.x);
-    if (r >= R || j >= N) return;
-    const int s = j / SC, jl = j - s * SC;
-    const int k = jl / NG, g = jl - k * NG;
-    const unsigned short *src = reinterpret_cast<const unsigned short *>(U) + (size_t)r * N + s * SC + g * W + k;
+    if (r >= R || j >= Nq) return;
+    const int s = j / SCq, jl = j - s * SCq;
+    const int k = jl / NB, gv0 = jl - k * NB;
+    const unsigned short *src = reinterpret_cast<const unsigned short *>(U) + (size_t)r * N;
     uint32_t v[4];
 #pragma unroll
-    for (int m = 0; m < 4; ++m) v[m] = (uint32_t)src[(2 * m) * W] | ((uint32_t)src[(2 * m + 1) * W] << 16);
-    *reinterpret_cast<uint4 *>(Up + (size_t)r * N + j) = make_uint4(v[0], v[1], v[2], v[3]);
+    for (int m = 0; m < 4; ++m) {
+        uint32_t h2[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+            const int gv = gv0 + 2 * m + e;
+            h2[e] = gv < NGV ? (uint32_t)src[(size_t)((s * 64 + gv * GV) / G) * W + k] : 0u;
+        }
+        v[m] = h2[0] | (h2[1] << 16);
+    }
+    *reinterpret_cast<uint4 *>(Up + (size_t)r * Nq + j) = make_uint4(v[0], v[1], v[2], v[3]);
 }
 
 // ------------------------------------------------------------------ host side
@@ -871,20 +938,23 @@ bool layout_smem(BwdParams &p, int stages, int nU) {
 // layouts, and the A x Bg grid.  false: the tensor-core backward does not take them.
 bool plan_bwd(int B, int T, int D, int G, int W, int R, int nsm, BwdParams &p) {
     if (!(R == 16 || R == 32 || R == 64)) return false;
-    if (D % kDt || !(G == 1 || G == 2 || G == 4) || W < 1 || W > 8) return false;
+    if (D % kDt || !(G == 1 || G == 2 || G == 4 || G == 8 || G == 16 || G == 32 || G == 64) || W < 1 || W > 8)
+        return false;
     p = BwdParams{};
     p.B = B; p.T = T; p.D = D; p.G = G; p.W = W; p.R = R;
     p.NGs = kDt / G;
-    p.NGp = p.NGs < 16 ? 16 : p.NGs;
+    const int gv = G < 16 ? G : 16;                   // mirrors Cols<W, G>
+    p.NGp = (kDt / gv) < 16 ? 16 : kDt / gv;
     p.SC = p.NGs * W;
-    if (p.SC % 16) return false;
-    p.SCp = (p.SC + 127) / 128 * 128;
+    p.SCq = p.NGp * W;
+    if (p.SCq % 16) return false;
+    p.SCp = (p.SCq + 127) / 128 * 128;
     p.n_slices = D / kDt;
     p.tiles_per_seq = (T + kTt - 1) / kTt;
     const long long ntt = (long long)B * p.tiles_per_seq;
     if (ntt >= (1ll << 30) || (long long)p.n_slices * ntt >= (1ll << 31)) return false;
     p.n_tt = (int)ntt;
-    p.u_boxes = (p.SC + 63) / 64;
+    p.u_boxes = (p.SCq + 63) / 64;
     // TMEM: w (W tap blocks) | dz (two buffers) | dU^T (one slot per slice of the CTA)
     p.tm_w = 0;
     p.tm_dz = (uint32_t)(W * p.NGp + 31) / 32 * 32;
@@ -954,7 +1024,11 @@ cudaError_t launch_w(int G, const CUtensorMap *m, const BwdParams &p, cudaStream
     switch (G) {
         case 1: return launch_t<W, 1>(m, p, s);
         case 2: return launch_t<W, 2>(m, p, s);
-        default: return launch_t<W, 4>(m, p, s);
+        case 4: return launch_t<W, 4>(m, p, s);
+        case 8: return launch_t<W, 8>(m, p, s);
+        case 16: return launch_t<W, 16>(m, p, s);
+        case 32: return launch_t<W, 32>(m, p, s);
+        default: return launch_t<W, 64>(m, p, s);
     }
 }
 
@@ -965,8 +1039,9 @@ struct WsLayout {
 WsLayout ws_layout(const BwdParams &p) {
     WsLayout l;
     const size_t N = (size_t)p.n_slices * p.SC;
+    const size_t Nq = (size_t)p.n_slices * p.SCq;
     l.up = 0;
-    l.dz = a256(l.up + (size_t)p.R * N * 2);
+    l.dz = a256(l.up + (size_t)p.R * Nq * 2);
     l.du = a256(l.dz + (size_t)p.Bg * p.B * p.T * p.R * 4);
     l.flags = a256(l.du + (size_t)p.A * p.R * N * 4);
     l.total = a256(l.flags + (size_t)(p.n_tt + p.Bg) * 4);
@@ -1004,15 +1079,17 @@ cudaError_t launch_tc_lowrank_bwd(const void *x, const void *z, const void *U, c
     p.dz = dz;
     p.dU = dU;
     const int N = p.n_slices * p.SC;
-    k_permute_u<<<dim3((N / 8 + 255) / 256, R), 256, 0, s>>>((const bf16 *)U, Up, R, N, p.SC, p.NGs, W,
-                                                              p.flag_dz, p.n_tt + p.Bg);
+    const int Nq = p.n_slices * p.SCq;
+    const int gv = G < 16 ? G : 16;
+    k_permute_u<<<dim3((Nq / 8 + 255) / 256, R), 256, 0, s>>>((const bf16 *)U, Up, R, N, Nq, p.SCq, p.NGp,
+                                                               kDt / gv, gv, G, W, p.flag_dz, p.n_tt + p.Bg);
 
     CUtensorMap m[5];
     const uint64_t dxyz[3] = {(uint64_t)D, (uint64_t)T, (uint64_t)B};
     const uint32_t bxy[3] = {(uint32_t)kDt, p.rows, 1};
     const uint64_t dzz[3] = {(uint64_t)R, (uint64_t)T, (uint64_t)B};
     const uint32_t bz[3] = {8, p.rows, 1};
-    const uint64_t du[2] = {(uint64_t)N, (uint64_t)R};
+    const uint64_t du[2] = {(uint64_t)Nq, (uint64_t)R};
     const uint32_t bu[2] = {64, (uint32_t)R};
     const uint32_t bdx[3] = {(uint32_t)kDt, (uint32_t)kTt, 1};
     if (!make_map(&m[0], dy, 3, dxyz, bxy, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) ||

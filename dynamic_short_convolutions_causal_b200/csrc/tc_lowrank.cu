@@ -13,11 +13,12 @@
 // the z tile and the U slice arrive by TMA; y leaves through shared memory by TMA.
 //
 // Warp roles (persistent CTAs, one per SM, tiles in token-major round-robin order):
-//   warp 0  TMA producer: the MMA operands of a tile (z tile, U slice) into a 2-deep
-//           operand ring that the MMA releases as soon as its MMAs complete, and the x
-//           tile into a deeper x ring that the epilogue releases.  Splitting the two keeps
-//           the x loads several tiles ahead of the epilogue, which both epilogue sets
-//           need: each holds one x stage while it works.
+//   warp 0  TMA producer of the x tiles, into an x ring that the epilogue releases
+//   warp 18 (after the epilogue warps) TMA producer of the MMA operands of a tile (z tile,
+//           U slice), into a 2-deep operand ring that the MMA releases as soon as its
+//           MMAs complete.  The two producers are independent, so the x loads run several
+//           tiles ahead of the epilogue, which both epilogue sets need (each holds one x
+//           stage while it works), whatever the operand ring does.
 //   warp 1  TMEM allocator and MMA issuer (one elected lane), double-buffered accumulator
 //   warps 2-17  two epilogue sets of 8 warps taking alternating tiles: warp w reads TMEM
 //              lanes 32*(w%4).. (its 32 tokens) and handles 32 channels (half the slice);
@@ -121,7 +122,8 @@ template <int W, int GC>
 struct EpiShape {
     static constexpr int SETS = (Taps<W, GC>::NCOL <= 32 && DSC_FWD_SETS >= 2) ? 2 : 1;
     static constexpr int WARPS = 8 * SETS;
-    static constexpr int THREADS = 32 * (2 + WARPS);
+    static constexpr int OPWARP = 2 + WARPS;       // the operand (z, U) producer
+    static constexpr int THREADS = 32 * (3 + WARPS);
     static constexpr int CPW = 32;                 // channels per epilogue warp
     static constexpr int CHUNKS = CPW / 8;
     static constexpr int YBUF = 32 * CPW * 2;      // one warp's y staging: 32 rows x 32 bf16
@@ -215,16 +217,8 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
                 const int slice = i % p.n_slices, tl_ = i / p.n_slices;
                 const int b = tl_ / p.tiles_per_seq, t0 = (tl_ % p.tiles_per_seq) * kTt;
                 const int s = it % S, n = it / S;
-                const int o = it % p.op_stages, on = it / p.op_stages;
-                if (!mbar_wait<kWaitHint>(bar.oempty(o), (on & 1) ^ 1, abort, 2u, &g_fault, p.wt.wait_ns)) break;
                 if (!mbar_wait<kWaitHint>(bar.empty(s), (n & 1) ^ 1, abort, 2u, &g_fault, p.wt.wait_ns)) break;
                 if (it == 0 && (int)blockIdx.x == p.wt.withhold_cta) continue;   // test hook: no loads
-                const uint32_t os = sb + p.off_op + o * p.op_bytes;
-                mbar_arrive_expect_tx(bar.ofull(o), p.z_stage_bytes + p.u_bytes);
-                tma_load_3d(os + p.off_z, &tm_z, bar.ofull(o), 0, t0, b);
-                for (int bx = 0; bx < p.u_boxes; ++bx)
-                    tma_load_2d(os + p.off_u + bx * (uint32_t)(p.R * 128), &tm_u, bar.ofull(o),
-                                slice * p.slice_cols + 64 * bx, 0);
                 mbar_arrive_expect_tx(bar.full(s), p.x_stage_tx);
                 tma_load_3d(sb + p.off_x + s * p.x_stage_bytes, &tm_x, bar.full(s), slice * kDt, t0 - (W - 1), b);
             }
@@ -233,10 +227,6 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
             for (int s = 0; s < S && s < issued; ++s) {
                 const int last = issued - 1 - ((issued - 1 - s) % S);   // last tile using stage s
                 mbar_drain(bar.full(s), (last / S) & 1, p.wt.wait_ns);
-            }
-            for (int o = 0; o < p.op_stages && o < issued; ++o) {
-                const int last = issued - 1 - ((issued - 1 - o) % p.op_stages);
-                mbar_drain(bar.ofull(o), (last / p.op_stages) & 1, p.wt.wait_ns);
             }
         }
         __syncwarp();
@@ -278,6 +268,30 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
             __syncwarp();
         }
         if (elect_one()) mma_commit(bar.done());
+        __syncwarp();
+    } else if (warp == ES::OPWARP) {
+        // ---------------------------------------------------------- TMA producer: operands
+        if (lane == 0) {
+            int it = 0;
+            for (int i = blockIdx.x; i < p.n_tiles; i += gridDim.x, ++it) {
+                const int slice = i % p.n_slices, tl_ = i / p.n_slices;
+                const int b = tl_ / p.tiles_per_seq, t0 = (tl_ % p.tiles_per_seq) * kTt;
+                const int o = it % p.op_stages, on = it / p.op_stages;
+                if (!mbar_wait<kWaitHint>(bar.oempty(o), (on & 1) ^ 1, abort, 2u, &g_fault, p.wt.wait_ns)) break;
+                if (it == 0 && (int)blockIdx.x == p.wt.withhold_cta) continue;   // test hook: no loads
+                const uint32_t os = sb + p.off_op + o * p.op_bytes;
+                mbar_arrive_expect_tx(bar.ofull(o), p.z_stage_bytes + p.u_bytes);
+                tma_load_3d(os + p.off_z, &tm_z, bar.ofull(o), 0, t0, b);
+                for (int bx = 0; bx < p.u_boxes; ++bx)
+                    tma_load_2d(os + p.off_u + bx * (uint32_t)(p.R * 128), &tm_u, bar.ofull(o),
+                                slice * p.slice_cols + 64 * bx, 0);
+            }
+            const int issued = it;
+            for (int o = 0; o < p.op_stages && o < issued; ++o) {
+                const int last = issued - 1 - ((issued - 1 - o) % p.op_stages);
+                mbar_drain(bar.ofull(o), (last / p.op_stages) & 1, p.wt.wait_ns);
+            }
+        }
         __syncwarp();
     } else {
         // ---------------------------------------------------------- epilogue

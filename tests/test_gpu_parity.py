@@ -138,6 +138,13 @@ LOWRANK = [
     (2, 500, 256, 4, 4, 16, "bf16"),     # backward: 64 filter columns, padded dU^T block
     (2, 260, 128, 1, 3, 32, "bf16"),     # backward: 192 filter columns, padded dU^T block
     (1, 300, 128, 2, 8, 32, "bf16"),     # backward: G = 2, W = 8
+    # tensor-core backward with grouped filters (tap blocks padded to 16 columns; for
+    # G >= 32 one virtual group per 16 channels, summed into dU)
+    (2, 500, 512, 64, 4, 32, "bf16"),
+    (2, 300, 384, 32, 3, 16, "bf16"),
+    (1, 260, 256, 8, 5, 64, "bf16"),
+    (2, 129, 192, 16, 8, 64, "bf16"),
+    (3, 70, 128, 8, 2, 16, "bf16"),
 ]
 
 
@@ -172,6 +179,14 @@ def test_tensor_core_path_is_selected(dsc):
     for name in ("lowrank_qkv", "lowrank_mlp"):
         wl = di.WORKLOADS[name]
         assert dsc.dsc_lowrank_path(wl.B, wl.T, wl.D, wl.G, wl.W, wl.R) == 3, name
+
+
+def test_grouped_filters_take_the_tensor_core_backward(dsc):
+    """G = 8..64 with R in {16, 32, 64} and D a multiple of 64: the tcgen05 backward
+    (bit 1), which keeps w and dw on chip."""
+    for (B, T, D, G, W, R) in [(2, 500, 512, 64, 4, 32), (2, 300, 384, 32, 3, 16), (1, 260, 256, 8, 5, 64),
+                               (2, 129, 192, 16, 8, 64), (2, 300, 256, 16, 2, 32), (1, 200, 128, 64, 8, 32)]:
+        assert dsc.dsc_lowrank_path(B, T, D, G, W, R) & 2, (B, T, D, G, W, R)
 
 
 def test_no_device_fault_recorded(dsc):
