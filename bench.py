@@ -262,10 +262,10 @@ def run_ours(args, wl, world, rank, local):
     gbs_step = (fwd_b + bwd_b) / (ms_step * 1e-3) / 1e9
     dom = ("dsc_bwd_lowrank", bwd_b, bwd_ms) if bwd_ms >= fwd_ms else ("dsc_fwd_lowrank", fwd_b, fwd_ms)
     achieved = dom[1] / (dom[2] * 1e-3) / 1e9
-    # kernels per call: tcgen05 forward 1; tcgen05 backward 3 (U reorder, main, the dz and
-    # dU reductions in one launch); CUDA-core forward 1, backward 5
+    # kernels per call: tcgen05 forward 1; tcgen05 backward 2 (U reorder with the counter
+    # reset, then the main kernel, which also reduces dz and dU); CUDA-core forward 1, backward 5
     launches_fwd = 1
-    launches_bwd = 3 if path & 2 else 5
+    launches_bwd = 2 if path & 2 else 5
     traffic = load_traffic(dom[0], wl)
 
     # end to end through the public API with host buffers (pinned), copies inside the region

@@ -21,7 +21,7 @@ __all__ = [
     "DscError", "lib", "lib_path", "dsc_fwd", "dsc_fwd_lowrank", "dsc_bwd_lowrank",
     "dsc_bwd_lowrank_workspace_bytes", "dsc_bwd", "dsc_static_fwd", "dsc_static_bwd",
     "dsc_static_bwd_workspace_bytes", "dsc_static_bwd_noalloc", "dsc_lowrank_path",
-    "dsc_decode_step", "dsc_decode_step_lowrank",
+    "dsc_decode_step", "dsc_decode_step_lowrank", "dsc_fwd_lowrank_halo", "dsc_bwd_lowrank_halo",
     "DSC_F32", "DSC_BF16",
 ]
 
@@ -59,6 +59,8 @@ def _load():
         "dsc_lowrank_path": (i, [i, i, i, i, i, i, i]),
         "dsc_decode_step": (i, [vp, vp, vp, vp, i, i, i, i, i, vp]),
         "dsc_decode_step_lowrank": (i, [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]),
+        "dsc_fwd_lowrank_halo": (i, [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]),
+        "dsc_bwd_lowrank_halo": (i, [vp, vp, vp, vp, vp, vp, vp, fp, fp, i, i, i, i, i, i, i, vp]),
         "dsc_device_fault": (ctypes.c_uint, [i]),
         "dsc_test_arm_wait_timeout": (None, [ctypes.c_uint]),
         "dsc_status_string": (ctypes.c_char_p, [i]),
@@ -223,6 +225,33 @@ def dsc_decode_step_lowrank(x_t, z_t, U, state, y_t, G: int, W: int):
         _check(lib.dsc_decode_step_lowrank(_ptr(x_t), _ptr(z_t), _ptr(U), _ptr(state), _ptr(y_t), B, D, G,
                                            W, R, _dt(x_t), _stream(x_t)))
     return y_t
+
+
+def dsc_fwd_lowrank_halo(x, z, U, x_prev, y, G: int, W: int):
+    """Sequence shard fix-up after dsc_fwd_lowrank: recompute y rows t < W-1 with the W-1
+    tokens before the shard, x_prev [B,W-1,D] (oldest first; None for the first shard)."""
+    B, T, D = x.shape
+    R = z.shape[-1]
+    _same(x, z, U, y, *([x_prev] if x_prev is not None else []))
+    with torch.cuda.device(x.device):
+        _check(lib.dsc_fwd_lowrank_halo(_ptr(x), _ptr(z), _ptr(U), _ptr(x_prev), _ptr(y), B, T, D, G, W, R,
+                                        _dt(x), _stream(x)))
+    return y
+
+
+def dsc_bwd_lowrank_halo(x_prev, z, U, dy, dy_next, z_next, dx, dz, dU, G: int, W: int):
+    """Sequence shard fix-up after dsc_bwd_lowrank: recompute dx rows t >= T-(W-1) with the
+    W-1 tokens after the shard (dy_next [B,W-1,D], z_next [B,W-1,R]; None for the last
+    shard) and add the x_prev terms to dz rows t < W-1 and to dU (fp32, in place)."""
+    B, T, D = dy.shape
+    R = z.shape[-1]
+    _same(dy, z, U, dx, dz, dU, *[t for t in (x_prev, dy_next, z_next) if t is not None])
+    if dz.dtype != torch.float32 or dU.dtype != torch.float32:
+        raise TypeError("dsc_bwd_lowrank_halo: dz and dU must be fp32")
+    with torch.cuda.device(dy.device):
+        _check(lib.dsc_bwd_lowrank_halo(_ptr(x_prev), _ptr(z), _ptr(U), _ptr(dy), _ptr(dy_next), _ptr(z_next),
+                                        _ptr(dx), _ptr(dz), _ptr(dU), B, T, D, G, W, R, _dt(dy), _stream(dy)))
+    return dx, dz, dU
 
 
 def dsc_device_fault(reset: bool = False) -> int:

@@ -245,6 +245,46 @@ DSC_API dsc_status_t dsc_decode_step_lowrank(const void *x_t, const void *z_t, c
                                                        (cudaStream_t)stream));
 }
 
+DSC_API dsc_status_t dsc_fwd_lowrank_halo(const void *x, const void *z, const void *U, const void *x_prev,
+                                          void *y, int B, int T, int D, int G, int W, int R, dsc_dtype_t dt,
+                                          dsc_stream_t stream) {
+    const char *fn = "dsc_fwd_lowrank_halo";
+    dsc_status_t st = check_dims(fn, Dims{B, T, D, G, W, R}, dt);
+    if (st != DSC_OK) return st;
+    const void *p[] = {x, z, U, y};
+    const char *n[] = {"x", "z", "U", "y"};
+    if ((st = check_ptrs(fn, p, n, 4)) != DSC_OK) return st;
+    if (x_prev && W > 1) {
+        const void *hp[] = {x_prev};
+        const char *hn[] = {"x_prev"};
+        if ((st = check_ptrs(fn, hp, hn, 1)) != DSC_OK) return st;
+    }
+    return check_launch(fn, dsc::launch_halo_fwd_lowrank(x, z, U, x_prev, y, B, T, D, G, W, R, dt == DSC_BF16,
+                                                         (cudaStream_t)stream));
+}
+
+DSC_API dsc_status_t dsc_bwd_lowrank_halo(const void *x_prev, const void *z, const void *U, const void *dy,
+                                          const void *dy_next, const void *z_next, void *dx, float *dz,
+                                          float *dU, int B, int T, int D, int G, int W, int R, dsc_dtype_t dt,
+                                          dsc_stream_t stream) {
+    const char *fn = "dsc_bwd_lowrank_halo";
+    dsc_status_t st = check_dims(fn, Dims{B, T, D, G, W, R}, dt);
+    if (st != DSC_OK) return st;
+    const void *p[] = {z, U, dy, dx, dz, dU};
+    const char *n[] = {"z", "U", "dy", "dx", "dz", "dU"};
+    if ((st = check_ptrs(fn, p, n, 6)) != DSC_OK) return st;
+    if ((dy_next == nullptr) != (z_next == nullptr))
+        return fail(DSC_ERR_INVALID_ARG, "%s: dy_next and z_next must both be given or both be NULL", fn);
+    if (W > 1) {
+        const void *hp[] = {x_prev, dy_next, z_next};
+        const char *hn[] = {"x_prev", "dy_next", "z_next"};
+        for (int i = 0; i < 3; ++i)
+            if (hp[i] && (st = check_ptrs(fn, hp + i, hn + i, 1)) != DSC_OK) return st;
+    }
+    return check_launch(fn, dsc::launch_halo_bwd_lowrank(x_prev, z, U, dy, dy_next, z_next, dx, dz, dU, B, T, D, G,
+                                                         W, R, dt == DSC_BF16, (cudaStream_t)stream));
+}
+
 DSC_API int dsc_lowrank_path(int B, int T, int D, int G, int W, int R, dsc_dtype_t dt) {
     if (check_dims("dsc_lowrank_path", Dims{B, T, D, G, W, R}, dt) != DSC_OK) return -1;
     const bool bf16 = dt == DSC_BF16;

@@ -29,6 +29,13 @@ cudaError_t launch_decode_lowrank(const void *x, const void *z, const void *U, v
 cudaError_t launch_decode(const void *x, const void *w, void *state, void *y, int B, int D, int G,
                           int W, bool bf16, cudaStream_t s);
 
+// Sequence-shard halo fix-ups (halo.cu)
+cudaError_t launch_halo_fwd_lowrank(const void *x, const void *z, const void *U, const void *x_prev, void *y,
+                                    int B, int T, int D, int G, int W, int R, bool bf16, cudaStream_t s);
+cudaError_t launch_halo_bwd_lowrank(const void *x_prev, const void *z, const void *U, const void *dy,
+                                    const void *dy_next, const void *z_next, void *dx, float *dz, float *dU,
+                                    int B, int T, int D, int G, int W, int R, bool bf16, cudaStream_t s);
+
 // CUDA-core kernels (simt.cu)
 void launch_conv_dx(const void *w, bool w_is_f32, const void *dy, void *dx, int B, int T, int D,
                     int G, int W, bool bf16, bool is_static, cudaStream_t s);

@@ -17,16 +17,13 @@
 // CTAs: CTA (a, b) owns the token tiles of range a and the S slices of group b, and
 // walks them token tile by token tile, its S slices innermost.  Hence
 //   - dz of a token tile accumulates over the CTA's S slices in TMEM and leaves the
-//     CTA once, as one partial of Bg;
+//     CTA once, added into dz with fp32 vector reductions in L2 (the Bg slice groups'
+//     additions land in whatever order they arrive: dz is reproducible to rounding,
+//     not bitwise);
 //   - dU of each of its slices accumulates over all its token tiles in TMEM and
-//     leaves the CTA once, as one partial of A.
-// The Bg CTAs of a token range move through the same token tiles at the same pace, so
-// the partials of a token tile are written close together in time and are summed
-// while they are still in L2: after writing its partial of token tile m, each CTA
-// counts itself in on a per-tile counter, and a reducer warp in every CTA sums its
-// share of the tile's rows (slice groups in a fixed order) once all Bg partials are
-// in.  The A dU partials of each slice group are summed the same way at the end.
-// Every sum runs in a fixed order, so results are deterministic.
+//     leaves the CTA once, as one partial of A; after the last tile the A partials of
+//     each slice group are summed in a fixed order (a counter per group says when all
+//     are written), so dU and dx are bitwise deterministic.
 //
 // Per tile (token tile m, slice s) the CTA's warps do:
 //   warp 0      TMA: dy and x tiles (3-stage ring), z once per token tile, the
@@ -34,15 +31,14 @@
 //               TMA store of dx from the stage once the epilogue has written it there
 //   warp 1      recompute: one MMA per tap k with the z tile shifted by k rows,
 //                 Wk[t, g] = sum_r z[t0+t+k, r] Up[r, k*NG+g],
-//               so TMEM lane t holds w[t+k, g, k] for every k; between tiles, the
-//               gpu-scope publication of each finished dz partial
+//               so TMEM lane t holds w[t+k, g, k] for every k
 //   warp 2      dz[m] += dw Up^T  (A = dw tile, B = Up slice; M=128 tokens, N=R) and
 //               dU^T[s] += dw^T z  (A = dw tile read MN-major, B = z; M=128 columns)
-//   warp 3      reducer: sums the dz partials of its rows of each token tile
+//   warp 3      idle (keeps the epilogue warps four to a sub-partition)
 //   warps 4-19  epilogue, one token row per thread, 16 channels per warp:
 //                 A2: dw (bf16) into the shared-memory dw tile;
 //                 A1: dx, written over the stage's x tile (dead after A2);
-//                 after a token tile's last slice: its dz partial to global memory
+//                 after a token tile's last slice: its dz sum, added into dz
 // The recompute of tile i runs during A2 of tile i, and the dz/dU MMAs of tile i
 // during A1 of tile i.  Every wait is bounded (one second); a wait that runs out
 // makes the CTA leave its loops, record a fault code and free its TMEM.
@@ -70,8 +66,7 @@ constexpr int kCPW = kDt / 4;                   // channels per epilogue warp
 // Warp roles.  Warps 0-3 sit on the SM's four sub-partitions, one each, and the
 // epilogue warps 4-19 four to a sub-partition; 20 warps keep 96 registers a thread.
 constexpr int kRecWarp = 1;
-constexpr int kMmaWarp = 2;                     // dz and dU MMAs
-constexpr int kRedWarp = 3;
+constexpr int kMmaWarp = 2;                     // dz and dU MMAs (warp 3 idles)
 constexpr int kEpi0 = 4;
 constexpr int kThreads = 32 * (kEpi0 + kEpiWarps);
 constexpr int kMaxStages = 3;
@@ -95,9 +90,7 @@ struct BwdParams {
     uint32_t stage_bytes;     // dy tile + x tile
     uint32_t off_z, off_u, off_dw, off_bar;
     uint32_t tm_w, tm_dz, tm_du, tmem_cols;   // TMEM column map
-    float *dz_part;           // [Bg][B*T][R]
     float *du_part;           // [A][R][N]
-    unsigned *flag_dz;        // [n_tt] partials written per token tile (16 per CTA)
     unsigned *flag_du;        // [Bg]   dU partials written per slice group (16 per CTA)
     float *dz;                // [B*T][R]
     float *dU;                // [R][N]
@@ -121,9 +114,8 @@ struct Bars {
     __device__ uint32_t dufull() const { return base + 8 * 22; }
     __device__ uint32_t done() const { return base + 8 * 23; }
     __device__ uint32_t xdead() const { return base + 8 * 24; }
-    __device__ uint32_t dzdone(int d) const { return base + 8 * (25 + d); }
 };
-constexpr uint32_t kBarBytes = 8 * 29;
+constexpr uint32_t kBarBytes = 8 * 25;
 
 __device__ __forceinline__ void unpack8(const uint4 &u, float (&v)[8]) {
     v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x);
@@ -160,13 +152,21 @@ __device__ __forceinline__ void sts64(uint32_t addr, uint32_t a, uint32_t b) {
 }
 
 // ------------------------------------------------------------------ global counters
-// A writer's stores become visible before its count: every lane fences, the warp
-// synchronises, one lane adds with release semantics.  A reader polls with acquire
+// A writer's stores become visible before its count: the writers synchronise with the
+// publishing warp (an mbarrier), which fences at gpu scope and then adds (relaxed; the
+// fence before it makes the pair a release).  A reader polls with acquire
 // semantics (every lane), then reads the data through L2.
 __device__ __forceinline__ void fence_gpu() { asm volatile("fence.acq_rel.gpu;" ::: "memory"); }
 
 __device__ __forceinline__ void red_release_add(unsigned *p, unsigned v) {
     asm volatile("red.release.gpu.global.add.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// dst[0..3] += v (fp32, one vector reduction in L2).
+__device__ __forceinline__ void red_add_v4(float *dst, const uint32_t (&v)[4]) {
+    asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(__uint_as_float(v[0])),
+                 "f"(__uint_as_float(v[1])), "f"(__uint_as_float(v[2])), "f"(__uint_as_float(v[3]))
+                 : "memory");
 }
 
 __device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
@@ -250,7 +250,6 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             mbar_init(bar.dzfull(z), 1);
             mbar_init(bar.dzempty(z), kEpiWarps);
         }
-        for (int z = 0; z < 4; ++z) mbar_init(bar.dzdone(z), kEpiWarps);
         mbar_init(bar.wfull(), 1);
         mbar_init(bar.wempty(), kEpiWarps);
         mbar_init(bar.dwready(), kEpiWarps);
@@ -368,32 +367,12 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
         // Tile i's filters are recomputed once the epilogue has read those of tile i-1:
         //   Wk[t, g] = sum_r z[t0+t+k, r] Up[r, k*NB+g], one MMA chain per tap with the z
         //   tile shifted by k rows (A: z, K-major; B: Up, MN-major).
-        // Between tiles the warp, otherwise idle, publishes each finished dz partial: the
-        // epilogue arrives on dzdone[mz % 4] once token tile mz's partial is stored, and a
-        // gpu-scope fence, then one add of 16 to the tile's counter, make it visible to the
-        // other CTAs.  The epilogue never waits for that fence.
         const uint64_t t_zk = desc_tmpl(p.z_slab, 128, kSwNone);               // z, K-major, no swizzle
         const uint64_t t_u_mn = desc_tmpl((uint32_t)(p.R * 128), 1024, kSw128);  // Up as MN-major B
         const uint32_t i_rec = idesc_bf16(128, p.NGp, false, true);
         const int ksr = p.R / 16;
         const uint32_t ubox = (uint32_t)(p.R * 128);
         const uint64_t st_zk = (2 * p.z_slab) >> 4;   // 16 more z columns (start field units)
-        int published = 0;                            // token tiles published so far
-        auto dz_publish = [&](int upto, bool block) -> bool {   // publish [published, upto)
-            for (; published < upto; ++published) {
-                const int mz = published;
-                if (!block && !__all_sync(0xffffffffu, mbar_try_wait(bar.dzdone(mz & 3), (mz >> 2) & 1)))
-                    return true;   // not stored yet: try again after the next tile
-                if (!warp_wait(bar.dzdone(mz & 3), (mz >> 2) & 1, abort, 2048u, &g_fault_bwd, p.wt.wait_ns))
-                    return false;
-                fence_gpu();
-                __syncwarp();
-                if (lane == 0) red_release_add(p.flag_dz + sp.m0 + mz, (unsigned)kEpiWarps);
-                __syncwarp();
-            }
-            return true;
-        };
-        bool ok = true;
         for (int i = 0; i < nt; ++i) {
             const int j = i % S, mz = i / S, zb = mz & 1;
             const int ub = u_res ? j : (i & 1);
@@ -423,13 +402,9 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
                 if (!u_res) mma_commit(bar.uempty(ub));
             }
             __syncwarp();
-            // partials of the token tiles before this one are stored by now or soon;
-            // publish those that are (without waiting), the rest at a later tile
-            if (!(ok = dz_publish(mz, false))) break;
         }
         if (elect_one()) mma_commit(bar.done());
         __syncwarp();
-        if (ok) dz_publish(nt / S, true);   // the remaining token tiles, the last one included
     } else if (warp >= kEpi0) {
         // ---------------------------------------------------------- epilogue
         const int ew = warp - kEpi0;
@@ -453,9 +428,8 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
         const uint32_t tl = tmem + ((uint32_t)(32 * q) << 16);
         const int nc = p.R / 4;              // dz columns a warp reads out (its group's share)
 
-        // dz partial of token tile mz (this CTA's slices) -> global memory.  The warps then
-        // arrive on a CTA barrier; the reducer warp, off the epilogue's critical path, makes
-        // the partial visible to the other CTAs (gpu-scope release of the tile's count).
+        // dz of token tile mz summed over this CTA's slices, added into dz (fp32 vector
+        // reductions in L2; dz starts at zero, written by the U reorder kernel).
         auto dz_out = [&](int mz) -> bool {
             const int db = mz & 1;
             if (!warp_wait(bar.dzfull(db), (mz >> 1) & 1, abort, 256u, &g_fault_bwd, p.wt.wait_ns)) return false;
@@ -463,21 +437,18 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             const int m = sp.m0 + mz;
             const int b = m / p.tiles_per_seq, t0 = (m - b * p.tiles_per_seq) * kTt;
             const int tok = t0 + row;
-            float *dst = p.dz_part + ((size_t)sp.b * p.B * p.T + (size_t)b * p.T + tok) * p.R + h * nc;
+            float *dst = p.dz + ((size_t)b * p.T + tok) * p.R + h * nc;
             const uint32_t src = tl + p.tm_dz + db * p.R + h * nc;
 #pragma unroll 1
             for (int c0 = 0; c0 < nc; c0 += 4) {
                 uint32_t v[4];
                 tmem_ld<4>(src + c0, v);
                 tmem_wait_ld_regs(v);
-                if (tok < p.T) *reinterpret_cast<uint4 *>(dst + c0) = make_uint4(v[0], v[1], v[2], v[3]);
+                if (tok < p.T) red_add_v4(dst + c0, v);
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(bar.dzempty(db));
-                mbar_arrive(bar.dzdone(mz & 3));
-            }
+            if (lane == 0) mbar_arrive(bar.dzempty(db));
             return true;
         };
 
@@ -795,43 +766,6 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             mma_commit(bar.done());
         }
         __syncwarp();
-    } else if (warp == kRedWarp) {
-        // ---------------------------------------------------------- dz reducer
-        // Once all Bg slice groups have written their partial of token tile m, sum this
-        // CTA's share of its rows over the groups in order and write dz.
-        const int r4 = p.R / 4;                   // float4 per row
-        const int rows_per_pass = 32 / r4;
-        const int lr = lane / r4, l4 = lane - lr * r4;
-        const size_t part_stride = (size_t)p.B * p.T * p.R;
-        const unsigned target = (unsigned)(kEpiWarps * p.Bg);
-        for (int m = sp.m0; m < sp.m1; ++m) {
-            if (!wait_count(p.flag_dz + m, target, abort, 2048u, p.wt.wait_ns)) break;
-            const int b = m / p.tiles_per_seq, t0 = (m - b * p.tiles_per_seq) * kTt;
-            const int nrows = min(kTt, p.T - t0);
-            const int lo = (int)((long long)nrows * sp.b / p.Bg), hi = (int)((long long)nrows * (sp.b + 1) / p.Bg);
-            for (int r0 = lo; r0 < hi; r0 += rows_per_pass) {
-                const int rr = r0 + lr;
-                const bool act = rr < hi;
-                const size_t off = ((size_t)b * p.T + t0 + (act ? rr : lo)) * p.R + 4 * l4;
-                const float *src = p.dz_part + off;
-                // 8 loads in flight per lane; the sum runs over the groups in order
-                float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-                for (int g0 = 0; g0 < p.Bg; g0 += 8) {
-                    float4 v[8];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        if (act && g0 + u < p.Bg)
-                            v[u] = __ldcg(reinterpret_cast<const float4 *>(src + (size_t)(g0 + u) * part_stride));
-#pragma unroll
-                    for (int u = 0; u < 8; ++u)
-                        if (act && g0 + u < p.Bg) {
-                            acc.x += v[u].x; acc.y += v[u].y; acc.z += v[u].z; acc.w += v[u].w;
-                        }
-                }
-                if (act) *reinterpret_cast<float4 *>(p.dz + off) = acc;
-            }
-        }
-        __syncwarp();
     }
 
     __syncthreads();
@@ -848,11 +782,19 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
 // reordering Up[r, s*SC + k*NG + g] = U[r, s*SC + g*W + k].
 // Grid (ceil(N'/2048), R): one row r per grid row; each thread writes 8 consecutive output
 // columns (one tap, 8 consecutive (virtual) groups) with one 16-byte store.  Block (0, 0)
-// also clears the main kernel's counters.
+// also clears the main kernel's counters, and all threads zero dz (which the main
+// kernel adds into).
 __global__ void k_permute_u(const bf16 *__restrict__ U, bf16 *__restrict__ Up, int R, int N, int Nq, int SCq,
-                            int NB, int NGV, int GV, int G, int W, unsigned *__restrict__ flags, int nflags) {
+                            int NB, int NGV, int GV, int G, int W, unsigned *__restrict__ flags, int nflags,
+                            float4 *__restrict__ dz, long long ndz4) {
     if (blockIdx.x == 0 && blockIdx.y == 0)
         for (int f = threadIdx.x; f < nflags; f += blockDim.x) flags[f] = 0u;
+    {
+        // dz is summed into by the main kernel: start it at zero
+        const long long nth = (long long)gridDim.x * gridDim.y * blockDim.x;
+        const long long id = ((long long)blockIdx.y * gridDim.x + blockIdx.x) * blockDim.x + threadIdx.x;
+        for (long long e = id; e < ndz4; e += nth) dz[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     const int r = blockIdx.y;
     const int j = 8 * (blockIdx.x * blockDim.x + threadIdx.x);
     if (r >= R || j >= Nq) return;
@@ -1033,7 +975,7 @@ cudaError_t launch_w(int G, const CUtensorMap *m, const BwdParams &p, cudaStream
 }
 
 struct WsLayout {
-    size_t up, dz, du, flags, total;
+    size_t up, du, flags, total;
 };
 
 WsLayout ws_layout(const BwdParams &p) {
@@ -1041,10 +983,9 @@ WsLayout ws_layout(const BwdParams &p) {
     const size_t N = (size_t)p.n_slices * p.SC;
     const size_t Nq = (size_t)p.n_slices * p.SCq;
     l.up = 0;
-    l.dz = a256(l.up + (size_t)p.R * Nq * 2);
-    l.du = a256(l.dz + (size_t)p.Bg * p.B * p.T * p.R * 4);
+    l.du = a256(l.up + (size_t)p.R * Nq * 2);
     l.flags = a256(l.du + (size_t)p.A * p.R * N * 4);
-    l.total = a256(l.flags + (size_t)(p.n_tt + p.Bg) * 4);
+    l.total = a256(l.flags + (size_t)p.Bg * 4);
     return l;
 }
 
@@ -1072,17 +1013,16 @@ cudaError_t launch_tc_lowrank_bwd(const void *x, const void *z, const void *U, c
     const WsLayout l = ws_layout(p);
     uint8_t *w8 = (uint8_t *)ws;
     bf16 *Up = (bf16 *)(w8 + l.up);
-    p.dz_part = (float *)(w8 + l.dz);
     p.du_part = (float *)(w8 + l.du);
-    p.flag_dz = (unsigned *)(w8 + l.flags);
-    p.flag_du = p.flag_dz + p.n_tt;
+    p.flag_du = (unsigned *)(w8 + l.flags);
     p.dz = dz;
     p.dU = dU;
     const int N = p.n_slices * p.SC;
     const int Nq = p.n_slices * p.SCq;
     const int gv = G < 16 ? G : 16;
     k_permute_u<<<dim3((Nq / 8 + 255) / 256, R), 256, 0, s>>>((const bf16 *)U, Up, R, N, Nq, p.SCq, p.NGp,
-                                                               kDt / gv, gv, G, W, p.flag_dz, p.n_tt + p.Bg);
+                                                               kDt / gv, gv, G, W, p.flag_du, p.Bg,
+                                                               (float4 *)dz, (long long)B * T * R / 4);
 
     CUtensorMap m[5];
     const uint64_t dxyz[3] = {(uint64_t)D, (uint64_t)T, (uint64_t)B};

@@ -184,6 +184,37 @@ DSC_API dsc_status_t dsc_decode_step_lowrank(const void *x_t, const void *z_t, c
                                              int B, int D, int G, int W, int R,
                                              dsc_dtype_t dt, dsc_stream_t stream);
 
+/* Sequence sharding (a sequence of length P*T split into P consecutive shards of T
+ * tokens, one per rank).  Each rank calls dsc_fwd_lowrank / dsc_bwd_lowrank on its own
+ * shard, which treats the shard as a whole sequence, and then the matching halo call
+ * below on the same stream.  The causal window reaches W-1 tokens back ("Metodologia:
+ * Mecanismo"), so only W-1 rows per sequence differ from the unsharded result:
+ *   dsc_fwd_lowrank_halo: recomputes y rows t < min(W-1, T) with x[t-k], t-k < 0, read
+ *     from x_prev (overwrites those rows of y);
+ *   dsc_bwd_lowrank_halo: recomputes dx rows t >= T-(W-1) with dy[t+k] and
+ *     w[t+k] = z[t+k] U, t+k >= T, read from dy_next / z_next (overwrites those rows of
+ *     dx), and adds to dz rows t < W-1 and to dU the filter-gradient terms
+ *     dw[t,g,k] = sum_{c in g} dy[t,c] x_prev[W-1+t-k, c] for k > t that the shard's call
+ *     could not see (dz and dU are accumulated in fp32, not overwritten).
+ *   x_prev  [B, W-1, D]: the W-1 tokens just before the shard (row 0 the oldest), or
+ *           NULL for the first shard (nothing to do: the zero padding is right);
+ *   dy_next [B, W-1, D], z_next [B, W-1, R]: the W-1 tokens just after the shard, or
+ *           both NULL for the last shard;
+ *   the other arguments, shapes and types are those of the shard's own call (T is the
+ *   shard length, any T >= 1; when T < W-1 the halos span several shards and the caller
+ *   assembles them).  dU is this rank's: summing it over the ranks (and over data-
+ *   parallel replicas) is the caller's collective.  Deterministic: fixed summation
+ *   orders, no atomics.  DSC_ERR_INVALID_ARG if exactly one of dy_next / z_next is NULL. */
+DSC_API dsc_status_t dsc_fwd_lowrank_halo(const void *x, const void *z, const void *U,
+                                          const void *x_prev, void *y,
+                                          int B, int T, int D, int G, int W, int R,
+                                          dsc_dtype_t dt, dsc_stream_t stream);
+DSC_API dsc_status_t dsc_bwd_lowrank_halo(const void *x_prev, const void *z, const void *U,
+                                          const void *dy, const void *dy_next, const void *z_next,
+                                          void *dx, float *dz, float *dU,
+                                          int B, int T, int D, int G, int W, int R,
+                                          dsc_dtype_t dt, dsc_stream_t stream);
+
 /* Which implementations the low-rank entry points use for these sizes: bit 0 set when
  * dsc_fwd_lowrank runs on the tensor-core (tcgen05) kernel, bit 1 when
  * dsc_bwd_lowrank does; 0 = both on CUDA cores; -1 = invalid sizes.  The tensor-core

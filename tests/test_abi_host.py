@@ -112,3 +112,22 @@ def test_lowrank_path_query(dsc):
     assert L.dsc_lowrank_path(2, 8, 64, 1, 4, 32, 0) == 0      # fp32: CUDA cores
     assert L.dsc_lowrank_path(2, 8, 64, 1, 4, 3, 1) == 0       # R=3: CUDA cores
     assert L.dsc_lowrank_path(2, 8, 64, 1, 4, 32, 1) in (0, 1, 2, 3)
+
+
+def test_halo_validation(dsc):
+    """The sequence-shard fix-ups check their arguments before launching anything."""
+    L = dsc.lib
+    B, T, D, G, W, R = 2, 8, 64, 1, 4, 32
+    # a next-shard halo needs both dy_next and z_next
+    assert L.dsc_bwd_lowrank_halo(FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE,
+                                  B, T, D, G, W, R, 1, None) == 1
+    assert L.dsc_bwd_lowrank_halo(FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE,
+                                  B, T, D, G, W, R, 1, None) == 1
+    # required tensors, alignment, sizes
+    assert L.dsc_bwd_lowrank_halo(FAKE, FAKE, FAKE, FAKE, None, None, None, FAKE, FAKE,
+                                  B, T, D, G, W, R, 1, None) == 1
+    assert L.dsc_bwd_lowrank_halo(ODD, FAKE, FAKE, FAKE, None, None, FAKE, FAKE, FAKE,
+                                  B, T, D, G, W, R, 1, None) == 2
+    assert L.dsc_fwd_lowrank_halo(FAKE, FAKE, FAKE, FAKE, None, B, T, D, G, W, R, 1, None) == 1
+    assert L.dsc_fwd_lowrank_halo(FAKE, FAKE, FAKE, ODD, FAKE, B, T, D, G, W, R, 1, None) == 2
+    assert L.dsc_fwd_lowrank_halo(FAKE, FAKE, FAKE, FAKE, FAKE, B, T, D, G, 9, R, 1, None) == 2
