@@ -203,6 +203,29 @@ struct Span {
     __device__ int S() const { return s1 - s0; }
     __device__ int tiles() const { return (m1 - m0) * (s1 - s0); }
 };
+// Position in a CTA's walk over its tiles (token tiles outermost, its S slices
+// innermost), advanced by increments so that the loops divide by nothing.
+struct Walk {
+    int i = 0;                // tile
+    int j = 0, mz = 0;        // slice within the segment, token tile within the CTA
+    int st = 0, n = 0;        // ring stage and round
+    int b, tt;                // sequence and tile within it of token tile m0 + mz
+    __device__ Walk(int m0, int tiles_per_seq) {
+        b = m0 / tiles_per_seq;
+        tt = m0 - b * tiles_per_seq;
+    }
+    __device__ int t0() const { return tt * kTt; }
+    __device__ void next(int S, int NST, int tiles_per_seq) {
+        ++i;
+        if (++st == NST) { st = 0; ++n; }
+        if (++j == S) {
+            j = 0;
+            ++mz;
+            if (++tt == tiles_per_seq) { tt = 0; ++b; }
+        }
+    }
+};
+
 __device__ __forceinline__ Span span_of(const BwdParams &p) {
     Span s;
     s.a = (int)blockIdx.x / p.Bg;
@@ -222,6 +245,7 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
     using CL = Cols<W, G>;
     constexpr int GV = CL::GV;
     constexpr int NG8 = GV <= 8 ? 8 / GV : 1;   // (virtual) groups in one 8-channel chunk
+    constexpr int NGS = kDt / G;                 // filter groups per slice
     constexpr int CH = kCPW / 8;        // 16-byte chunks of a warp's channels in a row
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -306,11 +330,9 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             bool ok = true;
             if (u_res)
                 for (int j = 0; j < S; ++j) { load_up(j, sp.s0 + j); ++uissued; }
-            for (int i = 0; i < nt && ok; ++i) {
-                const int st = i % NST, n = i / NST;
-                const int j = i % S, mz = i / S;
-                const int m = sp.m0 + mz, slice = sp.s0 + j;
-                const int b = m / p.tiles_per_seq, t0 = (m - b * p.tiles_per_seq) * kTt;
+            for (Walk w(sp.m0, p.tiles_per_seq); w.i < nt && ok; w.next(S, NST, p.tiles_per_seq)) {
+                const int i = w.i, st = w.st, n = w.n, j = w.j, mz = w.mz;
+                const int slice = sp.s0 + j, b = w.b, t0 = w.t0();
                 if (i >= NST) {
                     // the stage is free once tile i-NST's dx, written over its x tile, is stored
                     if (!mbar_wait(bar.dxr(st), (n - 1) & 1, abort, 1u, &g_fault_bwd, p.wt.wait_ns)) { ok = false; break; }
@@ -362,19 +384,19 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
         __syncwarp();
     } else if (warp == kRecWarp) {
         // ---------------------------------------------------------- MMA issuer: recompute
-        // Each MMA warp runs its schedule warp-uniformly; one elected lane issues each
-        // tcgen05 instruction, and descriptors advance by adding to their start field.
+        // Each MMA warp waits warp-uniformly; one elected lane then issues a tile's
+        // tcgen05 instructions in a row, descriptors advancing by adds to their start field.
         // Tile i's filters are recomputed once the epilogue has read those of tile i-1:
         //   Wk[t, g] = sum_r z[t0+t+k, r] Up[r, k*NB+g], one MMA chain per tap with the z
         //   tile shifted by k rows (A: z, K-major; B: Up, MN-major).
         const uint64_t t_zk = desc_tmpl(p.z_slab, 128, kSwNone);               // z, K-major, no swizzle
         const uint64_t t_u_mn = desc_tmpl((uint32_t)(p.R * 128), 1024, kSw128);  // Up as MN-major B
-        const uint32_t i_rec = idesc_bf16(128, p.NGp, false, true);
+        const uint32_t i_rec = idesc_bf16(128, CL::NB, false, true);
         const int ksr = p.R / 16;
         const uint32_t ubox = (uint32_t)(p.R * 128);
         const uint64_t st_zk = (2 * p.z_slab) >> 4;   // 16 more z columns (start field units)
-        for (int i = 0; i < nt; ++i) {
-            const int j = i % S, mz = i / S, zb = mz & 1;
+        for (Walk w(sp.m0, p.tiles_per_seq); w.i < nt; w.next(S, NST, p.tiles_per_seq)) {
+            const int i = w.i, j = w.j, mz = w.mz, zb = mz & 1;
             const int ub = u_res ? j : (i & 1);
             const int upar = u_res ? 0 : ((i >> 1) & 1);
             if (j == 0 && !warp_wait(bar.zfull(zb), (mz >> 1) & 1, abort, 4u, &g_fault_bwd, p.wt.wait_ns)) break;
@@ -383,20 +405,19 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             tc_fence_after();
             const uint32_t zs = sb + p.off_z + zb * p.z_bytes;
             const uint32_t us = sb + p.off_u + ub * p.u_bytes;
+            if (elect_one()) {      // one lane issues the tile's MMAs and commits
 #pragma unroll
-            for (int k = 0; k < W; ++k) {
-                const int col0 = k * CL::NB;
-                uint64_t da = desc_at(t_zk, zs + 16 * k);
-                uint64_t db = desc_at(t_u_mn, us + (col0 / 64) * ubox + (col0 % 64) * 2);
-                const uint32_t d = tmem + p.tm_w + k * p.NGp;
-                for (int kk = 0; kk < ksr; ++kk) {
-                    if (elect_one()) mma_bf16_ss(d, da, db, i_rec, kk > 0 ? 1u : 0u);
-                    __syncwarp();
-                    da += st_zk;
-                    db += 2048u >> 4;
+                for (int k = 0; k < W; ++k) {
+                    const int col0 = k * CL::NB;
+                    uint64_t da = desc_at(t_zk, zs + 16 * k);
+                    uint64_t db = desc_at(t_u_mn, us + (col0 / 64) * ubox + (col0 % 64) * 2);
+                    const uint32_t d = tmem + p.tm_w + k * CL::NB;
+                    for (int kk = 0; kk < ksr; ++kk) {
+                        mma_bf16_ss(d, da, db, i_rec, kk > 0 ? 1u : 0u);
+                        da += st_zk;
+                        db += 2048u >> 4;
+                    }
                 }
-            }
-            if (elect_one()) {
                 mma_commit(bar.wfull());
                 if (j == S - 1) mma_commit(bar.zempty(zb));
                 if (!u_res) mma_commit(bar.uempty(ub));
@@ -430,21 +451,27 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
 
         // dz of token tile mz summed over this CTA's slices, added into dz (fp32 vector
         // reductions in L2; dz starts at zero, written by the U reorder kernel).
-        auto dz_out = [&](int mz) -> bool {
+        auto dz_out = [&](int mz, int b, int t0) -> bool {
             const int db = mz & 1;
             if (!warp_wait(bar.dzfull(db), (mz >> 1) & 1, abort, 256u, &g_fault_bwd, p.wt.wait_ns)) return false;
             tc_fence_after();
-            const int m = sp.m0 + mz;
-            const int b = m / p.tiles_per_seq, t0 = (m - b * p.tiles_per_seq) * kTt;
             const int tok = t0 + row;
             float *dst = p.dz + ((size_t)b * p.T + tok) * p.R + h * nc;
             const uint32_t src = tl + p.tm_dz + db * p.R + h * nc;
 #pragma unroll 1
-            for (int c0 = 0; c0 < nc; c0 += 4) {
-                uint32_t v[4];
-                tmem_ld<4>(src + c0, v);
+            for (int c0 = 0; c0 < nc; c0 += 8) {
+                uint32_t v[8];
+                if (nc >= 8) {
+                    tmem_ld<8>(src + c0, v);
+                } else {
+                    tmem_ld<4>(src + c0, v);
+                    v[4] = v[5] = v[6] = v[7] = 0u;
+                }
                 tmem_wait_ld_regs(v);
-                if (tok < p.T) red_add_v4(dst + c0, v);
+                if (tok < p.T) {
+                    red_add_v4(dst + c0, *reinterpret_cast<const uint32_t(*)[4]>(v));
+                    if (nc >= 8) red_add_v4(dst + c0 + 4, *reinterpret_cast<const uint32_t(*)[4]>(v + 4));
+                }
             }
             tc_fence_before();
             __syncwarp();
@@ -453,9 +480,10 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
         };
 
         bool ok = true;
-        for (int i = 0; i < nt; ++i) {
-            const int j = i % S, mz = i / S;
-            const int st = i % NST, n = i / NST;
+        int pb = 0, pt0 = 0;                 // sequence and first token of the previous token tile
+        for (Walk w(sp.m0, p.tiles_per_seq); w.i < nt; w.next(S, NST, p.tiles_per_seq)) {
+            const int i = w.i, j = w.j, mz = w.mz;
+            const int st = w.st, n = w.n;
             if (!warp_wait(bar.full(st), n & 1, abort, 64u, &g_fault_bwd, p.wt.wait_ns)) { ok = false; break; }
             const uint32_t dys = sb + st * p.stage_bytes, xs = dys + p.xy_tile_bytes;
 
@@ -499,7 +527,7 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
                 const int g8 = (kCPW * h + 8 * cq) / G;
 #pragma unroll
                 for (int k = 0; k < W; ++k) {
-                    const int jp = k * p.NGs + g8;                    // first tap-major column
+                    const int jp = k * NGS + g8;                      // first tap-major column
                     const uint32_t atom = (uint32_t)(jp >> 6), within = (uint32_t)(jp & 63);
                     const uint32_t a = dwrow + atom * 16384u + ((((within >> 3) << 4) ^ dwsw) | ((within & 7) * 2));
                     if constexpr (NG8 == 8) {
@@ -560,7 +588,10 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar.dwready());
+            if (lane == 0) {
+                mbar_arrive(bar.dwready());
+                mbar_arrive(bar.xdead());       // this warp's reads of the x tile are done
+            }
 
             // ---- A1: dx[t,c] = dy[t,c] + sum_k w[t+k,g,k] dy[t+k,c]
             if (!warp_wait(bar.wfull(), i & 1, abort, 128u, &g_fault_bwd, p.wt.wait_ns)) { ok = false; break; }
@@ -582,7 +613,7 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
 #pragma unroll
                     for (int kb = 0; kb < KB; ++kb)
                         if (k0 + kb < W)
-                            tmem_ld<NGB>(tl + p.tm_w + (k0 + kb) * p.NGp + (kCPW * h + 8 * cq) / GV, wr[kb]);
+                            tmem_ld<NGB>(tl + p.tm_w + (k0 + kb) * CL::NB + (kCPW * h + 8 * cq) / GV, wr[kb]);
                     tmem_wait_ld();
 #pragma unroll
                     for (int kb = 0; kb < KB; ++kb)
@@ -624,7 +655,6 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             if (lane == 0) mbar_arrive(bar.wempty());
             // once every epilogue warp is past A2 the x tile is dead, and dx goes there
             // (an mbarrier rather than a named barrier, so that the wait is bounded)
-            if (lane == 0) mbar_arrive(bar.xdead());
             if (!warp_wait(bar.xdead(), i & 1, abort, 4096u, &g_fault_bwd, p.wt.wait_ns)) { ok = false; break; }
 #pragma unroll
             for (int cq = 0; cq < CH; ++cq) sts128(xs + (dxr0 ^ ((uint32_t)cq << 4)), dxo[cq]);
@@ -633,9 +663,13 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             if (lane == 0) mbar_arrive(bar.dxr(st));
 
             // ---- dz of the previous token tile, complete once its last slice's MMAs ran
-            if (j == 0 && mz > 0 && !dz_out(mz - 1)) { ok = false; break; }
+            if (j == 0 && mz > 0 && !dz_out(mz - 1, pb, pt0)) { ok = false; break; }
+            if (j == S - 1) {
+                pb = w.b;
+                pt0 = w.t0();
+            }
         }
-        if (ok && nt > 0) ok = dz_out(nt / S - 1);
+        if (ok && nt > 0) ok = dz_out(nt / S - 1, pb, pt0);
 
         // ---- dU: this CTA's partial of each of its slices, then the slice group's sum
         if (ok && warp_wait(bar.dufull(), 0, abort, 512u, &g_fault_bwd, p.wt.wait_ns)) {
@@ -714,8 +748,8 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
         const uint64_t st_wrap_a = (16384u - 96u) >> 4;   // next 64-column dw atom
         const uint64_t st_wrap_b = (ubox - 96u) >> 4;     // next 64-column Up box
         const uint32_t dw0 = sb + p.off_dw;
-        for (int i = 0; i < nt; ++i) {
-            const int j = i % S, mz = i / S, db = mz & 1, zb = mz & 1;
+        for (Walk w(sp.m0, p.tiles_per_seq); w.i < nt; w.next(S, NST, p.tiles_per_seq)) {
+            const int i = w.i, j = w.j, mz = w.mz, db = mz & 1, zb = mz & 1;
             const int ub = u_res ? j : (i & 1);
             const int upar = u_res ? 0 : ((i >> 1) & 1);
             if (!warp_wait(bar.ufull(ub), upar, abort, 4u, &g_fault_bwd, p.wt.wait_ns)) break;
@@ -723,35 +757,33 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             if (!warp_wait(bar.dwready(), i & 1, abort, 8u, &g_fault_bwd, p.wt.wait_ns)) break;
             if (j == 0 && !warp_wait(bar.dzempty(db), ((mz >> 1) & 1) ^ 1, abort, 8u, &g_fault_bwd, p.wt.wait_ns)) break;
             tc_fence_after();
-            {
-                const uint32_t us = sb + p.off_u + ub * p.u_bytes;
-                uint64_t da = desc_at(t_k128, dw0), dbd = desc_at(t_k128, us);
-                const uint32_t d = tmem + p.tm_dz + db * p.R;
+            if (elect_one()) {      // one lane issues the tile's MMAs and commits
+                {
+                    const uint32_t us = sb + p.off_u + ub * p.u_bytes;
+                    uint64_t da = desc_at(t_k128, dw0), dbd = desc_at(t_k128, us);
+                    const uint32_t d = tmem + p.tm_dz + db * p.R;
 #pragma unroll
-                for (int kk = 0; kk < KSC; ++kk) {
-                    if (elect_one()) mma_bf16_ss(d, da, dbd, i_dz, (j > 0 || kk > 0) ? 1u : 0u);
-                    __syncwarp();
-                    const bool wrap = (kk & 3) == 3;
-                    da += wrap ? st_wrap_a : 2u;
-                    dbd += wrap ? st_wrap_b : 2u;
-                }
-            }
-            {
-                const uint32_t zs = sb + p.off_z + zb * p.z_bytes;
-#pragma unroll
-                for (int mb = 0; mb < NMB; ++mb) {
-                    const uint32_t d = tmem + p.tm_du + (j * NMB + mb) * p.R;
-                    uint64_t da = desc_at(t_dwt, dw0 + mb * 32768u), dbd = desc_at(t_zmn, zs);
-#pragma unroll
-                    for (int kk = 0; kk < kTt / 16; ++kk) {
-                        if (elect_one()) mma_bf16_ss(d, da, dbd, i_du, (mz == 0 && kk == 0) ? 0u : 1u);
-                        __syncwarp();
-                        da += 2048u >> 4;
-                        dbd += 256u >> 4;
+                    for (int kk = 0; kk < KSC; ++kk) {
+                        mma_bf16_ss(d, da, dbd, i_dz, (j > 0 || kk > 0) ? 1u : 0u);
+                        const bool wrap = (kk & 3) == 3;
+                        da += wrap ? st_wrap_a : 2u;
+                        dbd += wrap ? st_wrap_b : 2u;
                     }
                 }
-            }
-            if (elect_one()) {
+                {
+                    const uint32_t zs = sb + p.off_z + zb * p.z_bytes;
+#pragma unroll
+                    for (int mb = 0; mb < NMB; ++mb) {
+                        const uint32_t d = tmem + p.tm_du + (j * NMB + mb) * p.R;
+                        uint64_t da = desc_at(t_dwt, dw0 + mb * 32768u), dbd = desc_at(t_zmn, zs);
+#pragma unroll
+                        for (int kk = 0; kk < kTt / 16; ++kk) {
+                            mma_bf16_ss(d, da, dbd, i_du, (mz == 0 && kk == 0) ? 0u : 1u);
+                            da += 2048u >> 4;
+                            dbd += 256u >> 4;
+                        }
+                    }
+                }
                 mma_commit(bar.dwfree());
                 if (!u_res) mma_commit(bar.uempty(ub));
                 if (j == S - 1) {

@@ -232,8 +232,8 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
         __syncwarp();
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
-        // The whole warp runs the schedule; one elected lane issues each tcgen05
-        // instruction, and descriptors advance by adding to their start-address field.
+        // The whole warp waits; one elected lane then issues a tile's tcgen05 instructions
+        // in a row, descriptors advancing by adds to their start-address field.
         const int nchunks = (p.n_pad + 255) / 256;
         const uint32_t ubox = (uint32_t)(p.R * 128);
         const int ksteps = p.R / 16;
@@ -241,31 +241,30 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
         const uint64_t t_u = desc_tmpl(ubox, 1024, kSw128);              // U slice, MN-major
         const uint32_t i_full = idesc_bf16(128, 256, false, true);
         const uint32_t i_last = idesc_bf16(128, p.n_pad - 256 * (nchunks - 1), false, true);
-        int it = 0;
+        int it = 0, a = 0, m = 0;    // accumulator a of round m, advanced by increments
         for (int i = blockIdx.x; i < p.n_tiles; i += gridDim.x, ++it) {
-            const int o = it % p.op_stages, on = it / p.op_stages;
-            const int a = it % p.nbuf, m = it / p.nbuf;
+            const int o = it % kOpStages, on = it / kOpStages;
             if (!warp_wait<kWaitHint>(bar.ofull(o), on & 1, abort, 8u, &g_fault, p.wt.wait_ns)) break;
             if (!warp_wait<kWaitHint>(bar.acce(a), (m & 1) ^ 1, abort, 16u, &g_fault, p.wt.wait_ns)) break;
             tc_fence_after();
             const uint32_t d = tmem + a * p.bufcols;
             const uint32_t za = sb + p.off_op + o * p.op_bytes + p.off_z;
             const uint32_t ua = sb + p.off_op + o * p.op_bytes + p.off_u;
-            for (int nc = 0; nc < nchunks; ++nc) {
-                const uint32_t idesc = nc + 1 < nchunks ? i_full : i_last;
-                uint64_t dz = desc_at(t_z, za), du = desc_at(t_u, ua + nc * 4 * ubox);
-                for (int kk = 0; kk < ksteps; ++kk) {
-                    if (elect_one()) mma_bf16_ss(d + 256 * nc, dz, du, idesc, kk > 0 ? 1u : 0u);
-                    __syncwarp();
-                    dz += 32u >> 4;
-                    du += 2048u >> 4;
+            if (elect_one()) {      // one lane issues the tile's MMAs and commits
+                for (int nc = 0; nc < nchunks; ++nc) {
+                    const uint32_t idesc = nc + 1 < nchunks ? i_full : i_last;
+                    uint64_t dz = desc_at(t_z, za), du = desc_at(t_u, ua + nc * 4 * ubox);
+                    for (int kk = 0; kk < ksteps; ++kk) {
+                        mma_bf16_ss(d + 256 * nc, dz, du, idesc, kk > 0 ? 1u : 0u);
+                        dz += 32u >> 4;
+                        du += 2048u >> 4;
+                    }
                 }
-            }
-            if (elect_one()) {
                 mma_commit(bar.accf(a));
                 mma_commit(bar.oempty(o));
             }
             __syncwarp();
+            if (++a == p.nbuf) { a = 0; ++m; }
         }
         if (elect_one()) mma_commit(bar.done());
         __syncwarp();
@@ -276,7 +275,7 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
             for (int i = blockIdx.x; i < p.n_tiles; i += gridDim.x, ++it) {
                 const int slice = i % p.n_slices, tl_ = i / p.n_slices;
                 const int b = tl_ / p.tiles_per_seq, t0 = (tl_ % p.tiles_per_seq) * kTt;
-                const int o = it % p.op_stages, on = it / p.op_stages;
+                const int o = it % kOpStages, on = it / kOpStages;
                 if (!mbar_wait<kWaitHint>(bar.oempty(o), (on & 1) ^ 1, abort, 2u, &g_fault, p.wt.wait_ns)) break;
                 if (it == 0 && (int)blockIdx.x == p.wt.withhold_cta) continue;   // test hook: no loads
                 const uint32_t os = sb + p.off_op + o * p.op_bytes;
@@ -313,15 +312,17 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
             xrow[k] = (r * 128u) ^ ((r & 7u) << 4) ^ ((uint32_t)(4 * h) << 4);
         }
         int yc = 0;
-        int it = set;
+        const int it0 = set;
         int i = blockIdx.x + set * gridDim.x;
+        // this set's position, advanced by increments: slice and token tile (tlin; its
+        // sequence b and tile tt within it), x stage s of round n, accumulator a of round m
         int slice = i % p.n_slices, tlin = i / p.n_slices;
+        int b = tlin / p.tiles_per_seq, tt = tlin - b * p.tiles_per_seq;
+        int s = it0 % S, n = it0 / S, a = it0 % p.nbuf, m = it0 / p.nbuf;
         const int step = ES::SETS * gridDim.x;
         const int dslice = step % p.n_slices, dtl = step / p.n_slices;
-        for (; i < p.n_tiles; it += ES::SETS, i += step) {
-            const int b = tlin / p.tiles_per_seq, t0 = (tlin - b * p.tiles_per_seq) * kTt;
-            const int s = it % S, n = it / S;
-            const int a = it % p.nbuf, m = it / p.nbuf;
+        for (; i < p.n_tiles; i += step) {
+            const int t0 = tt * kTt;
             if (!warp_wait<kWaitHint>(bar.full(s), n & 1, abort, 32u, &g_fault, p.wt.wait_ns)) break;
             if (!warp_wait<kWaitHint>(bar.accf(a), m & 1, abort, 64u, &g_fault, p.wt.wait_ns)) break;
             tc_fence_after();
@@ -373,10 +374,19 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
             }
             ++yc;
             slice += dslice;
-            tlin += dtl;
+            tt += dtl;
             if (slice >= p.n_slices) {
                 slice -= p.n_slices;
-                ++tlin;
+                ++tt;
+            }
+            if (tt >= p.tiles_per_seq) {
+                b += tt / p.tiles_per_seq;
+                tt -= (tt / p.tiles_per_seq) * p.tiles_per_seq;
+            }
+            if ((s += ES::SETS) >= S) { s -= S; ++n; }
+            if ((a += ES::SETS) >= p.nbuf) {
+                m += a / p.nbuf;
+                a -= (a / p.nbuf) * p.nbuf;
             }
         }
         if (lane == 0) bulk_wait_all();
