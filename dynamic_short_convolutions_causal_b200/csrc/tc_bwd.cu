@@ -468,7 +468,24 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
                     v[4] = v[5] = v[6] = v[7] = 0u;
                 }
                 tmem_wait_ld_regs(v);
-                if (tok < p.T) {
+                if (nc == 8) {
+                    // a lane holds 32 contiguous bytes of its row; regrouped so that each
+                    // reduction covers 16 rows x 32 bytes (16 sectors) instead of 32 rows
+                    // x 16 bytes (32 sectors): lane l adds half l&1 of row 16*ps + l/2
+#pragma unroll
+                    for (int ps = 0; ps < 2; ++ps) {
+                        const int sl = 16 * ps + (lane >> 1), hf = lane & 1;
+                        uint32_t u[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const uint32_t lo = __shfl_sync(0xffffffffu, v[e], sl);
+                            const uint32_t hi = __shfl_sync(0xffffffffu, v[4 + e], sl);
+                            u[e] = hf ? hi : lo;
+                        }
+                        const int rt = t0 + 32 * q + sl;
+                        if (rt < p.T) red_add_v4(p.dz + ((size_t)b * p.T + rt) * p.R + h * nc + c0 + 4 * hf, u);
+                    }
+                } else if (tok < p.T) {
                     red_add_v4(dst + c0, *reinterpret_cast<const uint32_t(*)[4]>(v));
                     if (nc >= 8) red_add_v4(dst + c0 + 4, *reinterpret_cast<const uint32_t(*)[4]>(v + 4));
                 }
@@ -508,14 +525,15 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
                         pk[k][2] = bf16x2_mul(d0.z, xu[k].z);
                         pk[k][3] = bf16x2_mul(d0.w, xu[k].w);
                     } else if constexpr (G <= 4) {
-                        float dv[8], xv[8], dw[NG8];
-                        unpack8(d0, dv);
-                        unpack8(xu[k], xv);
+                        const uint32_t dq[4] = {d0.x, d0.y, d0.z, d0.w};
+                        const uint32_t xq[4] = {xu[k].x, xu[k].y, xu[k].z, xu[k].w};
+                        float dw[NG8];
 #pragma unroll
                         for (int gl = 0; gl < NG8; ++gl) {
                             float acc = 0.f;
 #pragma unroll
-                            for (int e = gl * G; e < (gl + 1) * G; ++e) acc = fmaf(dv[e], xv[e], acc);
+                            for (int e = gl * G; e < (gl + 1) * G; ++e)
+                                acc = (e & 1) ? fma_bf16_hi(dq[e >> 1], xq[e >> 1], acc) : fma_bf16_lo(dq[e >> 1], xq[e >> 1], acc);
                             dw[gl] = acc;
                         }
 #pragma unroll
@@ -545,15 +563,16 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
                 float sv[CH][W];
 #pragma unroll
                 for (int cq = 0; cq < CH; ++cq) {
-                    float dv[8];
-                    unpack8(lds128(dys + (dyr[0] ^ ((uint32_t)cq << 4))), dv);
+                    const uint4 d4 = lds128(dys + (dyr[0] ^ ((uint32_t)cq << 4)));
+                    const uint32_t dq[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
                     for (int k = 0; k < W; ++k) {
-                        float xv[8];
-                        unpack8(lds128(xs + (xr[k] ^ ((uint32_t)cq << 4))), xv);
+                        const uint4 x4 = lds128(xs + (xr[k] ^ ((uint32_t)cq << 4)));
+                        const uint32_t xq[4] = {x4.x, x4.y, x4.z, x4.w};
                         float acc = 0.f;
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) acc = fmaf(dv[e], xv[e], acc);
+                        for (int e = 0; e < 8; ++e)
+                            acc = (e & 1) ? fma_bf16_hi(dq[e >> 1], xq[e >> 1], acc) : fma_bf16_lo(dq[e >> 1], xq[e >> 1], acc);
                         sv[cq][k] = acc;
                     }
                 }
@@ -663,7 +682,12 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             if (lane == 0) mbar_arrive(bar.dxr(st));
 
             // ---- dz of the previous token tile, complete once its last slice's MMAs ran
-            if (j == 0 && mz > 0 && !dz_out(mz - 1, pb, pt0)) { ok = false; break; }
+            // the previous token tile's dz; half the warps a slice later, so that fewer
+            // reductions queue at once (lowrank_qkv 0.238 -> 0.227 ms)
+            {
+                const int jd = (S >= 2 && h >= 2) ? 1 : 0;
+                if (j == jd && mz > 0 && !dz_out(mz - 1, pb, pt0)) { ok = false; break; }
+            }
             if (j == S - 1) {
                 pb = w.b;
                 pt0 = w.t0();
