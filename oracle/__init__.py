@@ -60,6 +60,7 @@ def _bind(lib):
         "oracle_static_bwd": (None, [dp, dp, dp, dp, dp, i, i, i, i]),
         "oracle_decode": (None, [dp, dp, dp, dp, dp, i, i, i, i]),
         "oracle_decode_lowrank": (i, [dp, dp, dp, dp, dp, dp, i, i, i, i, i]),
+        "oracle_rope": (None, [dp, dp, i, i, i, i, i, i]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -220,6 +221,29 @@ class Oracle:
             raise MemoryError("oracle_decode_lowrank")
         return y, st
 
+    def rope(self, y, cs, dh, n_rot, transpose=False):
+        """RoPE of the first n_rot channels of y [B,T,D] (heads of dh channels, adjacent
+        pairs rotated; cs [T, dh/2, 2] holds cos, sin); returns a rotated copy.
+        transpose=True rotates by the opposite angle (the transpose)."""
+        y = np.asarray(y)
+        B, T, D = y.shape
+        if dh < 2 or dh % 2 or n_rot % dh or not 0 <= n_rot <= D:
+            raise ValueError("oracle.rope: bad dh=%d n_rot=%d for D=%d" % (dh, n_rot, D))
+        out = _in(y, (B, T, D)).copy()
+        cs = _in(cs, (T, dh // 2, 2))
+        self._l.oracle_rope(_p(out), _p(cs), B, T, D, dh, n_rot, 1 if transpose else 0)
+        return out
+
+    def fwd_lowrank_rope(self, x, z, U, cs, G, W, dh, n_rot):
+        """RoPE(x + dynconv(x; w = z U)): the op followed by the rotation of its Q and K
+        channels (Posicionamento: the convolution sits before RoPE)."""
+        return self.rope(self.fwd_lowrank(x, z, U, G, W), cs, dh, n_rot)
+
+    def bwd_lowrank_rope(self, x, z, U, cs, dy_rot, G, W, dh, n_rot):
+        """Backward of fwd_lowrank_rope given the gradient of its rotated output:
+        bwd_lowrank with dy = RoPE^T(dy_rot).  Returns (dx, dz, dU)."""
+        return self.bwd_lowrank(x, z, U, self.rope(dy_rot, cs, dh, n_rot, transpose=True), G, W)
+
 
 def default() -> Oracle:
     global _default
@@ -269,6 +293,18 @@ def static_bwd(x, ws, dy):
 
 def decode(x_t, w_t, state, G):
     return default().decode(x_t, w_t, state, G)
+
+
+def rope(y, cs, dh, n_rot, transpose=False):
+    return default().rope(y, cs, dh, n_rot, transpose)
+
+
+def fwd_lowrank_rope(x, z, U, cs, G, W, dh, n_rot):
+    return default().fwd_lowrank_rope(x, z, U, cs, G, W, dh, n_rot)
+
+
+def bwd_lowrank_rope(x, z, U, cs, dy_rot, G, W, dh, n_rot):
+    return default().bwd_lowrank_rope(x, z, U, cs, dy_rot, G, W, dh, n_rot)
 
 
 def decode_lowrank(x_t, z_t, U, state, G, W):

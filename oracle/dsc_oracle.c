@@ -275,3 +275,35 @@ int oracle_decode_lowrank(const double *x_t, const double *z_t, const double *U,
     free(wt);
     return 0;
 }
+
+/* Rotary position embedding of the first n_rot channels of y, in place.
+ *
+ * "Metodologia > Convolucoes Curtas Dinamicas > Posicionamento": the convolution is
+ * applied to the Q, K and V projections before RoPE, so the op's output on the Q and K
+ * channels is rotated next.  Reading: RoPE in its original form, pairs of adjacent
+ * channels (2i, 2i+1) of each head of dh channels rotated by the angle of pair i at
+ * the token's position t in its sequence, whose cosine and sine are given:
+ *   y'[2i]   = y[2i] cos - y[2i+1] sin
+ *   y'[2i+1] = y[2i] sin + y[2i+1] cos
+ * Channels n_rot..D-1 (V) are not rotated.  transpose != 0 applies the inverse
+ * rotation (angle -theta), which is the transpose the backward needs.
+ *   y  : [B, T, D]
+ *   cs : [T, dh/2, 2]   (cos, sin) per position and pair
+ * Requires dh even and n_rot a multiple of dh, n_rot <= D. */
+void oracle_rope(double *y, const double *cs, int B, int T, int D, int dh, int n_rot, int transpose)
+{
+    const int np = dh / 2;
+    for (int b = 0; b < B; ++b)
+        for (int t = 0; t < T; ++t) {
+            double *row = y + ((size_t)b * T + t) * D;
+            for (int c0 = 0; c0 < n_rot; c0 += dh)
+                for (int i = 0; i < np; ++i) {
+                    const double co = cs[((size_t)t * np + i) * 2 + 0];
+                    const double si = transpose ? -cs[((size_t)t * np + i) * 2 + 1]
+                                                : cs[((size_t)t * np + i) * 2 + 1];
+                    const double a = row[c0 + 2 * i], e = row[c0 + 2 * i + 1];
+                    row[c0 + 2 * i] = a * co - e * si;
+                    row[c0 + 2 * i + 1] = a * si + e * co;
+                }
+        }
+}

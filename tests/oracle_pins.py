@@ -25,6 +25,12 @@ gist.science/pt/paper/2606.03825, "Metodologia > Convolucoes Curtas Dinamicas"):
                      Jacobian; y is linear in each argument separately, so central
                      differences are exact up to rounding.
   * invariant     -- sum(dU*U) == sum(dz*z) (both equal sum_t <dw_t, w_t>).
+  * rope          -- the op sits before RoPE on the Q and K projections
+                     ("Posicionamento"); RoPE (original form: adjacent channel pairs
+                     of each head rotated by their angle) is checked against numpy's
+                     complex multiplication, its transpose against the inverse and
+                     the adjoint identity, and the fused backward against central
+                     differences of the rotated forward.
   * decode        -- one decode step (a token with its W-1 predecessors held in a
                      rolling window; "Significancia e Alegacoes" notes that inference
                      still needs engineering) is the forward at the last position of
@@ -364,6 +370,58 @@ def pin_decode_steps_match_forward(orc):
         _close(s_lr, pad[:, -(W - 1):] if W > 1 else pad[:, :0], 0, "window after step %d" % t)
 
 
+# ---------------------------------------------------------------- RoPE after the op
+def _angles(r, T, dh):
+    th = r.uniform(-np.pi, np.pi, size=(T, dh // 2))
+    return th, np.stack([np.cos(th), np.sin(th)], axis=-1)
+
+
+def pin_rope_complex(orc):
+    """Pair (2i, 2i+1) of each rotated head, read as the complex number y_2i + i y_2i+1,
+    is multiplied by exp(i theta_{t,i}); channels past n_rot are untouched."""
+    r = _rng(31)
+    for (D, dh, n_rot) in ((12, 4, 8), (16, 8, 16), (6, 2, 0)):
+        B, T = 2, 5
+        y = r.standard_normal((B, T, D))
+        th, cs = _angles(r, T, dh)
+        got = orc.rope(y, cs, dh, n_rot)
+        for c0 in range(0, n_rot, dh):
+            zc = y[:, :, c0:c0 + dh:2] + 1j * y[:, :, c0 + 1:c0 + dh:2]
+            ref = zc * np.exp(1j * th)[None]
+            _close(got[:, :, c0:c0 + dh:2], ref.real, 1e-14, "rope real part")
+            _close(got[:, :, c0 + 1:c0 + dh:2], ref.imag, 1e-14, "rope imaginary part")
+        assert np.array_equal(got[:, :, n_rot:], y[:, :, n_rot:]), "rope touched channels past n_rot"
+
+
+def pin_rope_transpose(orc):
+    """The transpose undoes the rotation and satisfies <R a, b> = <a, R^T b>."""
+    r = _rng(32)
+    B, T, D, dh, n_rot = 2, 6, 16, 8, 8
+    a = r.standard_normal((B, T, D))
+    b = r.standard_normal((B, T, D))
+    _, cs = _angles(r, T, dh)
+    _close(orc.rope(orc.rope(a, cs, dh, n_rot), cs, dh, n_rot, transpose=True), a, 1e-14, "rope^T rope")
+    lhs = float(np.sum(orc.rope(a, cs, dh, n_rot) * b))
+    rhs = float(np.sum(a * orc.rope(b, cs, dh, n_rot, transpose=True)))
+    assert abs(lhs - rhs) <= 1e-12 * max(1.0, abs(lhs)), "rope adjoint %.6e vs %.6e" % (lhs, rhs)
+
+
+def pin_fd_lowrank_rope(orc):
+    """The fused backward (bwd_lowrank of the un-rotated gradient) is the gradient of
+    <dy_rot, RoPE(fwd_lowrank)>, by central differences (linear in x, z and U)."""
+    r = _rng(33)
+    B, T, D, G, W, R, dh, n_rot = 2, 5, 8, 2, 3, 2, 4, 4
+    N = (D // G) * W
+    x = r.standard_normal((B, T, D))
+    z = r.standard_normal((B, T, R))
+    U = r.standard_normal((R, N))
+    dy = r.standard_normal((B, T, D))
+    _, cs = _angles(r, T, dh)
+    loss = lambda: float(np.sum(dy * orc.fwd_lowrank_rope(x, z, U, cs, G, W, dh, n_rot)))
+    dx, dz, dU = orc.bwd_lowrank_rope(x, z, U, cs, dy, G, W, dh, n_rot)
+    _fd_check(loss, {"x": x, "z": z, "U": U}, {"x": dx, "z": dz, "U": dU}, "lowrank + rope")
+
+
 PINS = [
     pin_hand_example,
     pin_identity_filter_doubles,
@@ -380,4 +438,7 @@ PINS = [
     pin_adjoint_and_invariant,
     pin_decode_is_forward_at_last_position,
     pin_decode_steps_match_forward,
+    pin_rope_complex,
+    pin_rope_transpose,
+    pin_fd_lowrank_rope,
 ]

@@ -44,6 +44,15 @@ MUTANTS = [
     ("decode drops the residual",
      "double acc = x_t[c];\n        acc += wt[g * W + 0] * x_t[c];",
      "double acc = 0.0;\n        acc += wt[g * W + 0] * x_t[c];"),
+    ("rope rotates the other way",
+     "row[c0 + 2 * i] = a * co - e * si;\n                    row[c0 + 2 * i + 1] = a * si + e * co;",
+     "row[c0 + 2 * i] = a * co + e * si;\n                    row[c0 + 2 * i + 1] = -a * si + e * co;"),
+    ("rope pairs channel i with i + dh/2",
+     "const double a = row[c0 + 2 * i], e = row[c0 + 2 * i + 1];\n                    row[c0 + 2 * i] = a * co - e * si;\n                    row[c0 + 2 * i + 1] = a * si + e * co;",
+     "const double a = row[c0 + i], e = row[c0 + np + i];\n                    row[c0 + i] = a * co - e * si;\n                    row[c0 + np + i] = a * si + e * co;"),
+    ("rope transpose ignored",
+     "const double si = transpose ? -cs[((size_t)t * np + i) * 2 + 1]",
+     "const double si = transpose ? cs[((size_t)t * np + i) * 2 + 1]"),
     ("explicit dw misses the group sum (last channel wins)",
      "dw[(bt * NG + g) * W + k] += gy * x[(bt - k) * D + c];",
      "dw[(bt * NG + g) * W + k] = gy * x[(bt - k) * D + c];"),
