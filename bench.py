@@ -353,8 +353,9 @@ def _time_graph(fn, dev, n):
 def measure_comparators(dsc, dev, peak, args):
     """Other paths timed in the same run, each on its own workload: the in-repo static
     depthwise causal convolution (the primitive the method generalises) on the MLP-width
-    shape, the explicit-filter forward on the stacked-QKV shape, and the fused low-rank
-    step on the MLP-width shape.  Inputs exceed L2; times are CUDA events per call."""
+    shape, the fused low-rank step on the MLP-width shape, the stacked-QKV step with RoPE
+    fused, the explicit-filter forward on the stacked-QKV shape, and the decode step.
+    Inputs exceed L2; times are CUDA events per call."""
     stream = torch.cuda.current_stream(dev)
     steps = max(3, min(args.steps, 10))
     out = {}
@@ -400,6 +401,31 @@ def measure_comparators(dsc, dev, peak, args):
         "fwd_bwd": entry(fwd_ms + bwd_ms, fb + bb, wl.tokens),
         "path": dsc.dsc_lowrank_path(wl.B, wl.T, wl.D, wl.G, wl.W, wl.R)}
     del t, x, z, U, dy, y, dx, dz, dU, ws
+
+    # the stacked-QKV step with RoPE fused on Q and K (heads of 128 channels): the op's
+    # output rotated before it is stored, and the backward from the rotated gradient
+    wl = di.WORKLOADS["lowrank_qkv"]
+    t = di.make(wl, dev, ("x", "z", "U", "dy"))
+    x, z, U, dy = t["x"], t["z"], t["U"], t["dy"]
+    dh, n_rot = 128, 2 * wl.D // 3
+    inv = 10000.0 ** (-torch.arange(0, dh, 2, dtype=torch.float64, device=dev) / dh)
+    th = torch.arange(wl.T, dtype=torch.float64, device=dev)[:, None] * inv[None, :]
+    cs = torch.stack([torch.cos(th), torch.sin(th)], dim=-1).to(torch.float32).permute(1, 0, 2).contiguous()
+    y = torch.empty_like(x)
+    dx = torch.empty_like(x)
+    dz = torch.empty((wl.B, wl.T, wl.R), dtype=torch.float32, device=dev)
+    dU = torch.empty((wl.R, wl.N), dtype=torch.float32, device=dev)
+    ws = dsc.workspace(dsc.dsc_bwd_lowrank_workspace_bytes(wl.B, wl.T, wl.D, wl.G, wl.W, wl.R), dev)
+    fwd_ms = _time_calls(lambda: dsc.dsc_fwd_lowrank_rope(x, z, U, cs, y, wl.G, wl.W, dh, n_rot), stream, steps)
+    bwd_ms = _time_calls(lambda: dsc.dsc_bwd_lowrank_rope(x, z, U, cs, dy, dx, dz, dU, ws, wl.G, wl.W, dh, n_rot),
+                         stream, steps)
+    fb, bb = algorithmic_bytes(wl)
+    out["lowrank_rope_" + wl.name.split("_", 1)[1]] = {
+        "shape": {"B": wl.B, "T": wl.T, "D": wl.D, "G": wl.G, "W": wl.W, "R": wl.R, "dh": dh, "n_rot": n_rot},
+        "fwd": entry(fwd_ms, fb, wl.tokens), "bwd": entry(bwd_ms, bb, wl.tokens),
+        "fwd_bwd": entry(fwd_ms + bwd_ms, fb + bb, wl.tokens),
+        "note": "bytes exclude the 0.5 MB RoPE table; a separate rotation pass would add 4 x 134 MB"}
+    del t, x, z, U, dy, y, dx, dz, dU, ws, cs
 
     # explicit-filter forward on the stacked-QKV shape
     wl = di.WORKLOADS["tied_qkv"]

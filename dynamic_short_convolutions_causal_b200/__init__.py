@@ -22,6 +22,7 @@ __all__ = [
     "dsc_bwd_lowrank_workspace_bytes", "dsc_bwd", "dsc_static_fwd", "dsc_static_bwd",
     "dsc_static_bwd_workspace_bytes", "dsc_static_bwd_noalloc", "dsc_lowrank_path",
     "dsc_decode_step", "dsc_decode_step_lowrank", "dsc_fwd_lowrank_halo", "dsc_bwd_lowrank_halo",
+    "dsc_fwd_lowrank_rope", "dsc_bwd_lowrank_rope",
     "DSC_F32", "DSC_BF16",
 ]
 
@@ -61,6 +62,8 @@ def _load():
         "dsc_decode_step_lowrank": (i, [vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]),
         "dsc_fwd_lowrank_halo": (i, [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]),
         "dsc_bwd_lowrank_halo": (i, [vp, vp, vp, vp, vp, vp, vp, fp, fp, i, i, i, i, i, i, i, vp]),
+        "dsc_fwd_lowrank_rope": (i, [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, vp]),
+        "dsc_bwd_lowrank_rope": (i, [vp, vp, vp, vp, vp, vp, fp, fp, vp, sz, i, i, i, i, i, i, i, i, i, vp]),
         "dsc_device_fault": (ctypes.c_uint, [i]),
         "dsc_test_arm_wait_timeout": (None, [ctypes.c_uint]),
         "dsc_status_string": (ctypes.c_char_p, [i]),
@@ -251,6 +254,36 @@ def dsc_bwd_lowrank_halo(x_prev, z, U, dy, dy_next, z_next, dx, dz, dU, G: int, 
     with torch.cuda.device(dy.device):
         _check(lib.dsc_bwd_lowrank_halo(_ptr(x_prev), _ptr(z), _ptr(U), _ptr(dy), _ptr(dy_next), _ptr(z_next),
                                         _ptr(dx), _ptr(dz), _ptr(dU), B, T, D, G, W, R, _dt(dy), _stream(dy)))
+    return dx, dz, dU
+
+
+def dsc_fwd_lowrank_rope(x, z, U, cs, y, G: int, W: int, dh: int, n_rot: int):
+    """dsc_fwd_lowrank followed by RoPE of the first n_rot channels of y (heads of dh,
+    adjacent pairs); cs fp32 [dh/2, T, 2] holds (cos, sin) per pair and position."""
+    B, T, D = x.shape
+    R = z.shape[-1]
+    _same(x, z, U, y, cs)
+    if cs.dtype != torch.float32:
+        raise TypeError("dsc_fwd_lowrank_rope: cs must be fp32")
+    with torch.cuda.device(x.device):
+        _check(lib.dsc_fwd_lowrank_rope(_ptr(x), _ptr(z), _ptr(U), _ptr(cs), _ptr(y), B, T, D, G, W, R, dh, n_rot,
+                                        _dt(x), _stream(x)))
+    return y
+
+
+def dsc_bwd_lowrank_rope(x, z, U, cs, dy_rot, dx, dz, dU, workspace, G: int, W: int, dh: int, n_rot: int):
+    """Backward of dsc_fwd_lowrank_rope given dy_rot, the gradient of the rotated output;
+    same outputs and workspace as dsc_bwd_lowrank."""
+    B, T, D = x.shape
+    R = z.shape[-1]
+    _same(x, z, U, cs, dy_rot, dx, dz, dU)
+    if dz.dtype != torch.float32 or dU.dtype != torch.float32 or cs.dtype != torch.float32:
+        raise TypeError("dsc_bwd_lowrank_rope: dz, dU and cs must be fp32")
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    with torch.cuda.device(x.device):
+        _check(lib.dsc_bwd_lowrank_rope(_ptr(x), _ptr(z), _ptr(U), _ptr(cs), _ptr(dy_rot), _ptr(dx), _ptr(dz),
+                                        _ptr(dU), _ptr(workspace), ws_bytes, B, T, D, G, W, R, dh, n_rot, _dt(x),
+                                        _stream(x)))
     return dx, dz, dU
 
 

@@ -245,6 +245,64 @@ DSC_API dsc_status_t dsc_decode_step_lowrank(const void *x_t, const void *z_t, c
                                                        (cudaStream_t)stream));
 }
 
+namespace {
+dsc_status_t check_rope(const char *fn, const float *cs, int D, int dh, int n_rot, bool on_tc) {
+    if (dh < 16 || dh % 16 || n_rot < 0 || n_rot > D || (n_rot % dh))
+        return fail(DSC_ERR_INVALID_ARG, "%s: dh=%d must be a positive multiple of 16 and n_rot=%d a multiple of dh "
+                    "within [0, D=%d]", fn, dh, n_rot, D);
+    if (n_rot > 0) {
+        const void *p[] = {cs};
+        const char *n[] = {"cs"};
+        dsc_status_t st = check_ptrs(fn, p, n, 1);
+        if (st != DSC_OK) return st;
+    }
+    if (!on_tc)
+        return fail(DSC_ERR_UNSUPPORTED, "%s: these sizes are not on the tensor-core path (dsc_lowrank_path)", fn);
+    return DSC_OK;
+}
+}  // namespace
+
+DSC_API dsc_status_t dsc_fwd_lowrank_rope(const void *x, const void *z, const void *U, const float *cs, void *y,
+                                          int B, int T, int D, int G, int W, int R, int dh, int n_rot,
+                                          dsc_dtype_t dt, dsc_stream_t stream) {
+    const char *fn = "dsc_fwd_lowrank_rope";
+    dsc_status_t st = check_dims(fn, Dims{B, T, D, G, W, R}, dt);
+    if (st != DSC_OK) return st;
+    const void *p[] = {x, z, U, y};
+    const char *n[] = {"x", "z", "U", "y"};
+    if ((st = check_ptrs(fn, p, n, 4)) != DSC_OK) return st;
+    const bool bf16 = dt == DSC_BF16;
+    if ((st = check_rope(fn, cs, D, dh, n_rot, dsc::tc_lowrank_fwd_supported(B, T, D, G, W, R, bf16))) != DSC_OK)
+        return st;
+    return check_launch(fn, dsc::launch_tc_lowrank_fwd(x, z, U, y, B, T, D, G, W, R, (cudaStream_t)stream,
+                                                       n_rot > 0 ? cs : nullptr, dh, n_rot));
+}
+
+DSC_API dsc_status_t dsc_bwd_lowrank_rope(const void *x, const void *z, const void *U, const float *cs,
+                                          const void *dy_rot, void *dx, float *dz, float *dU, void *workspace,
+                                          size_t workspace_bytes, int B, int T, int D, int G, int W, int R, int dh,
+                                          int n_rot, dsc_dtype_t dt, dsc_stream_t stream) {
+    const char *fn = "dsc_bwd_lowrank_rope";
+    const Dims d{B, T, D, G, W, R};
+    dsc_status_t st = check_dims(fn, d, dt);
+    if (st != DSC_OK) return st;
+    const void *p[] = {x, z, U, dy_rot, dx, dz, dU};
+    const char *n[] = {"x", "z", "U", "dy_rot", "dx", "dz", "dU"};
+    if ((st = check_ptrs(fn, p, n, 7)) != DSC_OK) return st;
+    const bool bf16 = dt == DSC_BF16;
+    if ((st = check_rope(fn, cs, D, dh, n_rot, dsc::tc_lowrank_bwd_supported(B, T, D, G, W, R, bf16))) != DSC_OK)
+        return st;
+    const size_t need = lowrank_ws(d, bf16);
+    if (workspace_bytes < need)
+        return fail(DSC_ERR_UNSUPPORTED, "%s: workspace of %zu bytes is below the %zu required", fn, workspace_bytes,
+                    need);
+    const void *wp[] = {workspace};
+    const char *wn[] = {"workspace"};
+    if ((st = check_ptrs(fn, wp, wn, 1)) != DSC_OK) return st;
+    return check_launch(fn, dsc::launch_tc_lowrank_bwd(x, z, U, dy_rot, dx, dz, dU, workspace, B, T, D, G, W, R,
+                                                       (cudaStream_t)stream, n_rot > 0 ? cs : nullptr, dh, n_rot));
+}
+
 DSC_API dsc_status_t dsc_fwd_lowrank_halo(const void *x, const void *z, const void *U, const void *x_prev,
                                           void *y, int B, int T, int D, int G, int W, int R, dsc_dtype_t dt,
                                           dsc_stream_t stream) {

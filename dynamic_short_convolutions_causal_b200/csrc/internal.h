@@ -53,11 +53,15 @@ bool tc_lowrank_fwd_supported(int B, int T, int D, int G, int W, int R, bool bf1
 bool tc_lowrank_bwd_supported(int B, int T, int D, int G, int W, int R, bool bf16);
 unsigned read_device_fault(bool reset);
 unsigned read_device_fault_bwd(bool reset);
+// cs: RoPE table [T][dh/2][2] (cos, sin) applied to channels [0, n_rot) of y, or null
 cudaError_t launch_tc_lowrank_fwd(const void *x, const void *z, const void *U, void *y, int B,
-                                  int T, int D, int G, int W, int R, cudaStream_t s);
+                                  int T, int D, int G, int W, int R, cudaStream_t s,
+                                  const float *cs = nullptr, int dh = 0, int n_rot = 0);
 size_t tc_lowrank_bwd_workspace(int B, int T, int D, int G, int W, int R);
+// cs: RoPE table [T][dh/2][2]; dy is then the gradient of the rotated output
 cudaError_t launch_tc_lowrank_bwd(const void *x, const void *z, const void *U, const void *dy,
                                   void *dx, float *dz, float *dU, void *ws, int B, int T, int D,
-                                  int G, int W, int R, cudaStream_t s);
+                                  int G, int W, int R, cudaStream_t s,
+                                  const float *cs = nullptr, int dh = 0, int n_rot = 0);
 
 }  // namespace dsc

@@ -92,6 +92,8 @@ struct BwdParams {
     uint32_t tm_w, tm_dz, tm_du, tmem_cols;   // TMEM column map
     float *du_part;           // [A][R][N]
     unsigned *flag_du;        // [Bg]   dU partials written per slice group (16 per CTA)
+    const float *cs;          // RoPE table [T][dh/2][2] (cos, sin): dy arrives rotated, or null
+    int dh, n_rot;            // RoPE head size; channels [0, n_rot) rotated (0: none)
     float *dz;                // [B*T][R]
     float *dU;                // [R][N]
     WaitTest wt;
@@ -114,8 +116,9 @@ struct Bars {
     __device__ uint32_t dufull() const { return base + 8 * 22; }
     __device__ uint32_t done() const { return base + 8 * 23; }
     __device__ uint32_t xdead() const { return base + 8 * 24; }
+    __device__ uint32_t dyrot() const { return base + 8 * 25; }
 };
-constexpr uint32_t kBarBytes = 8 * 25;
+constexpr uint32_t kBarBytes = 8 * 26;
 
 __device__ __forceinline__ void unpack8(const uint4 &u, float (&v)[8]) {
     v[0] = bf16_lo(u.x); v[1] = bf16_hi(u.x);
@@ -281,6 +284,7 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
         mbar_init(bar.dufull(), 1);
         mbar_init(bar.done(), 2);               // recompute and dz/dU streams
         mbar_init(bar.xdead(), kEpiWarps);      // every epilogue warp is past A2
+        mbar_init(bar.dyrot(), kEpiWarps);      // every epilogue warp has un-rotated its dy rows
         *abort = 0;
         fence_barrier_init();
     }
@@ -498,11 +502,57 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
 
         bool ok = true;
         int pb = 0, pt0 = 0;                 // sequence and first token of the previous token tile
+        int nrot = 0;                        // dyrot phases waited for
         for (Walk w(sp.m0, p.tiles_per_seq); w.i < nt; w.next(S, NST, p.tiles_per_seq)) {
             const int i = w.i, j = w.j, mz = w.mz;
             const int st = w.st, n = w.n;
             if (!warp_wait(bar.full(st), n & 1, abort, 64u, &g_fault_bwd, p.wt.wait_ns)) { ok = false; break; }
             const uint32_t dys = sb + st * p.stage_bytes, xs = dys + p.xy_tile_bytes;
+
+            // ---- RoPE (when on): dy arrives as the gradient of the rotated output; each
+            // thread rotates its own row of the stage's dy tile back in place (the
+            // transpose: pair (2i, 2i+1) by minus its angle), lanes 0..W-2 of quarter 0
+            // also the tile's W-1 future-halo rows.  A2 reads only its own row; A1 reads
+            // neighbours' rows and waits for every warp (dyrot) first.
+            const int cslice = (sp.s0 + j) * kDt;
+            const bool rope = p.n_rot > 0 && cslice < p.n_rot;
+            if (rope) {
+                const int c16 = cslice + kCPW * h;
+                if (c16 < p.n_rot) {
+                    auto unrotate = [&](int r) {
+                        const int tok = w.t0() + r;
+                        if (tok >= p.T) return;     // zero rows past the sequence's end
+                        // pair-major table: a warp's 32 rows read 256 contiguous bytes per pair
+                        const float2 *csp = reinterpret_cast<const float2 *>(p.cs) + (size_t)((c16 % p.dh) / 2) * p.T + tok;
+                        const uint32_t ra = (uint32_t)r * 128u ^ (((uint32_t)r & 7u) << 4) ^ ((uint32_t)(CH * h) << 4);
+                        float2 c[CH * 4];           // every load issued before the first use
+#pragma unroll
+                        for (int m2 = 0; m2 < CH * 4; ++m2) c[m2] = __ldg(csp + (size_t)m2 * p.T);
+                        uint4 u[CH];
+#pragma unroll
+                        for (int cq = 0; cq < CH; ++cq) u[cq] = lds128(dys + (ra ^ ((uint32_t)cq << 4)));
+#pragma unroll
+                        for (int cq = 0; cq < CH; ++cq) {
+                            float v[8];
+                            unpack8(u[cq], v);
+#pragma unroll
+                            for (int m2 = 0; m2 < 4; ++m2) {
+                                const float e0 = v[2 * m2], e1 = v[2 * m2 + 1];
+                                const float2 cc = c[4 * cq + m2];
+                                v[2 * m2] = fmaf(e0, cc.x, e1 * cc.y);
+                                v[2 * m2 + 1] = fmaf(e1, cc.x, -e0 * cc.y);
+                            }
+                            sts128(dys + (ra ^ ((uint32_t)cq << 4)),
+                                   make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                              pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7])));
+                        }
+                    };
+                    unrotate(row);
+                    if (q == 0 && lane < W - 1) unrotate(kTt + lane);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar.dyrot());
+            }
 
             // ---- A2: dw[t,g,k] = sum_{c in g} dy[t,c] x[t-k,c], tap-major column k*NG + g.
             // When they fit in registers the values of both chunks are computed before
@@ -613,6 +663,7 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             }
 
             // ---- A1: dx[t,c] = dy[t,c] + sum_k w[t+k,g,k] dy[t+k,c]
+            if (rope && !warp_wait(bar.dyrot(), (nrot++) & 1, abort, 8192u, &g_fault_bwd, p.wt.wait_ns)) { ok = false; break; }
             if (!warp_wait(bar.wfull(), i & 1, abort, 128u, &g_fault_bwd, p.wt.wait_ns)) { ok = false; break; }
             tc_fence_after();
             constexpr int NGB = NG8;                        // (virtual) groups of one chunk
@@ -1061,10 +1112,13 @@ size_t tc_lowrank_bwd_workspace(int B, int T, int D, int G, int W, int R) {
 
 cudaError_t launch_tc_lowrank_bwd(const void *x, const void *z, const void *U, const void *dy, void *dx,
                                   float *dz, float *dU, void *ws, int B, int T, int D, int G, int W, int R,
-                                  cudaStream_t s) {
+                                  cudaStream_t s, const float *cs, int dh, int n_rot) {
     using namespace tcb;
     BwdParams p;
     if (!plan_bwd(B, T, D, G, W, R, num_sms(), p)) return cudaErrorNotSupported;
+    p.cs = cs;
+    p.dh = dh;
+    p.n_rot = cs ? n_rot : 0;
     take_wait_test(&p.wt.wait_ns, &p.wt.withhold_cta);
     const WsLayout l = ws_layout(p);
     uint8_t *w8 = (uint8_t *)ws;

@@ -73,6 +73,8 @@ struct FwdParams {
     uint32_t off_x, off_op, off_y, off_bar;   // ring bases
     uint32_t off_z, off_u;    // within an operand stage
     uint32_t z_layout;        // swizzle of the z tile (32/64/128-byte rows)
+    const float *cs;          // RoPE table [T][dh/2][2] (cos, sin), or null
+    int dh, n_rot;            // RoPE head size; channels [0, n_rot) rotated (0: none)
     WaitTest wt;
 };
 
@@ -162,7 +164,7 @@ __device__ __forceinline__ void conv_chunk(const uint32_t *wr, const uint4 (&xu)
     }
 }
 
-template <int W, int GC>
+template <int W, int GC, bool ROPE>
 __global__ void __launch_bounds__(EpiShape<W, GC>::THREADS, 1)
 k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z,
                  const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_y,
@@ -350,15 +352,37 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
                 }
             };
             issue_taps(0, wr[0]);
+            // RoPE (when on): channel pairs (2i, 2i+1) of the first n_rot channels rotated by
+            // the angle of pair i = (c mod dh) / 2 at this row's position in its sequence
+            const int c_warp = slice * kDt + ES::CPW * h;
+            const bool rot_row = ROPE && t0 + row < p.T;
 #pragma unroll
             for (int cq = 0; cq < ES::CHUNKS; ++cq) {
                 uint4 xu[W];
 #pragma unroll
                 for (int k = 0; k < W; ++k) xu[k] = lds128(xs + (xrow[k] ^ ((uint32_t)cq << 4)));
+                float2 csv[4];
+                const int c8 = c_warp + 8 * cq;
+                const bool rot = rot_row && c8 < p.n_rot;
+                if (rot) {      // the chunk's 4 pairs, read ahead of the math; the table is
+                                // pair-major, so a warp's 32 rows read 256 contiguous bytes
+                    const float2 *src = reinterpret_cast<const float2 *>(p.cs) +
+                                        (size_t)((c8 % p.dh) / 2) * p.T + (t0 + row);
+#pragma unroll
+                    for (int m2 = 0; m2 < 4; ++m2) csv[m2] = __ldg(src + (size_t)m2 * p.T);
+                }
                 tmem_wait_ld_regs(wr[cq & 1]);
                 if (cq + 1 < ES::CHUNKS) issue_taps(cq + 1, wr[(cq + 1) & 1]);   // overlaps the math below
                 float out[8];
                 conv_chunk<W, GC>(wr[cq & 1], xu, out);
+                if (rot) {
+#pragma unroll
+                    for (int m2 = 0; m2 < 4; ++m2) {
+                        const float a = out[2 * m2], e = out[2 * m2 + 1];
+                        out[2 * m2] = fmaf(a, csv[m2].x, -e * csv[m2].y);
+                        out[2 * m2 + 1] = fmaf(a, csv[m2].y, e * csv[m2].x);
+                    }
+                }
                 uint4 o;
                 o.x = pack_bf16x2(out[0], out[1]);
                 o.y = pack_bf16x2(out[2], out[3]);
@@ -509,7 +533,7 @@ uint32_t smem_bytes(const FwdParams &p) { return p.off_bar + kBarBytes + 16 + 10
 template <int W, int GC>
 cudaError_t launch_fwd_t(const CUtensorMap &mx, const CUtensorMap &mz, const CUtensorMap &mu,
                          const CUtensorMap &my, const FwdParams &p, cudaStream_t s) {
-    auto kern = k_tc_lowrank_fwd<W, GC>;
+    auto kern = p.n_rot > 0 ? k_tc_lowrank_fwd<W, GC, true> : k_tc_lowrank_fwd<W, GC, false>;
     using ES = EpiShape<W, GC>;
     if (p.nwg != ES::SETS || p.y_buf_bytes != (uint32_t)ES::YBUF) return cudaErrorInvalidConfiguration;
     const uint32_t smem = smem_bytes(p);
@@ -541,10 +565,13 @@ bool tc_lowrank_fwd_supported(int B, int T, int D, int G, int W, int R, bool bf1
 }
 
 cudaError_t launch_tc_lowrank_fwd(const void *x, const void *z, const void *U, void *y, int B, int T,
-                                  int D, int G, int W, int R, cudaStream_t s) {
+                                  int D, int G, int W, int R, cudaStream_t s, const float *cs, int dh, int n_rot) {
     using namespace tc;
     FwdParams p;
     if (!plan_fwd(B, T, D, G, W, R, p)) return cudaErrorNotSupported;
+    p.cs = cs;
+    p.dh = dh;
+    p.n_rot = cs ? n_rot : 0;
     take_wait_test(&p.wt.wait_ns, &p.wt.withhold_cta);
     CUtensorMap mx, mz, mu, my;
     const uint64_t dx[3] = {(uint64_t)D, (uint64_t)T, (uint64_t)B};

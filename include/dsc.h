@@ -184,6 +184,34 @@ DSC_API dsc_status_t dsc_decode_step_lowrank(const void *x_t, const void *z_t, c
                                              int B, int D, int G, int W, int R,
                                              dsc_dtype_t dt, dsc_stream_t stream);
 
+/* The low-rank op followed by rotary position embedding (RoPE) of its output, fused:
+ * the convolution sits on the Q, K and V projections before RoPE ("Metodologia >
+ * Convolucoes Curtas Dinamicas > Posicionamento"), so with the projections stacked as
+ * [Q | K | V] along D the first n_rot channels (Q and K) of y = x + conv(x) are rotated
+ * before y is stored, and the backward takes the gradient of the rotated output.
+ * RoPE in its original form: within each head of dh channels, channel pair (2i, 2i+1)
+ * of token t (its position in the sequence) is rotated by the angle of pair i,
+ *   y'[2i] = y[2i] cos - y[2i+1] sin,   y'[2i+1] = y[2i] sin + y[2i+1] cos,
+ * with (cos, sin) read from the caller's table cs.
+ *   cs     fp32 [dh/2, T, 2], 16-byte aligned: (cos, sin) of pair i at position t is
+ *          cs[(i*T + t)*2 + 0..1] (pair-major, so that a warp's consecutive tokens read
+ *          contiguous bytes)
+ *   dh     head size, a multiple of 16;  n_rot a multiple of dh, 0 <= n_rot <= D
+ *   dsc_fwd_lowrank_rope: as dsc_fwd_lowrank, y rotated on its first n_rot channels;
+ *   dsc_bwd_lowrank_rope: as dsc_bwd_lowrank with dy_rot the gradient of the rotated
+ *     output: dy = RoPE^T(dy_rot) is formed in shared memory (rounded to the element
+ *     type once) and never written to HBM; same workspace as dsc_bwd_lowrank.
+ * Only sizes on the tensor-core path (dsc_lowrank_path() == 3) are taken; others get
+ * DSC_ERR_UNSUPPORTED.  n_rot = 0 is the plain op. */
+DSC_API dsc_status_t dsc_fwd_lowrank_rope(const void *x, const void *z, const void *U, const float *cs,
+                                          void *y, int B, int T, int D, int G, int W, int R,
+                                          int dh, int n_rot, dsc_dtype_t dt, dsc_stream_t stream);
+DSC_API dsc_status_t dsc_bwd_lowrank_rope(const void *x, const void *z, const void *U, const float *cs,
+                                          const void *dy_rot, void *dx, float *dz, float *dU,
+                                          void *workspace, size_t workspace_bytes,
+                                          int B, int T, int D, int G, int W, int R,
+                                          int dh, int n_rot, dsc_dtype_t dt, dsc_stream_t stream);
+
 /* Sequence sharding (a sequence of length P*T split into P consecutive shards of T
  * tokens, one per rank).  Each rank calls dsc_fwd_lowrank / dsc_bwd_lowrank on its own
  * shard, which treats the shard as a whole sequence, and then the matching halo call

@@ -131,3 +131,24 @@ def test_halo_validation(dsc):
     assert L.dsc_fwd_lowrank_halo(FAKE, FAKE, FAKE, FAKE, None, B, T, D, G, W, R, 1, None) == 1
     assert L.dsc_fwd_lowrank_halo(FAKE, FAKE, FAKE, ODD, FAKE, B, T, D, G, W, R, 1, None) == 2
     assert L.dsc_fwd_lowrank_halo(FAKE, FAKE, FAKE, FAKE, FAKE, B, T, D, G, 9, R, 1, None) == 2
+
+
+def test_rope_validation(dsc):
+    """RoPE head size, rotated range, table pointer and path are checked before any launch."""
+    L = dsc.lib
+    B, T, D, G, W, R = 2, 8, 128, 1, 4, 32
+    fwd = lambda cs, dh, n_rot, dt=1: L.dsc_fwd_lowrank_rope(FAKE, FAKE, FAKE, cs, FAKE, B, T, D, G, W, R, dh, n_rot,
+                                                             dt, None)
+    assert fwd(FAKE, 8, 64) == 1            # dh not a multiple of 16
+    assert fwd(FAKE, 64, 96) == 1           # n_rot not a multiple of dh
+    assert fwd(FAKE, 64, 192) == 1          # n_rot > D
+    assert fwd(None, 64, 64) == 1           # no table
+    assert fwd(ODD, 64, 64) == 2            # misaligned table
+    assert fwd(FAKE, 64, 64, dt=0) == 2     # fp32: not on the tensor-core path
+    need = L.dsc_bwd_lowrank_workspace_bytes(B, T, D, G, W, R, 1)
+    bwd = lambda ws_bytes: L.dsc_bwd_lowrank_rope(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, ws_bytes,
+                                                  B, T, D, G, W, R, 64, 64, 1, None)
+    if need:
+        assert bwd(need - 1) == 2
+    assert L.dsc_bwd_lowrank_rope(FAKE, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, FAKE, 1 << 40,
+                                  B, T, D, G, W, R, 64, 64, 1, None) == 1
