@@ -427,16 +427,20 @@ def measure_comparators(dsc, dev, peak, args):
         "note": "bytes exclude the 0.5 MB RoPE table; a separate rotation pass would add 4 x 134 MB"}
     del t, x, z, U, dy, y, dx, dz, dU, ws, cs
 
-    # explicit-filter forward on the stacked-QKV shape
+    # explicit-filter forward and backward on the stacked-QKV shape
     wl = di.WORKLOADS["tied_qkv"]
-    t = di.make(wl, dev, ("x", "w"))
-    x, w = t["x"], t["w"]
+    t = di.make(wl, dev, ("x", "w", "dy"))
+    x, w, dy = t["x"], t["w"], t["dy"]
     y = torch.empty_like(x)
     ms = _time_calls(lambda: dsc.dsc_fwd(x, w, y, wl.G), stream, steps)
     nb = 2 * wl.tokens * wl.D * 2 + wl.tokens * wl.NG * wl.W * 2
-    out["explicit_fwd_" + wl.name] = {"shape": {"B": wl.B, "T": wl.T, "D": wl.D, "G": wl.G, "W": wl.W},
-                                      "fwd": entry(ms, nb, wl.tokens)}
-    del t, x, w, y
+    dx = torch.empty_like(x)
+    dw = torch.empty((wl.B, wl.T, wl.NG, wl.W), dtype=torch.float32, device=dev)
+    ms_b = _time_calls(lambda: dsc.dsc_bwd(x, w, dy, dx, dw, wl.G), stream, steps)
+    nb_b = 3 * wl.tokens * wl.D * 2 + wl.tokens * wl.NG * wl.W * (2 + 4)   # x, dy, dx; w in, dw out (fp32)
+    out["explicit_" + wl.name] = {"shape": {"B": wl.B, "T": wl.T, "D": wl.D, "G": wl.G, "W": wl.W},
+                                  "fwd": entry(ms, nb, wl.tokens), "bwd": entry(ms_b, nb_b, wl.tokens)}
+    del t, x, w, dy, y, dx, dw
 
     # decode step (one token per sequence, rolling window) on the stacked-QKV width
     wl = di.WORKLOADS["lowrank_qkv"]

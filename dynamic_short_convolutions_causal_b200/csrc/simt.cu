@@ -121,6 +121,87 @@ k_conv_bwd_dx(const TW *__restrict__ w, const T *__restrict__ dy, T *__restrict_
     }
 }
 
+// ------------------------------------------------------------------ explicit dw, rows
+// dw[bt,g,k] = sum_{c in g, t-k >= 0} dy[bt,c] x[bt-k,c] with the channels along the
+// threads: a thread owns one 16-byte vector (V channels) and walks a chunk of tokens with
+// the W rows x[t-k] in registers, so each row of x and dy is read once, coalesced.  Its
+// V products per tap are summed in the thread (groups of at most V channels: V/G groups
+// per thread) or across the G/V threads of a group by a fixed xor-shuffle tree (G a
+// multiple of V, G/V <= 32, a power of two); one thread per group writes the W taps.
+template <typename T, int W>
+__global__ void __launch_bounds__(256)
+k_dyn_dw_rows(const T *__restrict__ x, const T *__restrict__ dy, float *__restrict__ dw,
+              int B, int T_, int D, int G, int chunk) {
+    constexpr int V = Vec<T>::N;
+    const int nv = D / V;
+    const int v = blockIdx.x * blockDim.x + threadIdx.x;
+    const bool active = v < nv;
+    const int nchunks = cdiv(T_, chunk);
+    const int b = blockIdx.y / nchunks;
+    const int t0 = (blockIdx.y % nchunks) * chunk;
+    const int t1 = min(t0 + chunk, T_);
+    const int c0 = (active ? v : 0) * V;
+    const int NG = D / G;
+    const int lanes = G > V ? G / V : 1;        // threads per group
+    const size_t row0 = (size_t)b * T_;
+    float xw[W][V];                             // xw[k] = x[t-k]
+#pragma unroll
+    for (int k = 1; k < W; ++k) {
+        if (active && t0 - k >= 0) Vec<T>::load(x + (row0 + t0 - k) * D + c0, xw[k]);
+        else
+#pragma unroll
+            for (int i = 0; i < V; ++i) xw[k][i] = 0.f;
+    }
+    for (int t = t0; t < t1; ++t) {
+        float g[V];
+        if (active) {
+            Vec<T>::load(x + (row0 + t) * D + c0, xw[0]);
+            Vec<T>::load(dy + (row0 + t) * D + c0, g);
+        } else {
+#pragma unroll
+            for (int i = 0; i < V; ++i) xw[0][i] = g[i] = 0.f;
+        }
+        float* out = dw + (row0 + t) * (size_t)NG * W;
+        if (G >= V) {
+            float s[W];
+#pragma unroll
+            for (int k = 0; k < W; ++k) {
+                float a = 0.f;
+#pragma unroll
+                for (int i = 0; i < V; ++i) a = fmaf(g[i], xw[k][i], a);
+                s[k] = a;
+            }
+            for (int o = 1; o < lanes; o <<= 1)
+#pragma unroll
+                for (int k = 0; k < W; ++k) s[k] += __shfl_xor_sync(0xffffffffu, s[k], o);
+            if (active && (v % lanes) == 0) {
+                float *q = out + (size_t)(c0 / G) * W;
+#pragma unroll
+                for (int k = 0; k < W; ++k) q[k] = s[k];
+            }
+        } else {
+            // V/G whole groups in the thread
+            for (int gl = 0; gl < V / G; ++gl) {
+                float s[W];
+#pragma unroll
+                for (int k = 0; k < W; ++k) s[k] = 0.f;
+                for (int e = gl * G; e < (gl + 1) * G; ++e)
+#pragma unroll
+                    for (int k = 0; k < W; ++k) s[k] = fmaf(g[e], xw[k][e], s[k]);
+                if (active) {
+                    float *q = out + (size_t)(c0 / G + gl) * W;
+#pragma unroll
+                    for (int k = 0; k < W; ++k) q[k] = s[k];
+                }
+            }
+        }
+#pragma unroll
+        for (int k = W - 1; k >= 1; --k)
+#pragma unroll
+            for (int i = 0; i < V; ++i) xw[k][i] = xw[k - 1][i];
+    }
+}
+
 // ------------------------------------------------------------------ explicit dw
 // dw[bt,g,k] = sum_{c in g, t-k >= 0} dy[bt,c] x[bt-k,c]; one thread per (bt, g).
 template <typename T>
@@ -296,8 +377,31 @@ void launch_conv_dx(const void *w, bool w_is_f32, const void *dy, void *dx, int 
     }
 }
 
+template <typename T>
+static bool launch_dw_rows(const void *x, const void *dy, float *dw, int B, int T_, int D, int G, int W,
+                           cudaStream_t s) {
+    constexpr int V = Vec<T>::N;
+    const bool ok = (G >= V) ? (G % V == 0 && (G / V) <= 32 && ((G / V) & (G / V - 1)) == 0) : (V % G == 0);
+    if (!ok) return false;
+    constexpr int kRowChunk = 64;
+    const dim3 grid(cdiv(D / V, 256), B * cdiv(T_, kRowChunk));
+    const T *xp = (const T *)x;
+    const T *gp = (const T *)dy;
+    switch (W) {
+#define DSC_CASE(WW) \
+    case WW: k_dyn_dw_rows<T, WW><<<grid, 256, 0, s>>>(xp, gp, dw, B, T_, D, G, kRowChunk); break;
+        DSC_CASE(1) DSC_CASE(2) DSC_CASE(3) DSC_CASE(4) DSC_CASE(5) DSC_CASE(6) DSC_CASE(7) DSC_CASE(8)
+#undef DSC_CASE
+    }
+    return true;
+}
+
 void launch_dyn_dw(const void *x, const void *dy, float *dw, int B, int T, int D, int G, int W,
                    bool bf16_, cudaStream_t s) {
+    // row-parallel kernel where the groups tile the threads' channel vectors; otherwise
+    // one thread per (token, group)
+    if (bf16_ ? launch_dw_rows<bf16>(x, dy, dw, B, T, D, G, W, s) : launch_dw_rows<float>(x, dy, dw, B, T, D, G, W, s))
+        return;
     const size_t n = (size_t)B * T * (D / G);
     const unsigned grid = (unsigned)std::min<size_t>((n + 255) / 256, 65535u * 8);
     if (bf16_) k_dyn_dw<bf16><<<grid, 256, 0, s>>>((const bf16 *)x, (const bf16 *)dy, dw, B, T, D, G, W);
