@@ -57,7 +57,10 @@ def read_peaks():
 
 
 class Clocks:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    """SM clocks and throttle reasons during the timed region: nvidia-smi (the recipe's
+    query, every 100 ms) and, since a timed region can be a few ms long, NVML read every
+    millisecond from a thread.  The GPU is named by its PCI bus id, so that the sampled
+    device is the one the CUDA device maps to whatever the visible-device numbering."""
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -67,6 +70,33 @@ class Clocks:
         self.index = index
         self.proc = None
         self.path = None
+        self.thread = None
+        self.nvml = []
+        try:
+            pr = torch.cuda.get_device_properties(index)
+            self.bus = "%08X:%02X:%02X.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
+        except Exception:
+            self.bus = None
+
+    def _poll(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            h = (pynvml.nvmlDeviceGetHandleByPciBusId(self.bus) if self.bus
+                 else pynvml.nvmlDeviceGetHandleByIndex(self.index))
+            bits = {"hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap}
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            while not self.stop_flag:
+                mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.nvml.append((mhz, sorted(k for k, v in bits.items() if r & v)))
+                time.sleep(0.001)
+            pynvml.nvmlShutdown()
+        except Exception:
+            pass
 
     def start(self):
         try:
@@ -75,38 +105,49 @@ class Clocks:
             os.close(fd)
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                ["nvidia-smi", "-i", self.bus or str(self.index), "--query-gpu=" + self.Q,
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=self.fh, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
+        import threading
+        self.stop_flag = False
+        self.max_mhz = None
+        self.thread = threading.Thread(target=self._poll, daemon=True)
+        self.thread.start()
 
     def stop(self):
-        if self.proc is None:
-            return None
-        time.sleep(0.15)
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.fh.close()
+        if self.thread is not None:
+            self.stop_flag = True
+            self.thread.join(timeout=5)
         rows = []
-        with open(self.path) as f:
-            for line in f:
-                parts = [s.strip() for s in line.split(",")]
-                if len(parts) >= 9:
-                    rows.append(parts)
-        os.unlink(self.path)
-        if not rows:
-            return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.fh.close()
+            with open(self.path) as f:
+                for line in f:
+                    parts = [s.strip() for s in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+            os.unlink(self.path)
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()] + [float(m) for m, _ in self.nvml]
         mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        if self.max_mhz:
+            mx.append(float(self.max_mhz))
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
-                "samples": len(rows)}
+        reasons = {names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"}
+        for _, rs in self.nvml:
+            reasons.update(rs)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(rows) + len(self.nvml),
+                "samples_nvidia_smi": len(rows), "samples_nvml": len(self.nvml), "gpu": self.bus}
 
 
 def dist_setup(args):
@@ -503,54 +544,99 @@ def load_traffic(kernel, wl):
 
 
 def measure_e2e(dsc, t, y, dx, dz, dU, ws, wl, world, dev, args):
+    """The step through the public binding with every input copied in from pinned host
+    memory (x, z, U, dy) and every output copied out (y, dx, dz, dU), each step.  Two
+    figures: `serial` (copies, compute and copies back one after another on one stream)
+    and the reported one, pipelined over two buffer sets: step i+1's inputs go in on a
+    copy stream and step i-1's outputs come out on another while step i computes, as a
+    training loop with a host data pipeline would run it.  Times are CUDA events; the
+    pipelined region starts before the first step's copies and ends after the last
+    step's outputs have landed."""
     G, W = wl.G, wl.W
-    hx = t["x"].cpu().pin_memory()
-    hz = t["z"].cpu().pin_memory()
-    hU = t["U"].cpu().pin_memory()
-    hdy = t["dy"].cpu().pin_memory()
-    hy = torch.empty_like(hx).pin_memory()
-    hdx = torch.empty_like(hx).pin_memory()
-    hdz = torch.empty(dz.shape, dtype=dz.dtype).pin_memory()
-    hdU = torch.empty(dU.shape, dtype=dU.dtype).pin_memory()
-    x = torch.empty_like(t["x"])
-    z = torch.empty_like(t["z"])
-    U = torch.empty_like(t["U"])
-    dy = torch.empty_like(t["dy"])
-    stream = torch.cuda.current_stream(dev)
-    h2d = sum(a.numel() * a.element_size() for a in (hx, hz, hU, hdy))
-    d2h = sum(a.numel() * a.element_size() for a in (hy, hdx, hdz, hdU))
+    hin = [t[k].cpu().pin_memory() for k in ("x", "z", "U", "dy")]
+    hout = [torch.empty(a.shape, dtype=a.dtype).pin_memory() for a in (y, dx, dz, dU)]
+    h2d = sum(a.numel() * a.element_size() for a in hin)
+    d2h = sum(a.numel() * a.element_size() for a in hout)
+    din = [[torch.empty_like(t[k]) for k in ("x", "z", "U", "dy")] for _ in range(2)]
+    dout = [[y, dx, dz, dU], [torch.empty_like(a) for a in (y, dx, dz, dU)]]
+    ws2 = [ws, torch.empty_like(ws)]
+    comp = torch.cuda.current_stream(dev)
+    s_in = torch.cuda.Stream(dev)
+    s_out = torch.cuda.Stream(dev)
     from dynamic_short_convolutions_causal_b200 import dp
 
-    def step():
-        x.copy_(hx, non_blocking=True)
-        z.copy_(hz, non_blocking=True)
-        U.copy_(hU, non_blocking=True)
-        dy.copy_(hdy, non_blocking=True)
-        dsc.dsc_fwd_lowrank(x, z, U, y, G, W)
-        dsc.dsc_bwd_lowrank(x, z, U, dy, dx, dz, dU, ws, G, W)
+    def compute(bi):
+        x, z, U, dy = din[bi]
+        yy, dxx, dzz, dUU = dout[bi]
+        dsc.dsc_fwd_lowrank(x, z, U, yy, G, W)
+        dsc.dsc_bwd_lowrank(x, z, U, dy, dxx, dzz, dUU, ws2[bi], G, W)
         if world > 1:
-            dp.allreduce_weight_grad(dU)
-        hy.copy_(y, non_blocking=True)
-        hdx.copy_(dx, non_blocking=True)
-        hdz.copy_(dz, non_blocking=True)
-        hdU.copy_(dU, non_blocking=True)
+            dp.allreduce_weight_grad(dUU)
 
-    for _ in range(max(1, args.warmup // 2)):
-        step()
-    torch.cuda.synchronize()
-    barrier(world)
+    def serial_step():
+        for d, h in zip(din[0], hin):
+            d.copy_(h, non_blocking=True)
+        compute(0)
+        for h, d in zip(hout, dout[0]):
+            h.copy_(d, non_blocking=True)
+
+    def timed(fn, steps):
+        torch.cuda.synchronize()
+        barrier(world)
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record(comp)
+        fn(s, steps)
+        e.record(comp)
+        torch.cuda.synchronize()
+        barrier(world)
+        return max_over_ranks(s.elapsed_time(e) / steps, world, dev)
+
+    def run_serial(start, steps):
+        for _ in range(steps):
+            serial_step()
+
+    def run_pipelined(start, steps):
+        s_in.wait_event(start)
+        s_out.wait_event(start)
+        freed = [None, None]      # compute of the buffer set done (inputs reusable)
+        drained = [None, None]    # outputs of the buffer set copied out (outputs reusable)
+        loaded = [None, None]
+        for i in range(steps):
+            bi = i & 1
+            with torch.cuda.stream(s_in):
+                if freed[bi] is not None:
+                    s_in.wait_event(freed[bi])
+                for d, h in zip(din[bi], hin):
+                    d.copy_(h, non_blocking=True)
+                loaded[bi] = torch.cuda.Event()
+                loaded[bi].record(s_in)
+            comp.wait_event(loaded[bi])
+            if drained[bi] is not None:
+                comp.wait_event(drained[bi])
+            compute(bi)
+            freed[bi] = torch.cuda.Event()
+            freed[bi].record(comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(freed[bi])
+                for h, d in zip(hout, dout[bi]):
+                    h.copy_(d, non_blocking=True)
+                drained[bi] = torch.cuda.Event()
+                drained[bi].record(s_out)
+        for ev in drained:
+            if ev is not None:
+                comp.wait_event(ev)
+
     steps = max(2, min(args.steps, 10))
-    s = torch.cuda.Event(enable_timing=True)
-    e = torch.cuda.Event(enable_timing=True)
-    s.record(stream)
-    for _ in range(steps):
-        step()
-    e.record(stream)
-    torch.cuda.synchronize()
-    barrier(world)
-    ms = max_over_ranks(s.elapsed_time(e) / steps, world, dev)
+    for _ in range(max(1, args.warmup // 2)):
+        serial_step()
+    ms_serial = timed(run_serial, steps)
+    timed(run_pipelined, 2)                  # warm-up of the copy streams
+    ms = timed(run_pipelined, steps)
     return {"value": wl.tokens * world / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "pipelined": "two buffer sets; step i+1's copies in and step i-1's copies out overlap step i",
+            "serial": {"value": wl.tokens * world / (ms_serial * 1e-3), "ms_per_step": ms_serial}}
 
 
 def main(argv=None):

@@ -168,8 +168,10 @@ DSC_API dsc_status_t dsc_bwd(const void *x, const void *w, const void *dy, void 
     const char *n[] = {"x", "w", "dy", "dx", "dw"};
     if ((st = check_ptrs(fn, p, n, 5)) != DSC_OK) return st;
     const bool bf16 = dt == DSC_BF16;
-    dsc::launch_conv_dx(w, false, dy, dx, B, T, D, G, W, bf16, false, (cudaStream_t)stream);
-    dsc::launch_dyn_dw(x, dy, dw, B, T, D, G, W, bf16, (cudaStream_t)stream);
+    if (!dsc::launch_dyn_bwd(x, w, dy, dx, dw, B, T, D, G, W, bf16, (cudaStream_t)stream)) {
+        dsc::launch_conv_dx(w, false, dy, dx, B, T, D, G, W, bf16, false, (cudaStream_t)stream);
+        dsc::launch_dyn_dw(x, dy, dw, B, T, D, G, W, bf16, (cudaStream_t)stream);
+    }
     return check_launch(fn);
 }
 

@@ -21,6 +21,9 @@ void launch_conv_fwd(const void *x, const void *w, void *y, int B, int T, int D,
 int static_dw_partials(int B, int T);
 void launch_static_bwd(const void *x, const void *w, const void *dy, void *dx, float *part,
                        float *dw, int B, int T, int D, int W, bool bf16, cudaStream_t s);
+// Explicit-filter backward in one pass (dx and dw); false: sizes it does not take
+bool launch_dyn_bwd(const void *x, const void *w, const void *dy, void *dx, float *dw, int B, int T, int D,
+                    int G, int W, bool bf16, cudaStream_t s);
 
 // Decode step (decode.cu)
 bool decode_supported(int D, int G, int W, int R);

@@ -291,6 +291,154 @@ k_stream_fwd(const T *__restrict__ x, const T *__restrict__ w, T *__restrict__ y
 }
 
 
+// ------------------------------------------------------------------ explicit backward
+// One pass over x, dy and the per-token taps of a chunk of tokens (dx in scatter form):
+//   token t adds dy[t] (the residual) and w[t,g,k] dy[t] into the open dx row t-k; row
+//   t-W+1 is then complete; W-1 tokens past the chunk finish its last rows;
+//   dw[t,g,k] = sum_{c in g} dy[t,c] x[t-k,c]: the thread's V channels are summed in the
+//   thread and across the G/V threads of a group by a fixed xor-shuffle tree.
+// Taken when the taps are staged with the rows (W * sizeof(T) of 4, 8 or 16 bytes) and
+// the groups tile the threads' channel vectors (G % V == 0, G/V a power of two <= 32).
+template <typename T, int W>
+__global__ void __launch_bounds__(256)
+k_dyn_bwd(const T *__restrict__ x, const T *__restrict__ w, const T *__restrict__ dy, T *__restrict__ dx,
+          float *__restrict__ dw, int B, int T_, int D, int G, int chunk) {
+    constexpr int V = Lanes<T, W>::V;
+    using P = Pack<T, V>;
+    constexpr int TB = W * (int)sizeof(T);                         // bytes of one token's taps
+    constexpr int SB = P::BYTES > TB ? P::BYTES : TB;              // slot size
+    constexpr int KU = Batch<SB>::KU;
+    using TR = typename RawOf<TB>::type;
+    extern __shared__ __align__(16) uint8_t stg_raw[];
+    const Staging<SB, 3, KU> stg((uint32_t)__cvta_generic_to_shared(stg_raw), (int)threadIdx.x);
+    const int nbx = cdiv(D / V, 256);
+    const int nch = cdiv(T_, chunk);
+    const int nitems = nbx * B * nch;
+    const int NG = D / G;
+    const int lanes = G / V;
+    for (int item = blockIdx.x; item < nitems; item += gridDim.x) {
+        const int bx = item % nbx, by = item / nbx;
+        const int v = bx * 256 + threadIdx.x;
+        const bool active = v < D / V;
+        const int b = by / nch;
+        const int t0 = (by - b * nch) * chunk;
+        const int t1 = min(t0 + chunk, T_);
+        const int t1e = min(t1 + W - 1, T_);         // dy and taps needed up to here
+        const int c0 = active ? v * V : 0;
+        const size_t row0 = (size_t)b * T_;
+        const T *xb = x + row0 * D + c0;
+        const T *gb = dy + row0 * D + c0;
+        T *ob = dx + row0 * D + c0;
+        const T *wb = w + (row0 * NG + c0 / G) * W;
+        float acc[W][V];                             // acc[k] = open dx row t-k
+        float xw[W][V];                              // xw[k] = x[t-k]
+#pragma unroll
+        for (int k = 0; k < W; ++k)
+#pragma unroll
+            for (int i = 0; i < V; ++i) acc[k][i] = 0.f;
+#pragma unroll
+        for (int k = 1; k < W; ++k) {
+            if (active && t0 - k >= 0) P::unpack(P::load(xb + (size_t)(t0 - k) * D), xw[k]);
+            else
+#pragma unroll
+                for (int i = 0; i < V; ++i) xw[k][i] = 0.f;
+        }
+        auto issue = [&](int tb, int stage) {
+#pragma unroll
+            for (int u = 0; u < KU; ++u) {
+                const bool ok = active && tb + u < t1e;
+                const int t = ok ? tb + u : t0;
+                cp_async<P::BYTES>(stg.at(stage, 0, u), xb + (size_t)t * D, ok && tb + u < t1);
+                cp_async<P::BYTES>(stg.at(stage, 1, u), gb + (size_t)t * D, ok);
+                cp_async<TB>(stg.at(stage, 2, u), wb + (size_t)t * NG * W, ok);
+            }
+            cp_commit();
+        };
+        const int nb = cdiv(t1e - t0, KU);
+        issue(t0, 0);
+        for (int bi = 0; bi < nb; ++bi) {
+            const int tb = t0 + bi * KU, stage = bi & 1;
+            if (bi + 1 < nb) issue(tb + KU, stage ^ 1);
+            else cp_commit();
+            cp_wait<1>();
+#pragma unroll
+            for (int u = 0; u < KU; ++u) {
+                const int t = tb + u;
+                if (t >= t1e) break;
+                float g[V];
+                P::unpack(lds_raw<typename P::raw_t>(stg.at(stage, 1, u)), g);
+                P::unpack(lds_raw<typename P::raw_t>(stg.at(stage, 0, u)), xw[0]);
+                const TR tr = lds_raw<TR>(stg.at(stage, 2, u));
+                uint32_t tw[TB / 4];
+                if constexpr (TB == 4) {
+                    tw[0] = tr;
+                } else if constexpr (TB == 8) {
+                    tw[0] = tr.x; tw[1] = tr.y;
+                } else {
+                    tw[0] = tr.x; tw[1] = tr.y; tw[2] = tr.z; tw[3] = tr.w;
+                }
+                float f[W];
+#pragma unroll
+                for (int k = 0; k < W; ++k) {
+                    if constexpr (sizeof(T) == 2) f[k] = (k & 1) ? bf16_hi(tw[k / 2]) : bf16_lo(tw[k / 2]);
+                    else f[k] = __uint_as_float(tw[k]);
+                }
+                // dx: open row t; add token t's contributions; row t-W+1 is complete
+#pragma unroll
+                for (int k = W - 1; k >= 1; --k)
+#pragma unroll
+                    for (int i = 0; i < V; ++i) acc[k][i] = acc[k - 1][i];
+#pragma unroll
+                for (int i = 0; i < V; ++i) acc[0][i] = g[i];
+#pragma unroll
+                for (int k = 0; k < W; ++k)
+#pragma unroll
+                    for (int i = 0; i < V; ++i) acc[k][i] = fmaf(f[k], g[i], acc[k][i]);
+                const int s = t - (W - 1);
+                if (active && s >= t0 && s < t1) P::store(ob + (size_t)s * D, acc[W - 1]);
+                // dw of token t (tokens of the chunk only)
+                if (t < t1) {
+                    float sw[W];
+#pragma unroll
+                    for (int k = 0; k < W; ++k) {
+                        float a = 0.f;
+#pragma unroll
+                        for (int i = 0; i < V; ++i) a = fmaf(g[i], xw[k][i], a);
+                        sw[k] = a;
+                    }
+                    for (int o = 1; o < lanes; o <<= 1)
+#pragma unroll
+                        for (int k = 0; k < W; ++k) sw[k] += __shfl_xor_sync(0xffffffffu, sw[k], o);
+                    if (active && (v % lanes) == 0) {
+                        float *q = dw + ((row0 + t) * NG + c0 / G) * W;
+#pragma unroll
+                        for (int k = 0; k < W; ++k) q[k] = sw[k];
+                    }
+                }
+#pragma unroll
+                for (int k = W - 1; k >= 1; --k)
+#pragma unroll
+                    for (int i = 0; i < V; ++i) xw[k][i] = xw[k - 1][i];
+            }
+        }
+        cp_wait<0>();
+        // at the sequence end the rows still open have all their contributions
+        if (t1e == T_) {
+#pragma unroll
+            for (int k = 1; k < W; ++k) {
+#pragma unroll
+                for (int kk = W - 1; kk >= 1; --kk)
+#pragma unroll
+                    for (int i = 0; i < V; ++i) acc[kk][i] = acc[kk - 1][i];
+#pragma unroll
+                for (int i = 0; i < V; ++i) acc[0][i] = 0.f;
+                const int s = T_ - 1 - (W - 1) + k;      // row completed by this virtual step
+                if (active && s >= t0 && s < t1) P::store(ob + (size_t)s * D, acc[W - 1]);
+            }
+        }
+    }
+}
+
 // ------------------------------------------------------------------ static backward
 // One pass over x and dy per chunk of tokens:
 //   dx[s]  = dy[s] + sum_k w[k] dy[s+k]             (dy rows t-k held in dyw[k])
@@ -462,6 +610,37 @@ int resident_blocks(K kern, int threads, int smem) {
     return nsm * per;
 }
 
+template <typename T>
+bool launch_dyn_bwd_T(const void *x, const void *w, const void *dy, void *dx, float *dw, int B, int T_, int D,
+                      int G, int W, cudaStream_t s) {
+    const T *xp = (const T *)x, *wp = (const T *)w, *gp = (const T *)dy;
+    T *op = (T *)dx;
+    constexpr int kRows = 64;   // tokens per chunk
+    switch (W) {
+#define DSC_CASE(WW)                                                                                   \
+    case WW: {                                                                                         \
+        constexpr int V = Lanes<T, WW>::V;                                                             \
+        constexpr int TB = WW * (int)sizeof(T);                                                        \
+        if constexpr (TB == 4 || TB == 8 || TB == 16) {                                                \
+            if (G % V != 0 || G / V > 32 || ((G / V) & (G / V - 1)) != 0) return false;                \
+            constexpr int SB = Pack<T, V>::BYTES > TB ? Pack<T, V>::BYTES : TB;                        \
+            const int smem = 256 * Staging<SB, 3, Batch<SB>::KU>::bytes_per_thread();                  \
+            auto kern = k_dyn_bwd<T, WW>;                                                              \
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);             \
+            const long long items = (long long)cdiv(D / V, 256) * B * cdiv(T_, kRows);                 \
+            const int grid = (int)std::min<long long>(items, (long long)resident_blocks(kern, 256, smem)); \
+            kern<<<grid, 256, smem, s>>>(xp, wp, gp, op, dw, B, T_, D, G, kRows);                       \
+            return true;                                                                               \
+        } else {                                                                                       \
+            return false;                                                                              \
+        }                                                                                              \
+    }
+        DSC_CASE(1) DSC_CASE(2) DSC_CASE(3) DSC_CASE(4) DSC_CASE(5) DSC_CASE(6) DSC_CASE(7) DSC_CASE(8)
+#undef DSC_CASE
+    }
+    return false;
+}
+
 template <typename T, int W, bool STATIC>
 void launch_fwd_k(int nitems, const T *x, const T *w, T *y, int B, int T_, int D, int G, int chunk,
                   cudaStream_t s) {
@@ -539,6 +718,12 @@ void launch_conv_fwd(const void *x, const void *w, void *y, int B, int T, int D,
         if (is_static) launch_stream_fwd_T<float, true>(x, w, y, B, T, D, 1, W, s);
         else launch_stream_fwd_T<float, false>(x, w, y, B, T, D, G, W, s);
     }
+}
+
+bool launch_dyn_bwd(const void *x, const void *w, const void *dy, void *dx, float *dw, int B, int T, int D, int G,
+                    int W, bool bf16_, cudaStream_t s) {
+    return bf16_ ? launch_dyn_bwd_T<bf16>(x, w, dy, dx, dw, B, T, D, G, W, s)
+                 : launch_dyn_bwd_T<float>(x, w, dy, dx, dw, B, T, D, G, W, s);
 }
 
 void launch_static_bwd(const void *x, const void *w, const void *dy, void *dx, float *part, float *dw, int B,
