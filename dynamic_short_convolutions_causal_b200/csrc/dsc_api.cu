@@ -9,6 +9,12 @@
 #include "../../include/dsc.h"
 #include "internal.h"
 
+#ifndef DSC_DECODE_TC_MIN_B
+#define DSC_DECODE_TC_MIN_B 8      // smallest batch whose decode step runs on the tensor cores
+                                   // (B200, D=6144: 5.05 us there against 5.12 on CUDA cores;
+                                   // at B=1 the CUDA cores win, 4.8 against 5.1 us)
+#endif
+
 namespace {
 
 thread_local char g_err[512] = "";
@@ -241,6 +247,10 @@ DSC_API dsc_status_t dsc_decode_step_lowrank(const void *x_t, const void *z_t, c
         const char *sn[] = {"state"};
         if ((st = check_ptrs(fn, sp, sn, 1)) != DSC_OK) return st;
     }
+    // tensor cores for w = z U when the batch fills enough of a 128-row tile, else CUDA cores
+    if (B >= DSC_DECODE_TC_MIN_B && dsc::tc_decode_lowrank_supported(B, D, G, W, R, dt == DSC_BF16))
+        return check_launch(fn, dsc::launch_tc_decode_lowrank(x_t, z_t, U, state, y_t, B, D, G, W, R,
+                                                              (cudaStream_t)stream));
     if (!dsc::decode_supported(D, G, W, R))
         return fail(DSC_ERR_UNSUPPORTED, "%s: R=%d with W=%d needs more shared memory than a block has", fn, R, W);
     return check_launch(fn, dsc::launch_decode_lowrank(x_t, z_t, U, state, y_t, B, D, G, W, R, dt == DSC_BF16,

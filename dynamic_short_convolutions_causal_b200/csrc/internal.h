@@ -31,6 +31,10 @@ cudaError_t launch_decode_lowrank(const void *x, const void *z, const void *U, v
                                   int B, int D, int G, int W, int R, bool bf16, cudaStream_t s);
 cudaError_t launch_decode(const void *x, const void *w, void *state, void *y, int B, int D, int G,
                           int W, bool bf16, cudaStream_t s);
+// ... on the tensor cores (tc_lowrank.cu): the forward kernel with the sequences as rows
+bool tc_decode_lowrank_supported(int B, int D, int G, int W, int R, bool bf16);
+cudaError_t launch_tc_decode_lowrank(const void *x, const void *z, const void *U, void *state, void *y, int B,
+                                     int D, int G, int W, int R, cudaStream_t s);
 
 // Sequence-shard halo fix-ups (halo.cu)
 cudaError_t launch_halo_fwd_lowrank(const void *x, const void *z, const void *U, const void *x_prev, void *y,

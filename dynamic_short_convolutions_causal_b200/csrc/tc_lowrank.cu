@@ -27,6 +27,7 @@
 #include <cudaTypedefs.h>
 
 #include <cstdio>
+#include <cstring>
 #include <mutex>
 
 #include "common.cuh"
@@ -78,6 +79,18 @@ struct FwdParams {
     WaitTest wt;
 };
 
+// Decode step (one new token per sequence): the kernel's token rows are the B sequences
+// (a "sequence" of B rows, z_t [B, R] as its z), and an x stage holds, per sequence, x_t
+// and its rolling window state [B, W-1, D] instead of a token tile and its halo.  The
+// window is read through a view with the sequence as the middle dimension (dims
+// {D, B, W-1}), so that one box lands in shared memory as [window row][128 sequences]
+// [64 channels] and rows 1.. of it are again one box: `load` (all W-1 rows), `shift`
+// (W-2 rows, stage rows 1.. to window rows 0..) and `push` (x_t to the newest row).
+struct DecMaps {
+    CUtensorMap load, shift, push;
+};
+constexpr uint32_t kDecRow = 128 * 128;       // one [128 sequences][64 channels] bf16 region
+
 // Barrier slots in shared memory (8 bytes each).
 constexpr int kMaxXStages = 8;
 constexpr int kOpStages = 2;
@@ -119,10 +132,13 @@ struct Taps {
 
 // Epilogue: each set of 8 warps covers one whole tile (warp = 32 token rows x 32
 // channels); with two sets, consecutive tiles (the two TMEM accumulator buffers) are
-// processed concurrently.  Two sets need the chunk's taps to fit in 32 registers.
-template <int W, int GC>
+// processed concurrently.  Two sets need the chunk's taps to fit in 32 registers, and
+// at least two x stages: a set waits for phase n of its stage's barrier before the
+// phases in between have completed, which an mbarrier's parity cannot tell apart when
+// both sets share one stage.  The decode step keeps one set (its stages are W x 16 KB).
+template <int W, int GC, bool DEC = false>
 struct EpiShape {
-    static constexpr int SETS = (Taps<W, GC>::NCOL <= 32 && DSC_FWD_SETS >= 2) ? 2 : 1;
+    static constexpr int SETS = (!DEC && Taps<W, GC>::NCOL <= 32 && DSC_FWD_SETS >= 2) ? 2 : 1;
     static constexpr int WARPS = 8 * SETS;
     static constexpr int OPWARP = 2 + WARPS;       // the operand (z, U) producer
     static constexpr int THREADS = 32 * (3 + WARPS);
@@ -164,12 +180,13 @@ __device__ __forceinline__ void conv_chunk(const uint32_t *wr, const uint4 (&xu)
     }
 }
 
-template <int W, int GC, bool ROPE>
-__global__ void __launch_bounds__(EpiShape<W, GC>::THREADS, 1)
-k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z,
-                 const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_y,
-                 const FwdParams p) {
-    using ES = EpiShape<W, GC>;
+// The whole kernel, for the forward (DEC false: tiles of 128 tokens of one sequence) and
+// the decode step (DEC true: tiles of 128 sequences, one token each).  The maps are the
+// kernels' grid-constant parameters.
+template <int W, int GC, bool ROPE, bool DEC>
+__device__ __forceinline__ void fwd_tiles(const CUtensorMap &tm_x, const CUtensorMap &tm_z, const CUtensorMap &tm_u,
+                                          const CUtensorMap &tm_y, const DecMaps *dm, const FwdParams &p) {
+    using ES = EpiShape<W, GC, DEC>;
     using TP = Taps<W, GC>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = (uint8_t *)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -202,6 +219,11 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
         tma_prefetch(&tm_z);
         tma_prefetch(&tm_u);
         tma_prefetch(&tm_y);
+        if (DEC && W > 1) {
+            tma_prefetch(&dm->load);
+            if (W > 2) tma_prefetch(&dm->shift);
+            tma_prefetch(&dm->push);
+        }
     }
     if (warp == 1) {
         tmem_alloc(smem_u32(tmem_holder), p.tmem_cols);
@@ -224,8 +246,27 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
                 const int s = it % S, n = it / S;
                 if (!mbar_wait<kWaitHint>(bar.empty(s), (n & 1) ^ 1, abort, 2u, &g_fault, p.wt.wait_ns)) break;
                 if (it == 0 && (int)blockIdx.x == p.wt.withhold_cta) continue;   // test hook: no loads
-                mbar_arrive_expect_tx(bar.full(s), p.x_stage_tx);
-                tma_load_3d(sb + p.off_x + s * p.x_stage_bytes, &tm_x, bar.full(s), slice * kDt, t0 - (W - 1), b);
+                const uint32_t xs = sb + p.off_x + s * p.x_stage_bytes;
+                if constexpr (DEC) {
+                    // x_t of the tile's sequences, then their windows; the stage's shift
+                    // stores of the previous round must have read it first
+                    if (W > 1) bulk_wait_read<0>();
+                    mbar_arrive_expect_tx(bar.full(s), p.x_stage_tx);
+                    tma_load_3d(xs, &tm_x, bar.full(s), slice * kDt, t0, b);
+                    if (W > 1) {
+                        tma_load_3d(xs + kDecRow, &dm->load, bar.full(s), slice * kDt, t0, 0);
+                        // once both have landed the window moves on in global memory: rows
+                        // 1..W-2 to rows 0..W-3 and x_t into row W-2 (only this tile's
+                        // sequences and channels, which no other tile reads)
+                        if (!mbar_wait<kWaitHint>(bar.full(s), n & 1, abort, 2u, &g_fault, p.wt.wait_ns)) break;
+                        if (W > 2) tma_store_3d(&dm->shift, xs + 2 * kDecRow, slice * kDt, t0, 0);
+                        tma_store_3d(&dm->push, xs, slice * kDt, t0, W - 2);
+                        bulk_commit();
+                    }
+                } else {
+                    mbar_arrive_expect_tx(bar.full(s), p.x_stage_tx);
+                    tma_load_3d(xs, &tm_x, bar.full(s), slice * kDt, t0 - (W - 1), b);
+                }
             }
             // Let every load this warp issued land before the CTA can exit.
             const int issued = it;
@@ -233,6 +274,7 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
                 const int last = issued - 1 - ((issued - 1 - s) % S);   // last tile using stage s
                 mbar_drain(bar.full(s), (last / S) & 1, p.wt.wait_ns);
             }
+            if (DEC) bulk_wait_all();    // the window stores are complete
         }
         __syncwarp();
     } else if (warp == 1) {
@@ -307,13 +349,14 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
         // y staging: row `lane` of this warp's buffer, 64-byte swizzle (16-byte chunk ^ (lane/2)%4)
         const uint32_t ystage = sb + p.off_y + (uint32_t)ew * 2 * ES::YBUF;
         const uint32_t yrow = (ystage + lane * 64) ^ ((uint32_t)((lane >> 1) & 3) << 4);
-        // x stage: the thread's rows r_k = row + W-1-k; a row is 128 bytes with 128-byte
-        // swizzle (16-byte chunk ^ r%8).  Rows are 128-byte aligned, so the swizzled address
-        // of chunk c is (row address ^ ((r%8) << 4)) ^ (c << 4).
+        // x stage: the thread's rows r_k = row + W-1-k (decode: x_t in region 0, window
+        // row W-1-k in region W-k, a region being 128 rows); a row is 128 bytes with
+        // 128-byte swizzle (16-byte chunk ^ r%8).  Rows are 128-byte aligned, so the
+        // swizzled address of chunk c is (row address ^ ((r%8) << 4)) ^ (c << 4).
         uint32_t xrow[W];
 #pragma unroll
         for (int k = 0; k < W; ++k) {
-            const uint32_t r = (uint32_t)(row + (W - 1) - k);
+            const uint32_t r = DEC ? (uint32_t)((k == 0 ? 0 : W - k) * kTt + row) : (uint32_t)(row + (W - 1) - k);
             xrow[k] = (r * 128u) ^ ((r & 7u) << 4) ^ ((uint32_t)(4 * h) << 4);
         }
         int yc = 0;
@@ -429,6 +472,22 @@ k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant
     }
 }
 
+template <int W, int GC, bool ROPE>
+__global__ void __launch_bounds__(EpiShape<W, GC>::THREADS, 1)
+k_tc_lowrank_fwd(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z,
+                 const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_y,
+                 const FwdParams p) {
+    fwd_tiles<W, GC, ROPE, false>(tm_x, tm_z, tm_u, tm_y, nullptr, p);
+}
+
+template <int W, int GC>
+__global__ void __launch_bounds__(EpiShape<W, GC, true>::THREADS, 1)
+k_tc_decode_lowrank(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_z,
+                    const __grid_constant__ CUtensorMap tm_u, const __grid_constant__ CUtensorMap tm_y,
+                    const __grid_constant__ DecMaps dm, const FwdParams p) {
+    fwd_tiles<W, GC, false, true>(tm_x, tm_z, tm_u, tm_y, &dm, p);
+}
+
 // ------------------------------------------------------------------ host side
 namespace {
 
@@ -480,7 +539,9 @@ bool is_pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
 
 constexpr uint32_t kSmemLimit = 227 * 1024;
 
-bool plan_fwd(int B, int T, int D, int G, int W, int R, FwdParams &p) {
+// dec: the decode step's layout (T = the number of sequences, B = 1; an x stage holds
+// x_t and the W-1 window rows of 128 sequences).
+bool plan_fwd(int B, int T, int D, int G, int W, int R, FwdParams &p, bool dec = false) {
     if (!(R == 16 || R == 32 || R == 64)) return false;
     if (D % kDt || !is_pow2(G) || G > 64 || W < 1 || W > 8) return false;
     p.B = B; p.T = T; p.D = D; p.G = G; p.R = R;
@@ -498,13 +559,13 @@ bool plan_fwd(int B, int T, int D, int G, int W, int R, FwdParams &p) {
     int cols = 32;
     while (cols < p.nbuf * p.bufcols) cols *= 2;
     p.tmem_cols = cols;
-    p.x_stage_tx = (uint32_t)(kDt * 2 * (kTt + W - 1));
+    p.x_stage_tx = dec ? (uint32_t)W * kDecRow : (uint32_t)(kDt * 2 * (kTt + W - 1));
     p.x_stage_bytes = (p.x_stage_tx + 1023) / 1024 * 1024;
     p.z_stage_bytes = (uint32_t)(kTt * R * 2);
     p.u_bytes = (uint32_t)(p.u_boxes * R * 128);
     p.z_layout = R == 16 ? kSw32 : (R == 32 ? kSw64 : kSw128);
     const int ncol = G <= 8 ? (8 / G) * W : W;      // must match EpiShape / Taps
-    p.nwg = (ncol <= 32 && DSC_FWD_SETS >= 2) ? 2 : 1;   // epilogue warp sets
+    p.nwg = (!dec && ncol <= 32 && DSC_FWD_SETS >= 2) ? 2 : 1;   // epilogue warp sets
     if (p.nbuf < p.nwg) p.nwg = p.nbuf;
     p.y_buf_bytes = (uint32_t)(32 * 32 * 2);
     p.off_z = 0;
@@ -514,7 +575,8 @@ bool plan_fwd(int B, int T, int D, int G, int W, int R, FwdParams &p) {
     p.off_op = 0;
     p.off_x = p.op_stages * p.op_bytes;
     // as deep an x ring as fits next to the operand ring and the y staging
-    for (int st = kMaxXStages; st >= 2; --st) {
+    // (at least one stage per epilogue set; the decode step's single set can do with one)
+    for (int st = kMaxXStages; st >= std::max(p.nwg, dec ? 1 : 2); --st) {
         const uint32_t off_y = p.off_x + st * p.x_stage_bytes;
         const uint32_t off_bar = off_y + 8 * p.nwg * 2 * p.y_buf_bytes;
         const uint32_t total = off_bar + kBarBytes + 16 + 1024;
@@ -530,6 +592,18 @@ bool plan_fwd(int B, int T, int D, int G, int W, int R, FwdParams &p) {
 
 uint32_t smem_bytes(const FwdParams &p) { return p.off_bar + kBarBytes + 16 + 1024; }
 
+// bf16 tensor map with explicit byte strides of dims 1.. (dims[0] contiguous).
+bool make_map_strided(CUtensorMap *m, const void *ptr, const uint64_t (&dims)[3], const uint64_t (&strides)[2],
+                      const uint32_t (&box)[3], CUtensorMapSwizzle sw) {
+    auto enc = encoder();
+    if (!enc) return false;
+    cuuint64_t gdim[3] = {dims[0], dims[1], dims[2]}, gstride[2] = {strides[0], strides[1]};
+    cuuint32_t bdim[3] = {box[0], box[1], box[2]}, estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(ptr), gdim, gstride, bdim, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int W, int GC>
 cudaError_t launch_fwd_t(const CUtensorMap &mx, const CUtensorMap &mz, const CUtensorMap &mu,
                          const CUtensorMap &my, const FwdParams &p, cudaStream_t s) {
@@ -542,6 +616,32 @@ cudaError_t launch_fwd_t(const CUtensorMap &mx, const CUtensorMap &mz, const CUt
     const int grid = std::min(p.n_tiles, num_sms());
     kern<<<grid, ES::THREADS, smem, s>>>(mx, mz, mu, my, p);
     return cudaGetLastError();
+}
+
+template <int W, int GC>
+cudaError_t launch_dec_t(const CUtensorMap &mx, const CUtensorMap &mz, const CUtensorMap &mu,
+                         const CUtensorMap &my, const DecMaps &dm, const FwdParams &p, cudaStream_t s) {
+    auto kern = k_tc_decode_lowrank<W, GC>;
+    using ES = EpiShape<W, GC, true>;
+    if (p.nwg != ES::SETS || p.y_buf_bytes != (uint32_t)ES::YBUF) return cudaErrorInvalidConfiguration;
+    const uint32_t smem = smem_bytes(p);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int grid = std::min(p.n_tiles, num_sms());
+    kern<<<grid, ES::THREADS, smem, s>>>(mx, mz, mu, my, dm, p);
+    return cudaGetLastError();
+}
+
+template <int W>
+cudaError_t launch_dec_w(int G, const CUtensorMap &mx, const CUtensorMap &mz, const CUtensorMap &mu,
+                         const CUtensorMap &my, const DecMaps &dm, const FwdParams &p, cudaStream_t s) {
+    switch (G) {
+        case 1: return launch_dec_t<W, 1>(mx, mz, mu, my, dm, p, s);
+        case 2: return launch_dec_t<W, 2>(mx, mz, mu, my, dm, p, s);
+        case 4: return launch_dec_t<W, 4>(mx, mz, mu, my, dm, p, s);
+        case 8: return launch_dec_t<W, 8>(mx, mz, mu, my, dm, p, s);
+        default: return launch_dec_t<W, 16>(mx, mz, mu, my, dm, p, s);
+    }
 }
 
 template <int W>
@@ -601,6 +701,63 @@ cudaError_t launch_tc_lowrank_fwd(const void *x, const void *z, const void *U, v
         case 6: return launch_fwd_w<6>(G, mx, mz, mu, my, p, s);
         case 7: return launch_fwd_w<7>(G, mx, mz, mu, my, p, s);
         default: return launch_fwd_w<8>(G, mx, mz, mu, my, p, s);
+    }
+}
+
+bool tc_decode_lowrank_supported(int B, int D, int G, int W, int R, bool bf16) {
+    tc::FwdParams p;
+    return bf16 && B > 0 && tc::plan_fwd(1, B, D, G, W, R, p, true);
+}
+
+cudaError_t launch_tc_decode_lowrank(const void *x, const void *z, const void *U, void *st, void *y, int B, int D,
+                                     int G, int W, int R, cudaStream_t s) {
+    using namespace tc;
+    FwdParams p;
+    if (!plan_fwd(1, B, D, G, W, R, p, true)) return cudaErrorNotSupported;
+    p.cs = nullptr;
+    p.dh = 0;
+    p.n_rot = 0;
+    take_wait_test(&p.wt.wait_ns, &p.wt.withhold_cta);
+    CUtensorMap mx, mz, mu, my;
+    DecMaps dm;
+    memset(&dm, 0, sizeof(dm));
+    const uint64_t dx[3] = {(uint64_t)D, (uint64_t)B, 1};
+    const uint32_t bx[3] = {(uint32_t)kDt, (uint32_t)kTt, 1};
+    const uint64_t dz[3] = {(uint64_t)R, (uint64_t)B, 1};
+    const uint32_t bz[3] = {(uint32_t)R, (uint32_t)kTt, 1};
+    const uint64_t du[2] = {(uint64_t)(D / G) * W, (uint64_t)R};
+    const uint32_t bu[2] = {64, (uint32_t)R};
+    const uint32_t by[3] = {32, 32, 1};
+    const CUtensorMapSwizzle zsw = R == 16 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                           : (R == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B);
+    bool ok = make_map(&mx, x, 3, dx, bx, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              make_map(&mz, z, 3, dz, bz, zsw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) &&
+              make_map(&mu, U, 2, du, bu, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) &&
+              make_map(&my, y, 3, dx, by, CU_TENSOR_MAP_SWIZZLE_64B);
+    if (ok && W > 1) {
+        // the window [B, W-1, D] as dims {D, B, W-1}: sequence stride (W-1)*D, row stride D
+        const uint64_t ds[3] = {(uint64_t)D, (uint64_t)B, (uint64_t)(W - 1)};
+        const uint64_t ss[2] = {(uint64_t)(W - 1) * D * 2, (uint64_t)D * 2};
+        const uint32_t bl[3] = {(uint32_t)kDt, (uint32_t)kTt, (uint32_t)(W - 1)};
+        const uint32_t bs[3] = {(uint32_t)kDt, (uint32_t)kTt, (uint32_t)(W > 2 ? W - 2 : 1)};
+        const uint32_t bp[3] = {(uint32_t)kDt, (uint32_t)kTt, 1};
+        ok = make_map_strided(&dm.load, st, ds, ss, bl, CU_TENSOR_MAP_SWIZZLE_128B) &&
+             (W == 2 || make_map_strided(&dm.shift, st, ds, ss, bs, CU_TENSOR_MAP_SWIZZLE_128B)) &&
+             make_map_strided(&dm.push, st, ds, ss, bp, CU_TENSOR_MAP_SWIZZLE_128B);
+    }
+    if (!ok) {
+        set_last_error("dsc_decode_step_lowrank: cuTensorMapEncodeTiled failed");
+        return cudaErrorInvalidValue;
+    }
+    switch (W) {
+        case 1: return launch_dec_w<1>(G, mx, mz, mu, my, dm, p, s);
+        case 2: return launch_dec_w<2>(G, mx, mz, mu, my, dm, p, s);
+        case 3: return launch_dec_w<3>(G, mx, mz, mu, my, dm, p, s);
+        case 4: return launch_dec_w<4>(G, mx, mz, mu, my, dm, p, s);
+        case 5: return launch_dec_w<5>(G, mx, mz, mu, my, dm, p, s);
+        case 6: return launch_dec_w<6>(G, mx, mz, mu, my, dm, p, s);
+        case 7: return launch_dec_w<7>(G, mx, mz, mu, my, dm, p, s);
+        default: return launch_dec_w<8>(G, mx, mz, mu, my, dm, p, s);
     }
 }
 

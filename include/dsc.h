@@ -173,9 +173,11 @@ DSC_API size_t dsc_static_bwd_noalloc_max_scratch_bytes(void);
  *   (inputs before its start count as zero, as in the forward).  state may be NULL
  *   when W = 1.  Stepping a sequence from a zero window reproduces the forward's
  *   outputs token by token.
- * Same element type, alignment and error rules as the other entry points; y_t must not
- * overlap x_t or state.  dsc_decode_step_lowrank returns DSC_ERR_UNSUPPORTED when R and W
- * are too large for its shared-memory tile (R = 256 with W = 8). */
+ * Same element type, alignment and error rules as the other entry points; no two of
+ * y_t, x_t and state may overlap.  dsc_decode_step_lowrank forms w_t on the tensor cores
+ * (the fused forward's kernel, one row per sequence) for bf16 shapes that kernel takes,
+ * else on CUDA cores; it returns DSC_ERR_UNSUPPORTED when R and W are too large for the
+ * CUDA-core shared-memory tile (R = 256 with W = 8). */
 DSC_API dsc_status_t dsc_decode_step(const void *x_t, const void *w_t, void *state, void *y_t,
                                      int B, int D, int G, int W,
                                      dsc_dtype_t dt, dsc_stream_t stream);

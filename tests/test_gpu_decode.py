@@ -29,13 +29,21 @@ def _draw(shape, std, dt, gen):
 
 DECODE = [
     # B, D, G, W, R, dtype
+    # CUDA cores (fewer than 8 sequences, or shapes the tensor-core kernel does not take)
     (1, 6144, 1, 4, 32, "bf16"),       # the stacked-QKV width, one sequence
-    (8, 6144, 1, 4, 32, "bf16"),
+    (8, 6144, 1, 4, 32, "bf16"),       # from here on bf16 with D % 64 == 0: tensor cores
     (64, 256, 4, 8, 64, "bf16"),
     (37, 96, 3, 5, 8, "bf16"),         # ragged sequence block, G not a power of two
     (3, 40, 8, 3, 16, "f32"),          # D not a multiple of the 32-channel block
     (5, 64, 1, 1, 4, "bf16"),          # W = 1: no window
     (2, 128, 64, 2, 48, "bf16"),
+    # tensor-core decode (the forward kernel with one row per sequence)
+    (256, 6144, 1, 4, 32, "bf16"),     # two full 128-sequence tiles
+    (130, 128, 2, 8, 16, "bf16"),      # a ragged second tile, W = 8
+    (200, 512, 8, 3, 64, "bf16"),
+    (129, 192, 16, 6, 32, "bf16"),
+    (33, 128, 1, 2, 16, "bf16"),       # W = 2: the window is x_t alone
+    (40, 64, 1, 1, 16, "bf16"),        # W = 1
 ]
 
 
@@ -63,7 +71,8 @@ def test_decode_step_matches_oracle(dsc, B, D, G, W, R, dt):
         assert np.array_equal(f64(st), rst), "window after the step (lowrank=%s)" % lowrank
 
 
-@pytest.mark.parametrize("B,T,D,G,W,R", [(3, 20, 128, 2, 4, 16), (2, 9, 64, 1, 7, 32)])
+@pytest.mark.parametrize("B,T,D,G,W,R", [(3, 20, 128, 2, 4, 16), (2, 9, 64, 1, 7, 32), (9, 12, 128, 1, 4, 32),
+                                         (130, 6, 64, 4, 5, 16)])
 def test_decode_steps_reproduce_forward(dsc, B, T, D, G, W, R):
     """Stepping from a zero window through T tokens gives the fused forward's outputs."""
     wl = di.small(B, T, D, G, W, R, "bf16", seed=T)
