@@ -58,9 +58,11 @@ def read_peaks():
 
 class Clocks:
     """SM clocks and throttle reasons during the timed region: nvidia-smi (the recipe's
-    query, every 100 ms) and, since a timed region can be a few ms long, NVML read every
-    millisecond from a thread.  The GPU is named by its PCI bus id, so that the sampled
-    device is the one the CUDA device maps to whatever the visible-device numbering."""
+    query, every 100 ms) and, since a timed region can be a few ms long, NVML read about
+    every half millisecond from a thread that is initialised and polling before the region
+    starts (arm) and keeps its samples only between start and stop.  The GPU is named by
+    its PCI bus id, so that the sampled device is the one the CUDA device maps to whatever
+    the visible-device numbering."""
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -72,6 +74,9 @@ class Clocks:
         self.path = None
         self.thread = None
         self.nvml = []
+        self.recording = False
+        self.stop_flag = False
+        self.max_mhz = None
         try:
             pr = torch.cuda.get_device_properties(index)
             self.bus = "%08X:%02X:%02X.0" % (pr.pci_domain_id, pr.pci_bus_id, pr.pci_device_id)
@@ -89,16 +94,21 @@ class Clocks:
                     "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
                     "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap}
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self.ready.set()
             while not self.stop_flag:
                 mhz = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
                 r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
-                self.nvml.append((mhz, sorted(k for k, v in bits.items() if r & v)))
-                time.sleep(0.001)
+                if self.recording:
+                    self.nvml.append((mhz, sorted(k for k, v in bits.items() if r & v)))
+                time.sleep(0.0005)
             pynvml.nvmlShutdown()
         except Exception:
             pass
+        finally:
+            self.ready.set()
 
-    def start(self):
+    def arm(self):
+        """Starts the samplers ahead of the timed region; nothing is kept until start()."""
         try:
             import tempfile
             fd, self.path = tempfile.mkstemp(prefix="dsc_clocks_", suffix=".csv")
@@ -111,12 +121,18 @@ class Clocks:
         except Exception:
             self.proc = None
         import threading
-        self.stop_flag = False
-        self.max_mhz = None
+        self.ready = threading.Event()
         self.thread = threading.Thread(target=self._poll, daemon=True)
         self.thread.start()
+        self.ready.wait(timeout=10)
+
+    def start(self):
+        if self.thread is None:
+            self.arm()
+        self.recording = True
 
     def stop(self):
+        self.recording = False
         if self.thread is not None:
             self.stop_flag = True
             self.thread.join(timeout=5)
@@ -275,12 +291,13 @@ def run_ours(args, wl, world, rank, local):
         if world > 1:
             dp.allreduce_weight_grad(dU)
 
+    clocks = Clocks(local)
+    clocks.arm()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     barrier(world)
     torch.cuda.synchronize()
-    clocks = Clocks(local)
     clocks.start()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     start = torch.cuda.Event(enable_timing=True)

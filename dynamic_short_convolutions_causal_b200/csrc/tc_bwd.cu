@@ -240,7 +240,9 @@ __device__ __forceinline__ Span span_of(const BwdParams &p) {
     return s;
 }
 
-template <int W, int G>
+// ROPE: the instantiation that rotates dy back (dsc_bwd_lowrank_rope); the plain one has
+// no RoPE code.
+template <int W, int G, bool ROPE>
 __global__ void __launch_bounds__(kThreads, 1)
 k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constant__ CUtensorMap tm_x,
                  const __grid_constant__ CUtensorMap tm_z, const __grid_constant__ CUtensorMap tm_u,
@@ -509,14 +511,16 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             if (!warp_wait(bar.full(st), n & 1, abort, 64u, &g_fault_bwd, p.wt.wait_ns)) { ok = false; break; }
             const uint32_t dys = sb + st * p.stage_bytes, xs = dys + p.xy_tile_bytes;
 
-            // ---- RoPE (when on): dy arrives as the gradient of the rotated output; each
-            // thread rotates its own row of the stage's dy tile back in place (the
-            // transpose: pair (2i, 2i+1) by minus its angle), lanes 0..W-2 of quarter 0
-            // also the tile's W-1 future-halo rows.  A2 reads only its own row; A1 reads
-            // neighbours' rows and waits for every warp (dyrot) first.
+            // ---- RoPE (when on): dy arrives as the gradient of the rotated output and is
+            // rotated back in the stage's dy tile (the transpose: pair (2i, 2i+1) by minus
+            // its angle) before A1, which reads neighbours' rows, waits for every warp
+            // (dyrot).  For G >= 8 each thread rotates its own row here (lanes 0..W-2 of
+            // quarter 0 also the tile's W-1 future-halo rows) and A2 reads only that row;
+            // for G < 8 A2's threads rotate the rows they read (below).
+            constexpr bool kRowPairs = G < 8;
             const int cslice = (sp.s0 + j) * kDt;
-            const bool rope = p.n_rot > 0 && cslice < p.n_rot;
-            if (rope) {
+            const bool rope = ROPE && cslice < p.n_rot;
+            if (!kRowPairs && rope) {
                 const int c16 = cslice + kCPW * h;
                 if (c16 < p.n_rot) {
                     auto unrotate = [&](int r) {
@@ -555,59 +559,17 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
             }
 
             // ---- A2: dw[t,g,k] = sum_{c in g} dy[t,c] x[t-k,c], tap-major column k*NG + g.
-            // When they fit in registers the values of both chunks are computed before
-            // the wait: only their stores need the previous tile's dz / dU MMAs to be done
-            // with the dw tile.
+            // For G < 8 a thread takes one 8-channel chunk (a2c) of two token rows (a2t,
+            // a2t+1): one pass over the tile's x rows a2t .. a2t+W serves both rows' W taps
+            // (W+3 row loads for two rows instead of 2W+2; lowrank_qkv 0.217 -> 0.210 ms,
+            // lowrank_mlp 0.463 -> 0.426 ms).  It reads other threads' dy rows, so with RoPE
+            // every warp's rotation is waited for first.  When they fit in registers the
+            // values are computed before the dwfree wait: only their stores need the
+            // previous tile's dz / dU MMAs to be done with the dw tile.
             constexpr int NPK = (NG8 + 1) / 2;           // packed bf16 pairs per (chunk, tap)
-            constexpr bool kPre = CH * W * NPK <= 32;
-            auto a2_compute = [&](int cq, uint32_t (&pk)[W][NPK]) {
-                const uint4 d0 = lds128(dys + (dyr[0] ^ ((uint32_t)cq << 4)));
-                uint4 xu[W];
-#pragma unroll
-                for (int k = 0; k < W; ++k) xu[k] = lds128(xs + (xr[k] ^ ((uint32_t)cq << 4)));
-#pragma unroll
-                for (int k = 0; k < W; ++k) {
-                    if constexpr (G == 1) {
-                        // one channel per group: dw = dy * x, exact in fp32 and rounded once
-                        // to bf16, which is what the packed bf16 multiply computes
-                        pk[k][0] = bf16x2_mul(d0.x, xu[k].x);
-                        pk[k][1] = bf16x2_mul(d0.y, xu[k].y);
-                        pk[k][2] = bf16x2_mul(d0.z, xu[k].z);
-                        pk[k][3] = bf16x2_mul(d0.w, xu[k].w);
-                    } else if constexpr (G <= 4) {
-                        const uint32_t dq[4] = {d0.x, d0.y, d0.z, d0.w};
-                        const uint32_t xq[4] = {xu[k].x, xu[k].y, xu[k].z, xu[k].w};
-                        float dw[NG8];
-#pragma unroll
-                        for (int gl = 0; gl < NG8; ++gl) {
-                            float acc = 0.f;
-#pragma unroll
-                            for (int e = gl * G; e < (gl + 1) * G; ++e)
-                                acc = (e & 1) ? fma_bf16_hi(dq[e >> 1], xq[e >> 1], acc) : fma_bf16_lo(dq[e >> 1], xq[e >> 1], acc);
-                            dw[gl] = acc;
-                        }
-#pragma unroll
-                        for (int m2 = 0; m2 < NG8 / 2; ++m2) pk[k][m2] = pack_bf16x2(dw[2 * m2], dw[2 * m2 + 1]);
-                    }
-                }
-            };
-            auto a2_store = [&](int cq, const uint32_t (&pk)[W][NPK]) {
-                const int g8 = (kCPW * h + 8 * cq) / G;
-#pragma unroll
-                for (int k = 0; k < W; ++k) {
-                    const int jp = k * NGS + g8;                      // first tap-major column
-                    const uint32_t atom = (uint32_t)(jp >> 6), within = (uint32_t)(jp & 63);
-                    const uint32_t a = dwrow + atom * 16384u + ((((within >> 3) << 4) ^ dwsw) | ((within & 7) * 2));
-                    if constexpr (NG8 == 8) {
-                        sts128(a, make_uint4(pk[k][0], pk[k][1], pk[k][2], pk[k][3]));
-                    } else if constexpr (NG8 == 4) {
-                        sts64(a, pk[k][0], pk[k][1]);
-                    } else {
-                        sts32(a, pk[k][0]);
-                    }
-                }
-            };
-            if constexpr (G >= 8) {
+            // (the products of both rows, next to the x window of W+1 rows, in registers)
+            constexpr bool kPre = 2 * W * NPK <= 32 && 2 * W * NPK + 4 * (W + 1) <= 52;
+            if constexpr (!kRowPairs) {
                 // one value per (virtual group, tap): GV = 8 gives one per chunk, and the
                 // two chunks' groups are adjacent columns; GV = 16 gives one per warp
                 float sv[CH][W];
@@ -639,20 +601,129 @@ k_tc_lowrank_bwd(const __grid_constant__ CUtensorMap tm_dy, const __grid_constan
                         sts16(a, (uint16_t)(pr & 0xffffu));
                     }
                 }
-            } else if constexpr (kPre) {
-                uint32_t pk[CH][W][NPK];
-#pragma unroll
-                for (int cq = 0; cq < CH; ++cq) a2_compute(cq, pk[cq]);
-                if (!warp_wait(bar.dwfree(), (i & 1) ^ 1, abort, 32u, &g_fault_bwd, p.wt.wait_ns)) { ok = false; break; }
-#pragma unroll
-                for (int cq = 0; cq < CH; ++cq) a2_store(cq, pk[cq]);
             } else {
-                if (!warp_wait(bar.dwfree(), (i & 1) ^ 1, abort, 32u, &g_fault_bwd, p.wt.wait_ns)) { ok = false; break; }
-#pragma unroll 1
-                for (int cq = 0; cq < CH; ++cq) {
-                    uint32_t pk[W][NPK];
-                    a2_compute(cq, pk);
-                    a2_store(cq, pk);
+                const int ee = ew * 32 + lane;
+                const int a2c = ee & 7, a2t = 2 * (ee >> 3);
+                auto raddr = [&](int r) {
+                    return ((uint32_t)r * 128u) ^ (((uint32_t)r & 7u) << 4) ^ ((uint32_t)a2c << 4);
+                };
+                uint4 xw[W + 1], d2[2];
+#pragma unroll
+                for (int ii = 0; ii < 2; ++ii) d2[ii] = lds128(dys + raddr(a2t + ii));
+                if (rope) {
+                    // rotate this thread's chunk of rows a2t, a2t+1 back (A2 uses the
+                    // registers, A1 the copy written back), threads ee < 8(W-1) also one
+                    // chunk of a future-halo row; then release A1 (dyrot)
+                    const int c8 = cslice + 8 * a2c;
+                    if (c8 < p.n_rot) {
+                        const float2 *csp = reinterpret_cast<const float2 *>(p.cs) + (size_t)((c8 % p.dh) / 2) * p.T;
+                        // every table load is issued before the first use (one round trip)
+                        const int tb = w.t0();
+                        const bool halo = ee < 8 * (W - 1);
+                        const int rh = kTt + (ee >> 3);                 // the halo row, if any
+                        const int toks[3] = {tb + a2t, tb + a2t + 1, tb + rh};
+                        const bool live[3] = {toks[0] < p.T, toks[1] < p.T, halo && toks[2] < p.T};
+                        float2 c[3][4];
+#pragma unroll
+                        for (int ii = 0; ii < 3; ++ii)
+#pragma unroll
+                            for (int m2 = 0; m2 < 4; ++m2)
+                                c[ii][m2] = live[ii] ? __ldg(csp + (size_t)m2 * p.T + toks[ii]) : make_float2(1.f, 0.f);
+                        uint4 uh = make_uint4(0u, 0u, 0u, 0u);
+                        if (live[2]) uh = lds128(dys + raddr(rh));
+                        auto unrot = [&](uint4 &u, const float2 (&cc)[4]) {
+                            float v[8];
+                            unpack8(u, v);
+#pragma unroll
+                            for (int m2 = 0; m2 < 4; ++m2) {
+                                const float e0 = v[2 * m2], e1 = v[2 * m2 + 1];
+                                v[2 * m2] = fmaf(e0, cc[m2].x, e1 * cc[m2].y);
+                                v[2 * m2 + 1] = fmaf(e1, cc[m2].x, -e0 * cc[m2].y);
+                            }
+                            u = make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                           pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+                        };
+                        // rows past the sequence's end stay zero
+#pragma unroll
+                        for (int ii = 0; ii < 2; ++ii) {
+                            if (live[ii]) {
+                                unrot(d2[ii], c[ii]);
+                                sts128(dys + raddr(a2t + ii), d2[ii]);
+                            }
+                        }
+                        if (live[2]) {
+                            unrot(uh, c[2]);
+                            sts128(dys + raddr(rh), uh);
+                        }
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar.dyrot());
+                }
+#pragma unroll
+                for (int jj = 0; jj <= W; ++jj) xw[jj] = lds128(xs + raddr(a2t + jj));
+                // dw of row a2t+ii, tap k: dy row a2t+ii times x tile row a2t+ii+W-1-k
+                auto product = [&](int ii, int k, uint32_t (&pk)[NPK]) {
+                    const uint4 &d0 = d2[ii];
+                    const uint4 &xk = xw[ii + W - 1 - k];
+                    if constexpr (G == 1) {
+                        // one channel per group: dw = dy * x, exact in fp32 and rounded once
+                        // to bf16, which is what the packed bf16 multiply computes
+                        pk[0] = bf16x2_mul(d0.x, xk.x);
+                        pk[1] = bf16x2_mul(d0.y, xk.y);
+                        pk[2] = bf16x2_mul(d0.z, xk.z);
+                        pk[3] = bf16x2_mul(d0.w, xk.w);
+                    } else {
+                        const uint32_t dq[4] = {d0.x, d0.y, d0.z, d0.w};
+                        const uint32_t xq[4] = {xk.x, xk.y, xk.z, xk.w};
+                        float dwv[NG8];
+#pragma unroll
+                        for (int gl = 0; gl < NG8; ++gl) {
+                            float acc = 0.f;
+#pragma unroll
+                            for (int e = gl * G; e < (gl + 1) * G; ++e)
+                                acc = (e & 1) ? fma_bf16_hi(dq[e >> 1], xq[e >> 1], acc) : fma_bf16_lo(dq[e >> 1], xq[e >> 1], acc);
+                            dwv[gl] = acc;
+                        }
+#pragma unroll
+                        for (int m2 = 0; m2 < NG8 / 2; ++m2) pk[m2] = pack_bf16x2(dwv[2 * m2], dwv[2 * m2 + 1]);
+                    }
+                };
+                const int g8 = (8 * a2c) / G;
+                auto store = [&](int ii, int k, const uint32_t (&pk)[NPK]) {
+                    const uint32_t t = (uint32_t)(a2t + ii);
+                    const int jp = k * NGS + g8;                      // first tap-major column
+                    const uint32_t atom = (uint32_t)(jp >> 6), within = (uint32_t)(jp & 63);
+                    const uint32_t a = sb + p.off_dw + t * 128u + atom * 16384u +
+                                       ((((within >> 3) << 4) ^ ((t & 7u) << 4)) | ((within & 7) * 2));
+                    if constexpr (NG8 == 8) {
+                        sts128(a, make_uint4(pk[0], pk[1], pk[2], pk[3]));
+                    } else if constexpr (NG8 == 4) {
+                        sts64(a, pk[0], pk[1]);
+                    } else {
+                        sts32(a, pk[0]);
+                    }
+                };
+                if constexpr (kPre) {
+                    uint32_t pk[2][W][NPK];
+#pragma unroll
+                    for (int ii = 0; ii < 2; ++ii)
+#pragma unroll
+                        for (int k = 0; k < W; ++k) product(ii, k, pk[ii][k]);
+                    if (!warp_wait(bar.dwfree(), (i & 1) ^ 1, abort, 32u, &g_fault_bwd, p.wt.wait_ns)) { ok = false; break; }
+#pragma unroll
+                    for (int ii = 0; ii < 2; ++ii)
+#pragma unroll
+                        for (int k = 0; k < W; ++k) store(ii, k, pk[ii][k]);
+                } else {
+                    if (!warp_wait(bar.dwfree(), (i & 1) ^ 1, abort, 32u, &g_fault_bwd, p.wt.wait_ns)) { ok = false; break; }
+#pragma unroll
+                    for (int ii = 0; ii < 2; ++ii)
+#pragma unroll
+                        for (int k = 0; k < W; ++k) {
+                            uint32_t pk[NPK];
+                            product(ii, k, pk);
+                            store(ii, k, pk);
+                        }
                 }
             }
             fence_proxy_async_smem();
@@ -1049,7 +1120,7 @@ bool plan_bwd(int B, int T, int D, int G, int W, int R, int nsm, BwdParams &p) {
 
 template <int W, int G>
 cudaError_t launch_t(const CUtensorMap *m, const BwdParams &p, cudaStream_t s) {
-    auto kern = k_tc_lowrank_bwd<W, G>;
+    auto kern = p.n_rot > 0 ? k_tc_lowrank_bwd<W, G, true> : k_tc_lowrank_bwd<W, G, false>;
     const uint32_t smem = smem_bytes(p);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
