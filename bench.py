@@ -423,122 +423,138 @@ def measure_comparators(dsc, dev, peak, args):
         return {"ms": ms, "algorithmic_bytes": nbytes, "gbs": gbs, "frac_of_peak": gbs / peak,
                 "tokens_per_s": tokens / (ms * 1e-3)}
 
-    # static depthwise causal conv, fwd + bwd, on the MLP-width shape
-    wl = di.WORKLOADS["lowrank_mlp"]
-    t = di.make(wl, dev, ("x", "dy", "ws"))
-    x, dy, w = t["x"], t["dy"], t["ws"]
-    y = torch.empty_like(x)
-    dx = torch.empty_like(x)
-    dw = torch.empty((wl.D, wl.W), dtype=torch.float32, device=dev)
-    ws = dsc.workspace(dsc.dsc_static_bwd_workspace_bytes(wl.B, wl.T, wl.D, wl.W), dev)
-    act = wl.tokens * wl.D * 2
-    fwd_ms = _time_calls(lambda: dsc.dsc_static_fwd(x, w, y), stream, steps)
-    bwd_ms = _time_calls(lambda: dsc.dsc_static_bwd(x, w, dy, dx, dw, ws), stream, steps)
-    sb_f = 2 * act + wl.D * wl.W * 2
-    sb_b = 3 * act + wl.D * wl.W * (2 + 4)
-    out["static_conv_" + wl.name] = {
-        "shape": {"B": wl.B, "T": wl.T, "D": wl.D, "W": wl.W},
-        "fwd": entry(fwd_ms, sb_f, wl.tokens), "bwd": entry(bwd_ms, sb_b, wl.tokens),
-        "fwd_bwd": entry(fwd_ms + bwd_ms, sb_f + sb_b, wl.tokens)}
-    del t, x, dy, w, y, dx, dw, ws
+    names = {"static", "mlp", "rope", "explicit", "decode"}
+    chosen = names if args.comparators == "all" else set(args.comparators.split(","))
+    if chosen - names:
+        raise SystemExit("--comparators: unknown %s (choose from %s)" % (sorted(chosen - names), sorted(names)))
 
-    # fused low-rank fwd + bwd on the MLP-width shape
-    t = di.make(wl, dev, ("x", "z", "U", "dy"))
-    x, z, U, dy = t["x"], t["z"], t["U"], t["dy"]
-    y = torch.empty_like(x)
-    dx = torch.empty_like(x)
-    dz = torch.empty((wl.B, wl.T, wl.R), dtype=torch.float32, device=dev)
-    dU = torch.empty((wl.R, wl.N), dtype=torch.float32, device=dev)
-    ws = dsc.workspace(dsc.dsc_bwd_lowrank_workspace_bytes(wl.B, wl.T, wl.D, wl.G, wl.W, wl.R), dev)
-    fwd_ms = _time_calls(lambda: dsc.dsc_fwd_lowrank(x, z, U, y, wl.G, wl.W), stream, steps)
-    bwd_ms = _time_calls(lambda: dsc.dsc_bwd_lowrank(x, z, U, dy, dx, dz, dU, ws, wl.G, wl.W), stream, steps)
-    fb, bb = algorithmic_bytes(wl)
-    out["lowrank_" + wl.name.split("_", 1)[1]] = {
-        "shape": {"B": wl.B, "T": wl.T, "D": wl.D, "G": wl.G, "W": wl.W, "R": wl.R},
-        "fwd": entry(fwd_ms, fb, wl.tokens), "bwd": entry(bwd_ms, bb, wl.tokens),
-        "fwd_bwd": entry(fwd_ms + bwd_ms, fb + bb, wl.tokens),
-        "path": dsc.dsc_lowrank_path(wl.B, wl.T, wl.D, wl.G, wl.W, wl.R)}
-    del t, x, z, U, dy, y, dx, dz, dU, ws
+    def want(name):
+        return name in chosen
 
-    # the stacked-QKV step with RoPE fused on Q and K (heads of 128 channels): the op's
-    # output rotated before it is stored, and the backward from the rotated gradient
-    wl = di.WORKLOADS["lowrank_qkv"]
-    t = di.make(wl, dev, ("x", "z", "U", "dy"))
-    x, z, U, dy = t["x"], t["z"], t["U"], t["dy"]
-    dh, n_rot = 128, 2 * wl.D // 3
-    inv = 10000.0 ** (-torch.arange(0, dh, 2, dtype=torch.float64, device=dev) / dh)
-    th = torch.arange(wl.T, dtype=torch.float64, device=dev)[:, None] * inv[None, :]
-    cs = torch.stack([torch.cos(th), torch.sin(th)], dim=-1).to(torch.float32).permute(1, 0, 2).contiguous()
-    y = torch.empty_like(x)
-    dx = torch.empty_like(x)
-    dz = torch.empty((wl.B, wl.T, wl.R), dtype=torch.float32, device=dev)
-    dU = torch.empty((wl.R, wl.N), dtype=torch.float32, device=dev)
-    ws = dsc.workspace(dsc.dsc_bwd_lowrank_workspace_bytes(wl.B, wl.T, wl.D, wl.G, wl.W, wl.R), dev)
-    fwd_ms = _time_calls(lambda: dsc.dsc_fwd_lowrank_rope(x, z, U, cs, y, wl.G, wl.W, dh, n_rot), stream, steps)
-    bwd_ms = _time_calls(lambda: dsc.dsc_bwd_lowrank_rope(x, z, U, cs, dy, dx, dz, dU, ws, wl.G, wl.W, dh, n_rot),
-                         stream, steps)
-    fb, bb = algorithmic_bytes(wl)
-    out["lowrank_rope_" + wl.name.split("_", 1)[1]] = {
-        "shape": {"B": wl.B, "T": wl.T, "D": wl.D, "G": wl.G, "W": wl.W, "R": wl.R, "dh": dh, "n_rot": n_rot},
-        "fwd": entry(fwd_ms, fb, wl.tokens), "bwd": entry(bwd_ms, bb, wl.tokens),
-        "fwd_bwd": entry(fwd_ms + bwd_ms, fb + bb, wl.tokens),
-        "note": "bytes exclude the 0.5 MB RoPE table; a separate rotation pass would add 4 x 134 MB"}
-    del t, x, z, U, dy, y, dx, dz, dU, ws, cs
-
-    # explicit-filter forward and backward on the stacked-QKV shape
-    wl = di.WORKLOADS["tied_qkv"]
-    t = di.make(wl, dev, ("x", "w", "dy"))
-    x, w, dy = t["x"], t["w"], t["dy"]
-    y = torch.empty_like(x)
-    ms = _time_calls(lambda: dsc.dsc_fwd(x, w, y, wl.G), stream, steps)
-    nb = 2 * wl.tokens * wl.D * 2 + wl.tokens * wl.NG * wl.W * 2
-    dx = torch.empty_like(x)
-    dw = torch.empty((wl.B, wl.T, wl.NG, wl.W), dtype=torch.float32, device=dev)
-    ms_b = _time_calls(lambda: dsc.dsc_bwd(x, w, dy, dx, dw, wl.G), stream, steps)
-    nb_b = 3 * wl.tokens * wl.D * 2 + wl.tokens * wl.NG * wl.W * (2 + 4)   # x, dy, dx; w in, dw out (fp32)
-    out["explicit_" + wl.name] = {"shape": {"B": wl.B, "T": wl.T, "D": wl.D, "G": wl.G, "W": wl.W},
-                                  "fwd": entry(ms, nb, wl.tokens), "bwd": entry(ms_b, nb_b, wl.tokens)}
-    del t, x, w, dy, y, dx, dw
-
-    # decode step (one token per sequence, rolling window) on the stacked-QKV width
-    wl = di.WORKLOADS["lowrank_qkv"]
-    D, G, W, R, N = wl.D, wl.G, wl.W, wl.R, wl.N
-    gen = torch.Generator(device=dev)
-    gen.manual_seed(wl.seed)
-    U = (torch.randn((R, N), generator=gen, device=dev) * R ** -0.5).to(torch.bfloat16)
-    dec = {}
-    for B in (1, 8, 64, 256, 512):
-        x = torch.randn((B, D), generator=gen, device=dev).to(torch.bfloat16)
-        z = torch.randn((B, R), generator=gen, device=dev).to(torch.bfloat16)
-        st = torch.randn((B, W - 1, D), generator=gen, device=dev).to(torch.bfloat16)
+    if want("static"):
+        # static depthwise causal conv, fwd + bwd, on the MLP-width shape
+        wl = di.WORKLOADS["lowrank_mlp"]
+        t = di.make(wl, dev, ("x", "dy", "ws"))
+        x, dy, w = t["x"], t["dy"], t["ws"]
         y = torch.empty_like(x)
-        ms = _time_graph(lambda: dsc.dsc_decode_step_lowrank(x, z, U, st, y, G, W), dev, 100)
-        nb = R * N * 2 + B * (D * 2 + R * 2 + 2 * (W - 1) * D * 2 + D * 2)
-        fl = B * (2 * R * N + 2 * W * D)
-        dec["B=%d" % B] = {"us": ms * 1e3, "algorithmic_bytes": nb, "gbs": nb / (ms * 1e-3) / 1e9,
-                           "frac_of_hbm_peak": nb / (ms * 1e-3) / 1e9 / peak,
-                           "tflops": fl / (ms * 1e-3) / 1e12, "tokens_per_s": B / (ms * 1e-3)}
-    out["decode_lowrank_" + wl.name.split("_", 1)[1]] = {
-        "shape": {"D": D, "G": G, "W": W, "R": R}, "per_batch": dec,
-        "note": "device time per step: 100 steps captured in a CUDA graph and replayed (a "
-                "generation loop's launch pattern), inputs and window resident in HBM; from "
-                "B = 8 the step is the fused forward's tensor-core kernel with one row per "
-                "sequence (w = z U by tcgen05, window moved by TMA stores), below it a "
-                "CUDA-core kernel"}
-    del U, x, z, st, y
-    torch.cuda.empty_cache()
+        dx = torch.empty_like(x)
+        dw = torch.empty((wl.D, wl.W), dtype=torch.float32, device=dev)
+        ws = dsc.workspace(dsc.dsc_static_bwd_workspace_bytes(wl.B, wl.T, wl.D, wl.W), dev)
+        act = wl.tokens * wl.D * 2
+        fwd_ms = _time_calls(lambda: dsc.dsc_static_fwd(x, w, y), stream, steps)
+        bwd_ms = _time_calls(lambda: dsc.dsc_static_bwd(x, w, dy, dx, dw, ws), stream, steps)
+        sb_f = 2 * act + wl.D * wl.W * 2
+        sb_b = 3 * act + wl.D * wl.W * (2 + 4)
+        out["static_conv_" + wl.name] = {
+            "shape": {"B": wl.B, "T": wl.T, "D": wl.D, "W": wl.W},
+            "fwd": entry(fwd_ms, sb_f, wl.tokens), "bwd": entry(bwd_ms, sb_b, wl.tokens),
+            "fwd_bwd": entry(fwd_ms + bwd_ms, sb_f + sb_b, wl.tokens)}
+        del t, x, dy, w, y, dx, dw, ws
+
+    if want("mlp"):
+        # fused low-rank fwd + bwd on the MLP-width shape
+        t = di.make(wl, dev, ("x", "z", "U", "dy"))
+        x, z, U, dy = t["x"], t["z"], t["U"], t["dy"]
+        y = torch.empty_like(x)
+        dx = torch.empty_like(x)
+        dz = torch.empty((wl.B, wl.T, wl.R), dtype=torch.float32, device=dev)
+        dU = torch.empty((wl.R, wl.N), dtype=torch.float32, device=dev)
+        ws = dsc.workspace(dsc.dsc_bwd_lowrank_workspace_bytes(wl.B, wl.T, wl.D, wl.G, wl.W, wl.R), dev)
+        fwd_ms = _time_calls(lambda: dsc.dsc_fwd_lowrank(x, z, U, y, wl.G, wl.W), stream, steps)
+        bwd_ms = _time_calls(lambda: dsc.dsc_bwd_lowrank(x, z, U, dy, dx, dz, dU, ws, wl.G, wl.W), stream, steps)
+        fb, bb = algorithmic_bytes(wl)
+        out["lowrank_" + wl.name.split("_", 1)[1]] = {
+            "shape": {"B": wl.B, "T": wl.T, "D": wl.D, "G": wl.G, "W": wl.W, "R": wl.R},
+            "fwd": entry(fwd_ms, fb, wl.tokens), "bwd": entry(bwd_ms, bb, wl.tokens),
+            "fwd_bwd": entry(fwd_ms + bwd_ms, fb + bb, wl.tokens),
+            "path": dsc.dsc_lowrank_path(wl.B, wl.T, wl.D, wl.G, wl.W, wl.R)}
+        del t, x, z, U, dy, y, dx, dz, dU, ws
+
+    if want("rope"):
+        # the stacked-QKV step with RoPE fused on Q and K (heads of 128 channels): the op's
+        # output rotated before it is stored, and the backward from the rotated gradient
+        wl = di.WORKLOADS["lowrank_qkv"]
+        t = di.make(wl, dev, ("x", "z", "U", "dy"))
+        x, z, U, dy = t["x"], t["z"], t["U"], t["dy"]
+        dh, n_rot = 128, 2 * wl.D // 3
+        inv = 10000.0 ** (-torch.arange(0, dh, 2, dtype=torch.float64, device=dev) / dh)
+        th = torch.arange(wl.T, dtype=torch.float64, device=dev)[:, None] * inv[None, :]
+        cs = torch.stack([torch.cos(th), torch.sin(th)], dim=-1).to(torch.float32).permute(1, 0, 2).contiguous()
+        y = torch.empty_like(x)
+        dx = torch.empty_like(x)
+        dz = torch.empty((wl.B, wl.T, wl.R), dtype=torch.float32, device=dev)
+        dU = torch.empty((wl.R, wl.N), dtype=torch.float32, device=dev)
+        ws = dsc.workspace(dsc.dsc_bwd_lowrank_workspace_bytes(wl.B, wl.T, wl.D, wl.G, wl.W, wl.R), dev)
+        fwd_ms = _time_calls(lambda: dsc.dsc_fwd_lowrank_rope(x, z, U, cs, y, wl.G, wl.W, dh, n_rot), stream, steps)
+        bwd_ms = _time_calls(lambda: dsc.dsc_bwd_lowrank_rope(x, z, U, cs, dy, dx, dz, dU, ws, wl.G, wl.W, dh, n_rot),
+                             stream, steps)
+        fb, bb = algorithmic_bytes(wl)
+        out["lowrank_rope_" + wl.name.split("_", 1)[1]] = {
+            "shape": {"B": wl.B, "T": wl.T, "D": wl.D, "G": wl.G, "W": wl.W, "R": wl.R, "dh": dh, "n_rot": n_rot},
+            "fwd": entry(fwd_ms, fb, wl.tokens), "bwd": entry(bwd_ms, bb, wl.tokens),
+            "fwd_bwd": entry(fwd_ms + bwd_ms, fb + bb, wl.tokens),
+            "note": "bytes exclude the 0.5 MB RoPE table; a separate rotation pass would add 4 x 134 MB"}
+        del t, x, z, U, dy, y, dx, dz, dU, ws, cs
+
+    if want("explicit"):
+        # explicit-filter forward and backward on the stacked-QKV shape
+        wl = di.WORKLOADS["tied_qkv"]
+        t = di.make(wl, dev, ("x", "w", "dy"))
+        x, w, dy = t["x"], t["w"], t["dy"]
+        y = torch.empty_like(x)
+        ms = _time_calls(lambda: dsc.dsc_fwd(x, w, y, wl.G), stream, steps)
+        nb = 2 * wl.tokens * wl.D * 2 + wl.tokens * wl.NG * wl.W * 2
+        dx = torch.empty_like(x)
+        dw = torch.empty((wl.B, wl.T, wl.NG, wl.W), dtype=torch.float32, device=dev)
+        ms_b = _time_calls(lambda: dsc.dsc_bwd(x, w, dy, dx, dw, wl.G), stream, steps)
+        nb_b = 3 * wl.tokens * wl.D * 2 + wl.tokens * wl.NG * wl.W * (2 + 4)   # x, dy, dx; w in, dw out (fp32)
+        out["explicit_" + wl.name] = {"shape": {"B": wl.B, "T": wl.T, "D": wl.D, "G": wl.G, "W": wl.W},
+                                      "fwd": entry(ms, nb, wl.tokens), "bwd": entry(ms_b, nb_b, wl.tokens)}
+        del t, x, w, dy, y, dx, dw
+
+    if want("decode"):
+        # decode step (one token per sequence, rolling window) on the stacked-QKV width
+        wl = di.WORKLOADS["lowrank_qkv"]
+        D, G, W, R, N = wl.D, wl.G, wl.W, wl.R, wl.N
+        gen = torch.Generator(device=dev)
+        gen.manual_seed(wl.seed)
+        U = (torch.randn((R, N), generator=gen, device=dev) * R ** -0.5).to(torch.bfloat16)
+        dec = {}
+        for B in (1, 8, 64, 256, 512):
+            x = torch.randn((B, D), generator=gen, device=dev).to(torch.bfloat16)
+            z = torch.randn((B, R), generator=gen, device=dev).to(torch.bfloat16)
+            st = torch.randn((B, W - 1, D), generator=gen, device=dev).to(torch.bfloat16)
+            y = torch.empty_like(x)
+            ms = _time_graph(lambda: dsc.dsc_decode_step_lowrank(x, z, U, st, y, G, W), dev, 100)
+            nb = R * N * 2 + B * (D * 2 + R * 2 + 2 * (W - 1) * D * 2 + D * 2)
+            fl = B * (2 * R * N + 2 * W * D)
+            dec["B=%d" % B] = {"us": ms * 1e3, "algorithmic_bytes": nb, "gbs": nb / (ms * 1e-3) / 1e9,
+                               "frac_of_hbm_peak": nb / (ms * 1e-3) / 1e9 / peak,
+                               "tflops": fl / (ms * 1e-3) / 1e12, "tokens_per_s": B / (ms * 1e-3)}
+        out["decode_lowrank_" + wl.name.split("_", 1)[1]] = {
+            "shape": {"D": D, "G": G, "W": W, "R": R}, "per_batch": dec,
+            "note": "device time per step: 100 steps captured in a CUDA graph and replayed (a "
+                    "generation loop's launch pattern), inputs and window resident in HBM; from "
+                    "B = 8 the step is the fused forward's tensor-core kernel with one row per "
+                    "sequence (w = z U by tcgen05, window moved by TMA stores), below it a "
+                    "CUDA-core kernel"}
+        del U, x, z, st, y
+        torch.cuda.empty_cache()
     return out
 
 
 def source_hash():
-    """Hash of the library's kernel and ABI sources (csrc/ and include/): a stored ncu
-    traffic figure is reported only for the build it was measured on."""
+    """Hash of the sources the tensor-core calls are built from (their kernels, the
+    headers they include, the entry points that dispatch to them, include/): a stored
+    ncu traffic figure for dsc_fwd_lowrank / dsc_bwd_lowrank is reported only for the
+    build it was measured on.  The CUDA-core kernels (stream.cu, simt.cu, decode.cu,
+    halo.cu) are not part of those calls."""
     import glob
     import hashlib
     h = hashlib.sha256()
     pkg = os.path.join(ROOT, "dynamic_short_convolutions_causal_b200", "csrc")
-    files = sorted(glob.glob(os.path.join(pkg, "*.cu")) + glob.glob(os.path.join(pkg, "*.cuh")) +
-                   glob.glob(os.path.join(pkg, "*.h")) + glob.glob(os.path.join(ROOT, "include", "*.h")))
+    names = ["common.cuh", "tc_common.cuh", "tc_lowrank.cu", "tc_bwd.cu", "internal.h", "dsc_api.cu"]
+    files = sorted([os.path.join(pkg, n) for n in names] + glob.glob(os.path.join(ROOT, "include", "*.h")))
     for p in files:
         h.update(os.path.basename(p).encode())
         with open(p, "rb") as fh:
@@ -671,6 +687,8 @@ def main(argv=None):
     ap.add_argument("--ref-budget", type=float, default=120.0,
                     help="seconds of oracle work for the whole reference run (warm-up + steps)")
     ap.add_argument("--no-comparators", action="store_true")
+    ap.add_argument("--comparators", default="all",
+                    help="comma list of static,mlp,rope,explicit,decode (default all)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -15,6 +15,15 @@
 // warp reads 32*V consecutive channels of a row (whole 128-byte lines), and the
 // staging layout interleaves the threads so that their shared-memory reads do not
 // conflict.  V shrinks as W grows, so that the taps and row windows stay in registers.
+// Two things keep the instruction count and the registers down (measured on B200):
+//   - bf16 rows and taps stay packed, two channels a word, and every product is a
+//     mixed fma.rn.f32.bf16 (exact product, one rounding: the results of widening
+//     first): 8-tap static forward of the MLP-width shape 0.133 -> 0.111 ms, its
+//     backward 0.272 -> 0.222 ms, tied-filter forward / backward of the stacked-QKV
+//     shape 0.083 -> 0.074 / 0.162 -> 0.143 ms;
+//   - the row window is a ring when a batch is a whole number of windows: row t sits
+//     in slot (t - t0) % W, a constant in each unrolled step, so no row is copied
+//     (0.141 -> 0.134 ms and 0.283 -> 0.272 ms on the static forward / backward).
 #include "common.cuh"
 #include "internal.h"
 
@@ -192,22 +201,6 @@ __device__ __forceinline__ void stream_fwd_item(const T *__restrict__ x, const T
     T *yb = y + (size_t)b * T_ * D + c0;
     const bool tap_stage = kTapVec && (G % V == 0);
     const T *wb = STATIC ? w : w + ((size_t)b * T_ * (D / G) + c0 / G) * W;   // taps of token 0
-
-    float f[W][V];
-    if (STATIC && active) {
-#pragma unroll
-        for (int i = 0; i < V; ++i)
-#pragma unroll
-            for (int k = 0; k < W; ++k) f[k][i] = to_f(__ldg(w + (size_t)(c0 + i) * W + k));
-    }
-    float win[W][V];   // win[k] = x[t-k]
-#pragma unroll
-    for (int k = 1; k < W; ++k) {
-        if (active && t0 - k >= 0) P::unpack(P::load(xb + (size_t)(t0 - k) * D), win[k]);
-        else
-#pragma unroll
-            for (int i = 0; i < V; ++i) win[k][i] = 0.f;
-    }
     auto issue = [&](int tb, int stage) {
 #pragma unroll
         for (int u = 0; u < KU; ++u) {
@@ -219,7 +212,141 @@ __device__ __forceinline__ void stream_fwd_item(const T *__restrict__ x, const T
         }
         cp_commit();
     };
+    // The W-row window.  When a batch is a whole number of windows (KU % W == 0) and the
+    // chunk starts at a multiple of W, row t sits in slot t % W, a constant in every
+    // unrolled step, so no row is copied (ring); otherwise win[k] = x[t-k] and the rows
+    // move down one slot per token (shift).
+    constexpr bool kRing = KU % W == 0;
+    const bool ring = kRing && t0 % W == 0;
     const int nb = cdiv(t1 - t0, KU);
+
+    if constexpr (sizeof(T) == 2) {
+        if (STATIC || tap_stage) {
+            // bf16 with static or staged taps: rows and taps stay packed (two channels a
+            // word) and every product is a mixed fma.rn.f32.bf16 (exact product, one
+            // rounding: the results of widening first), fewer registers and no unpacking
+            constexpr int NW = V / 2;
+            using RT = typename P::raw_t;
+            auto words = [](const RT &r, uint32_t (&o)[NW]) {
+                const uint32_t *q = reinterpret_cast<const uint32_t *>(&r);
+#pragma unroll
+                for (int j = 0; j < NW; ++j) o[j] = q[j];
+            };
+            uint32_t fw[W][NW];      // static taps of channel pairs (w[c0+2j, k], w[c0+2j+1, k])
+            if (STATIC && active) {
+                const uint16_t *wr = reinterpret_cast<const uint16_t *>(w);
+#pragma unroll
+                for (int j = 0; j < NW; ++j)
+#pragma unroll
+                    for (int k = 0; k < W; ++k)
+                        fw[k][j] = (uint32_t)__ldg(wr + (size_t)(c0 + 2 * j) * W + k) |
+                                   ((uint32_t)__ldg(wr + (size_t)(c0 + 2 * j + 1) * W + k) << 16);
+            }
+            uint32_t win[W][NW];
+#pragma unroll
+            for (int k = 1; k < W; ++k) {
+                uint32_t r[NW];
+                if (active && t0 - k >= 0) words(P::load(xb + (size_t)(t0 - k) * D), r);
+                else
+#pragma unroll
+                    for (int j = 0; j < NW; ++j) r[j] = 0u;
+                const int sk = (kRing && ring) ? W - k : k;
+#pragma unroll
+                for (int j = 0; j < NW; ++j) win[sk][j] = r[j];
+            }
+            issue(t0, 0);
+            for (int bi = 0; bi < nb; ++bi) {
+                const int tb = t0 + bi * KU, stage = bi & 1;
+                if (bi + 1 < nb) issue(tb + KU, stage ^ 1);
+                else cp_commit();
+                cp_wait<1>();
+                if (!active) continue;
+                auto token = [&](int t, int u, auto sl) {
+                    words(lds_raw<RT>(stg.at(stage, 0, u)), win[sl(0)]);
+                    uint32_t tw[TB / 4 > 0 ? TB / 4 : 1];          // the token's taps, two a word
+                    (void)tw;
+                    if constexpr (kTapVec) {
+                        if (!STATIC) {
+                            using TR = typename RawOf<TB>::type;
+                            const TR tr = lds_raw<TR>(stg.at(stage, 1, u));
+                            const uint32_t *q = reinterpret_cast<const uint32_t *>(&tr);
+#pragma unroll
+                            for (int m = 0; m < TB / 4; ++m) tw[m] = q[m];
+                        }
+                    }
+                    float out[V];
+#pragma unroll
+                    for (int j = 0; j < NW; ++j) {
+                        const uint32_t xt = win[sl(0)][j];
+                        float a0 = bf16_lo(xt), a1 = bf16_hi(xt);
+#pragma unroll
+                        for (int k = 0; k < W; ++k) {
+                            const uint32_t xk = win[sl(k)][j];
+                            if constexpr (STATIC) {
+                                a0 = fma_bf16_sel<0, 0>(fw[k][j], xk, a0);
+                                a1 = fma_bf16_sel<1, 1>(fw[k][j], xk, a1);
+                            } else if ((k & 1) == 0) {
+                                a0 = fma_bf16_sel<0, 0>(tw[k / 2], xk, a0);
+                                a1 = fma_bf16_sel<0, 1>(tw[k / 2], xk, a1);
+                            } else {
+                                a0 = fma_bf16_sel<1, 0>(tw[k / 2], xk, a0);
+                                a1 = fma_bf16_sel<1, 1>(tw[k / 2], xk, a1);
+                            }
+                        }
+                        out[2 * j] = a0;
+                        out[2 * j + 1] = a1;
+                    }
+                    P::store(yb + (size_t)t * D, out);
+                };
+                if (kRing && ring) {
+#pragma unroll
+                    for (int u = 0; u < KU; ++u) {
+                        const int t = tb + u;
+                        if (t >= t1) break;
+                        token(t, u, [&](int k) { return (u - k + W) % W; });
+                    }
+                } else {
+#pragma unroll
+                    for (int u = 0; u < KU; ++u) {
+                        const int t = tb + u;
+                        if (t >= t1) break;
+                        token(t, u, [](int k) { return k; });
+#pragma unroll
+                        for (int k = W - 1; k >= 1; --k)
+#pragma unroll
+                            for (int j = 0; j < NW; ++j) win[k][j] = win[k - 1][j];
+                    }
+                }
+            }
+            cp_wait<0>();
+            return;
+        }
+    }
+
+    float f[W][V];
+    if (STATIC && active) {
+#pragma unroll
+        for (int i = 0; i < V; ++i)
+#pragma unroll
+            for (int k = 0; k < W; ++k) f[k][i] = to_f(__ldg(w + (size_t)(c0 + i) * W + k));
+    }
+    float win[W][V];
+#pragma unroll
+    for (int k = 1; k < W; ++k) {
+        float r[V];
+        if (active && t0 - k >= 0) P::unpack(P::load(xb + (size_t)(t0 - k) * D), r);
+        else
+#pragma unroll
+            for (int i = 0; i < V; ++i) r[i] = 0.f;
+        // row t0-k: slot (t0-k) % W = W-k in the ring, k in the shift
+        if (kRing && ring) {
+#pragma unroll
+            for (int i = 0; i < V; ++i) win[W - k][i] = r[i];
+        } else {
+#pragma unroll
+            for (int i = 0; i < V; ++i) win[k][i] = r[i];
+        }
+    }
     issue(t0, 0);
     for (int bi = 0; bi < nb; ++bi) {
         const int tb = t0 + bi * KU, stage = bi & 1;
@@ -227,11 +354,9 @@ __device__ __forceinline__ void stream_fwd_item(const T *__restrict__ x, const T
         else cp_commit();
         cp_wait<1>();
         if (!active) continue;
-#pragma unroll
-        for (int u = 0; u < KU; ++u) {
-            const int t = tb + u;
-            if (t >= t1) break;
-            P::unpack(lds_raw<typename P::raw_t>(stg.at(stage, 0, u)), win[0]);
+        // y[t] from the window (slot of row t-k: sl(k)) and the token's taps
+        auto token = [&](int t, int u, auto sl) {
+            P::unpack(lds_raw<typename P::raw_t>(stg.at(stage, 0, u)), win[sl(0)]);
             if constexpr (!STATIC) {
                 bool staged = false;
                 if constexpr (kTapVec) {
@@ -262,16 +387,31 @@ __device__ __forceinline__ void stream_fwd_item(const T *__restrict__ x, const T
             float out[V];
 #pragma unroll
             for (int i = 0; i < V; ++i) {
-                float acc = win[0][i];
+                float acc = win[sl(0)][i];
 #pragma unroll
-                for (int k = 0; k < W; ++k) acc = fmaf(f[k][i], win[k][i], acc);
+                for (int k = 0; k < W; ++k) acc = fmaf(f[k][i], win[sl(k)][i], acc);
                 out[i] = acc;
             }
             P::store(yb + (size_t)t * D, out);
+        };
+        if (kRing && ring) {
 #pragma unroll
-            for (int k = W - 1; k >= 1; --k)
+            for (int u = 0; u < KU; ++u) {
+                const int t = tb + u;
+                if (t >= t1) break;
+                token(t, u, [&](int k) { return (u - k + W) % W; });
+            }
+        } else {
 #pragma unroll
-                for (int i = 0; i < V; ++i) win[k][i] = win[k - 1][i];
+            for (int u = 0; u < KU; ++u) {
+                const int t = tb + u;
+                if (t >= t1) break;
+                token(t, u, [](int k) { return k; });
+#pragma unroll
+                for (int k = W - 1; k >= 1; --k)
+#pragma unroll
+                    for (int i = 0; i < V; ++i) win[k][i] = win[k - 1][i];
+            }
         }
     }
     cp_wait<0>();
@@ -330,6 +470,157 @@ k_dyn_bwd(const T *__restrict__ x, const T *__restrict__ w, const T *__restrict_
         const T *gb = dy + row0 * D + c0;
         T *ob = dx + row0 * D + c0;
         const T *wb = w + (row0 * NG + c0 / G) * W;
+        if constexpr (sizeof(T) == 2) {
+            // bf16: rows and taps stay packed (two channels a word), every product is a
+            // mixed fma.rn.f32.bf16 (the results of widening first).  Windows: a ring
+            // (row r in slot (r - t0) % W, constant in every unrolled step) when a batch is
+            // a whole number of windows, else shifted one slot per token.
+            constexpr int NW = V / 2;
+            using RT = typename P::raw_t;
+            auto words = [](const RT &r, uint32_t (&o)[NW]) {
+                const uint32_t *q = reinterpret_cast<const uint32_t *>(&r);
+#pragma unroll
+                for (int j = 0; j < NW; ++j) o[j] = q[j];
+            };
+            constexpr bool kRing = KU % W == 0;
+            const bool ring = kRing && t0 % W == 0;
+            float acc[W][V];                         // open dx rows (slot of row t-k: sl(k))
+            uint32_t xw[W][NW];                      // x rows, packed
+#pragma unroll
+            for (int k = 0; k < W; ++k)
+#pragma unroll
+                for (int i = 0; i < V; ++i) acc[k][i] = 0.f;
+#pragma unroll
+            for (int k = 1; k < W; ++k) {
+                uint32_t r[NW];
+                if (active && t0 - k >= 0) words(P::load(xb + (size_t)(t0 - k) * D), r);
+                else
+#pragma unroll
+                    for (int j = 0; j < NW; ++j) r[j] = 0u;
+                const int sk = (kRing && ring) ? W - k : k;
+#pragma unroll
+                for (int j = 0; j < NW; ++j) xw[sk][j] = r[j];
+            }
+            auto issue = [&](int tb, int stage) {
+#pragma unroll
+                for (int u = 0; u < KU; ++u) {
+                    const bool ok = active && tb + u < t1e;
+                    const int t = ok ? tb + u : t0;
+                    cp_async<P::BYTES>(stg.at(stage, 0, u), xb + (size_t)t * D, ok && tb + u < t1);
+                    cp_async<P::BYTES>(stg.at(stage, 1, u), gb + (size_t)t * D, ok);
+                    cp_async<TB>(stg.at(stage, 2, u), wb + (size_t)t * NG * W, ok);
+                }
+                cp_commit();
+            };
+            // token t: its rows and taps from the stage; sl(k) is the slot of row t-k
+            auto token = [&](int t, int stage, int u, auto sl) {
+                uint32_t gw[NW], tw[TB / 4];
+                words(lds_raw<RT>(stg.at(stage, 1, u)), gw);
+                words(lds_raw<RT>(stg.at(stage, 0, u)), xw[sl(0)]);
+                {
+                    const TR tr = lds_raw<TR>(stg.at(stage, 2, u));
+                    const uint32_t *q = reinterpret_cast<const uint32_t *>(&tr);
+#pragma unroll
+                    for (int m = 0; m < TB / 4; ++m) tw[m] = q[m];
+                }
+                // dx: row t opens with dy[t] (its slot held row t-W, stored a step ago),
+                // every open row t-k gets w[t,k] dy[t]; row t-W+1 is then complete
+#pragma unroll
+                for (int j = 0; j < NW; ++j) {
+                    acc[sl(0)][2 * j] = bf16_lo(gw[j]);
+                    acc[sl(0)][2 * j + 1] = bf16_hi(gw[j]);
+                }
+#pragma unroll
+                for (int k = 0; k < W; ++k)
+#pragma unroll
+                    for (int j = 0; j < NW; ++j) {
+                        float &a0 = acc[sl(k)][2 * j], &a1 = acc[sl(k)][2 * j + 1];
+                        if ((k & 1) == 0) {
+                            a0 = fma_bf16_sel<0, 0>(tw[k / 2], gw[j], a0);
+                            a1 = fma_bf16_sel<0, 1>(tw[k / 2], gw[j], a1);
+                        } else {
+                            a0 = fma_bf16_sel<1, 0>(tw[k / 2], gw[j], a0);
+                            a1 = fma_bf16_sel<1, 1>(tw[k / 2], gw[j], a1);
+                        }
+                    }
+                const int s = t - (W - 1);
+                if (active && s >= t0 && s < t1) P::store(ob + (size_t)s * D, acc[sl(W - 1)]);
+                // dw of token t (tokens of the chunk only)
+                if (t < t1) {
+                    float sw[W];
+#pragma unroll
+                    for (int k = 0; k < W; ++k) {
+                        float a = 0.f;
+#pragma unroll
+                        for (int j = 0; j < NW; ++j) {
+                            a = fma_bf16_sel<0, 0>(gw[j], xw[sl(k)][j], a);
+                            a = fma_bf16_sel<1, 1>(gw[j], xw[sl(k)][j], a);
+                        }
+                        sw[k] = a;
+                    }
+                    for (int o = 1; o < lanes; o <<= 1)
+#pragma unroll
+                        for (int k = 0; k < W; ++k) sw[k] += __shfl_xor_sync(0xffffffffu, sw[k], o);
+                    if (active && (v % lanes) == 0) {
+                        float *q = dw + ((row0 + t) * NG + c0 / G) * W;
+#pragma unroll
+                        for (int k = 0; k < W; ++k) q[k] = sw[k];
+                    }
+                }
+            };
+            const int nb = cdiv(t1e - t0, KU);
+            issue(t0, 0);
+            for (int bi = 0; bi < nb; ++bi) {
+                const int tb = t0 + bi * KU, stage = bi & 1;
+                if (bi + 1 < nb) issue(tb + KU, stage ^ 1);
+                else cp_commit();
+                cp_wait<1>();
+                if (kRing && ring) {
+#pragma unroll
+                    for (int u = 0; u < KU; ++u) {
+                        if (tb + u >= t1e) break;
+                        token(tb + u, stage, u, [&](int k) { return (u - k + W) % W; });
+                    }
+                } else {
+#pragma unroll
+                    for (int u = 0; u < KU; ++u) {
+                        if (tb + u >= t1e) break;
+                        // open rows move down before the token (slot 0 is row t), x rows
+                        // after it (xw[k] = x[t-k] while the token runs)
+#pragma unroll
+                        for (int k = W - 1; k >= 1; --k)
+#pragma unroll
+                            for (int i = 0; i < V; ++i) acc[k][i] = acc[k - 1][i];
+                        token(tb + u, stage, u, [](int k) { return k; });
+#pragma unroll
+                        for (int k = W - 1; k >= 1; --k)
+#pragma unroll
+                            for (int j = 0; j < NW; ++j) xw[k][j] = xw[k - 1][j];
+                    }
+                }
+            }
+            cp_wait<0>();
+            // at the sequence end the rows still open have all their contributions: rows
+            // T-W+1 .. T-1, in slots (row - t0) % W (ring) or T-1-row (shift)
+            if (t1e == T_) {
+                auto store_open = [&](auto sl_of_row) {
+#pragma unroll
+                    for (int k = 1; k < W; ++k) {
+                        const int s = T_ - W + k;
+                        if (active && s >= t0 && s < t1) P::store(ob + (size_t)s * D, acc[sl_of_row(k)]);
+                    }
+                };
+                if (kRing && ring) {
+                    // slot of row T-W+k is (T - t0 - W + k) % W = (p + k) % W, p = (T - t0) % W
+                    const int p = (T_ - t0) % W;
+#pragma unroll
+                    for (int pp = 0; pp < W; ++pp)
+                        if (pp == p) store_open([&](int k) { return (pp + k) % W; });
+                } else {
+                    store_open([](int k) { return W - 1 - k; });   // row T-W+k = (T-1) - (W-1-k)
+                }
+            }
+        } else {
         float acc[W][V];                             // acc[k] = open dx row t-k
         float xw[W][V];                              // xw[k] = x[t-k]
 #pragma unroll
@@ -436,6 +727,7 @@ k_dyn_bwd(const T *__restrict__ x, const T *__restrict__ w, const T *__restrict_
                 if (active && s >= t0 && s < t1) P::store(ob + (size_t)s * D, acc[W - 1]);
             }
         }
+        }
     }
 }
 
@@ -475,41 +767,188 @@ __device__ __forceinline__ void static_bwd_item(const T *__restrict__ x, const T
         for (int i = 0; i < V; ++i) acc[k][i] = 0.f;
 
     if (active && t0 < t1) {
+      if constexpr (sizeof(T) == 2) {
+        // bf16: rows and taps stay packed (two channels a word) and every product is a
+        // mixed fma.rn.f32.bf16 (exact product, one rounding: the same results as widening
+        // first), which halves the registers the windows take and needs no unpacking
+        constexpr int NW = V / 2;
+        using RT = typename P::raw_t;
+        auto words = [](const RT &r, uint32_t (&o)[NW]) {
+            const uint32_t *q = reinterpret_cast<const uint32_t *>(&r);
+#pragma unroll
+            for (int j = 0; j < NW; ++j) o[j] = q[j];
+        };
+        uint32_t fw[W][NW];          // (w[c0+2j, k], w[c0+2j+1, k])
+        {
+            const uint16_t *wr = reinterpret_cast<const uint16_t *>(ws);
+#pragma unroll
+            for (int j = 0; j < NW; ++j)
+#pragma unroll
+                for (int k = 0; k < W; ++k)
+                    fw[k][j] = (uint32_t)__ldg(wr + (size_t)(c0 + 2 * j) * W + k) |
+                               ((uint32_t)__ldg(wr + (size_t)(c0 + 2 * j + 1) * W + k) << 16);
+        }
+        constexpr bool kRing = kU % W == 0;
+        const bool ring = kRing && (t1 - t0) % W == 0;
+        uint32_t xw[W][NW], dyw[W][NW];
+#pragma unroll
+        for (int k = 1; k < W; ++k) {
+            uint32_t r[NW];
+            if (t0 - k >= 0) words(P::load(x + off + (size_t)(t0 - k) * D), r);
+            else
+#pragma unroll
+                for (int j = 0; j < NW; ++j) r[j] = 0u;
+            const int sk = (kRing && ring) ? W - k : k;      // slot of row t0-k
+#pragma unroll
+            for (int j = 0; j < NW; ++j) {
+                xw[sk][j] = r[j];
+                dyw[sk][j] = 0u;        // rows before t0 feed no dx row of this chunk
+            }
+        }
+        auto step = [&](int t, bool in_chunk, auto sl) {
+            if (in_chunk) {
+#pragma unroll
+                for (int k = 0; k < W; ++k)
+#pragma unroll
+                    for (int j = 0; j < NW; ++j) {
+                        acc[k][2 * j] = fma_bf16_lo(dyw[sl(0)][j], xw[sl(k)][j], acc[k][2 * j]);
+                        acc[k][2 * j + 1] = fma_bf16_hi(dyw[sl(0)][j], xw[sl(k)][j], acc[k][2 * j + 1]);
+                    }
+            }
+            const int s = t - (W - 1);
+            if (s >= t0) {
+                float o[V];
+#pragma unroll
+                for (int j = 0; j < NW; ++j) {
+                    float a0 = bf16_lo(dyw[sl(W - 1)][j]), a1 = bf16_hi(dyw[sl(W - 1)][j]);
+#pragma unroll
+                    for (int k = 0; k < W; ++k) {
+                        a0 = fma_bf16_lo(fw[k][j], dyw[sl(W - 1 - k)][j], a0);
+                        a1 = fma_bf16_hi(fw[k][j], dyw[sl(W - 1 - k)][j], a1);
+                    }
+                    o[2 * j] = a0;
+                    o[2 * j + 1] = a1;
+                }
+                P::store(dx + off + (size_t)s * D, o);
+            }
+        };
+        auto shift = [&]() {
+#pragma unroll
+            for (int k = W - 1; k >= 1; --k)
+#pragma unroll
+                for (int j = 0; j < NW; ++j) {
+                    dyw[k][j] = dyw[k - 1][j];
+                    xw[k][j] = xw[k - 1][j];
+                }
+        };
+        const Staging<P::BYTES, 2, kU, kBX * kBY> stg((uint32_t)__cvta_generic_to_shared(stg_raw),
+                                                  (int)(threadIdx.y * kBX + threadIdx.x));
+        auto issue = [&](int tb, int stage) {
+#pragma unroll
+            for (int u = 0; u < kU; ++u) {
+                const bool ok = tb + u < t1;
+                const size_t r = (size_t)(ok ? tb + u : t0) * D;
+                cp_async<P::BYTES>(stg.at(stage, 0, u), x + off + r, ok);
+                cp_async<P::BYTES>(stg.at(stage, 1, u), dy + off + r, ok);
+            }
+            cp_commit();
+        };
+        const int nb = cdiv(t1 - t0, kU);
+        issue(t0, 0);
+        for (int bi = 0; bi < nb; ++bi) {
+            const int tb = t0 + bi * kU, stage = bi & 1;
+            if (bi + 1 < nb) issue(tb + kU, stage ^ 1);
+            else cp_commit();
+            cp_wait<1>();
+            if (kRing && ring) {
+#pragma unroll
+                for (int u = 0; u < kU; ++u) {
+                    if (tb + u >= t1) break;
+                    const int s0 = u % W;
+                    words(lds_raw<RT>(stg.at(stage, 0, u)), xw[s0]);
+                    words(lds_raw<RT>(stg.at(stage, 1, u)), dyw[s0]);
+                    step(tb + u, true, [&](int k) { return (u - k + W) % W; });
+                }
+            } else {
+#pragma unroll
+                for (int u = 0; u < kU; ++u) {
+                    if (tb + u >= t1) break;
+                    words(lds_raw<RT>(stg.at(stage, 0, u)), xw[0]);
+                    words(lds_raw<RT>(stg.at(stage, 1, u)), dyw[0]);
+                    step(tb + u, true, [](int k) { return k; });
+                    shift();
+                }
+            }
+        }
+        cp_wait<0>();
+        // rows t1-W+1 .. t1-1 need dy rows t1 .. t1+W-2 (zero past the sequence end)
+#pragma unroll
+        for (int e = 0; e < W - 1; ++e) {
+            const int t = t1 + e;
+            uint32_t r[NW];
+            if (t < T_) words(P::load(dy + off + (size_t)t * D), r);
+            else
+#pragma unroll
+                for (int j = 0; j < NW; ++j) r[j] = 0u;
+            if (kRing && ring) {       // row t1+e is in slot e % W
+#pragma unroll
+                for (int j = 0; j < NW; ++j) dyw[e % W][j] = r[j];
+                step(t, false, [&](int k) { return (e - k + W) % W; });
+            } else {
+#pragma unroll
+                for (int j = 0; j < NW; ++j) dyw[0][j] = r[j];
+                step(t, false, [](int k) { return k; });
+                shift();
+            }
+        }
+      } else {
         float f[W][V];
 #pragma unroll
         for (int i = 0; i < V; ++i)
 #pragma unroll
             for (int k = 0; k < W; ++k) f[k][i] = to_f(__ldg(ws + (size_t)(c0 + i) * W + k));
+        // The windows of x and dy rows: a ring (row r in slot (r - t0) % W, a constant in
+        // every unrolled step, no copies) when a batch is a whole number of windows and
+        // the chunk is too; else shifted down one slot per token (xw[k] = row t-k).
+        constexpr bool kRing = kU % W == 0;
+        const bool ring = kRing && (t1 - t0) % W == 0;
         float xw[W][V], dyw[W][V];
 #pragma unroll
         for (int k = 1; k < W; ++k) {
-#pragma unroll
-            for (int i = 0; i < V; ++i) dyw[k][i] = 0.f;   // rows before t0 feed no dx row of this chunk
-            if (t0 - k >= 0) P::unpack(P::load(x + off + (size_t)(t0 - k) * D), xw[k]);
+            float r[V];
+            if (t0 - k >= 0) P::unpack(P::load(x + off + (size_t)(t0 - k) * D), r);
             else
 #pragma unroll
-                for (int i = 0; i < V; ++i) xw[k][i] = 0.f;
+                for (int i = 0; i < V; ++i) r[i] = 0.f;
+            const int sk = (kRing && ring) ? W - k : k;      // slot of row t0-k
+#pragma unroll
+            for (int i = 0; i < V; ++i) {
+                xw[sk][i] = r[i];
+                dyw[sk][i] = 0.f;       // rows before t0 feed no dx row of this chunk
+            }
         }
-        auto step = [&](int t, bool in_chunk) {
-            // dyw[0] and (in the chunk) xw[0] hold row t
+        // one token t, its x and dy rows already in slot sl(0); sl(k) is the slot of row t-k
+        auto step = [&](int t, bool in_chunk, auto sl) {
             if (in_chunk) {
 #pragma unroll
                 for (int k = 0; k < W; ++k)
 #pragma unroll
-                    for (int i = 0; i < V; ++i) acc[k][i] = fmaf(dyw[0][i], xw[k][i], acc[k][i]);
+                    for (int i = 0; i < V; ++i) acc[k][i] = fmaf(dyw[sl(0)][i], xw[sl(k)][i], acc[k][i]);
             }
             const int s = t - (W - 1);
             if (s >= t0) {
                 float o[V];
 #pragma unroll
                 for (int i = 0; i < V; ++i) {
-                    float a = dyw[W - 1][i];
+                    float a = dyw[sl(W - 1)][i];
 #pragma unroll
-                    for (int k = 0; k < W; ++k) a = fmaf(f[k][i], dyw[W - 1 - k][i], a);
+                    for (int k = 0; k < W; ++k) a = fmaf(f[k][i], dyw[sl(W - 1 - k)][i], a);
                     o[i] = a;
                 }
                 P::store(dx + off + (size_t)s * D, o);
             }
+        };
+        auto shift = [&]() {
 #pragma unroll
             for (int k = W - 1; k >= 1; --k)
 #pragma unroll
@@ -537,12 +976,24 @@ __device__ __forceinline__ void static_bwd_item(const T *__restrict__ x, const T
             if (bi + 1 < nb) issue(tb + kU, stage ^ 1);
             else cp_commit();
             cp_wait<1>();
+            if (kRing && ring) {
 #pragma unroll
-            for (int u = 0; u < kU; ++u) {
-                if (tb + u >= t1) break;
-                P::unpack(lds_raw<typename P::raw_t>(stg.at(stage, 0, u)), xw[0]);
-                P::unpack(lds_raw<typename P::raw_t>(stg.at(stage, 1, u)), dyw[0]);
-                step(tb + u, true);
+                for (int u = 0; u < kU; ++u) {
+                    if (tb + u >= t1) break;
+                    const int s0 = u % W;
+                    P::unpack(lds_raw<typename P::raw_t>(stg.at(stage, 0, u)), xw[s0]);
+                    P::unpack(lds_raw<typename P::raw_t>(stg.at(stage, 1, u)), dyw[s0]);
+                    step(tb + u, true, [&](int k) { return (u - k + W) % W; });
+                }
+            } else {
+#pragma unroll
+                for (int u = 0; u < kU; ++u) {
+                    if (tb + u >= t1) break;
+                    P::unpack(lds_raw<typename P::raw_t>(stg.at(stage, 0, u)), xw[0]);
+                    P::unpack(lds_raw<typename P::raw_t>(stg.at(stage, 1, u)), dyw[0]);
+                    step(tb + u, true, [](int k) { return k; });
+                    shift();
+                }
             }
         }
         cp_wait<0>();
@@ -550,12 +1001,23 @@ __device__ __forceinline__ void static_bwd_item(const T *__restrict__ x, const T
 #pragma unroll
         for (int e = 0; e < W - 1; ++e) {
             const int t = t1 + e;
-            if (t < T_) P::unpack(P::load(dy + off + (size_t)t * D), dyw[0]);
+            float r[V];
+            if (t < T_) P::unpack(P::load(dy + off + (size_t)t * D), r);
             else
 #pragma unroll
-                for (int i = 0; i < V; ++i) dyw[0][i] = 0.f;
-            step(t, false);
+                for (int i = 0; i < V; ++i) r[i] = 0.f;
+            if (kRing && ring) {       // row t1+e is in slot e % W
+#pragma unroll
+                for (int i = 0; i < V; ++i) dyw[e % W][i] = r[i];
+                step(t, false, [&](int k) { return (e - k + W) % W; });
+            } else {
+#pragma unroll
+                for (int i = 0; i < V; ++i) dyw[0][i] = r[i];
+                step(t, false, [](int k) { return k; });
+                shift();
+            }
         }
+      }
     }
 #pragma unroll
     for (int k = 0; k < W; ++k) {

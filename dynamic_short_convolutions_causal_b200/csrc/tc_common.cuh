@@ -292,20 +292,6 @@ __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
     return d;
 }
 
-// c + (low or high bf16 half of a) * (same half of b) in fp32: the product of two bf16
-// values is exact in fp32, so this equals fmaf on the widened values (one rounding).
-__device__ __forceinline__ float fma_bf16_lo(uint32_t a, uint32_t b, float c) {
-    float d;
-    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
-        "fma.rn.f32.bf16 %0, al, bl, %3;\n\t}" : "=f"(d) : "r"(a), "r"(b), "f"(c));
-    return d;
-}
-__device__ __forceinline__ float fma_bf16_hi(uint32_t a, uint32_t b, float c) {
-    float d;
-    asm("{\n\t.reg .b16 al, ah, bl, bh;\n\tmov.b32 {al, ah}, %1;\n\tmov.b32 {bl, bh}, %2;\n\t"
-        "fma.rn.f32.bf16 %0, ah, bh, %3;\n\t}" : "=f"(d) : "r"(a), "r"(b), "f"(c));
-    return d;
-}
 
 // Packed fp32 pair arithmetic (sm_100): d = a * b + c on both halves.
 __device__ __forceinline__ uint64_t f2pack(float lo, float hi) {

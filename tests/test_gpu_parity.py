@@ -55,6 +55,11 @@ EXPLICIT = [
     (2, 45, 24, 3, 5, "bf16"),
     (2, 33, 96, 96, 2, "f32"),
     (1, 130, 40, 5, 7, "f32"),
+    # one-pass explicit backward, packed bf16: ring windows with a ragged last chunk
+    # (W=4: the open rows' slots depend on T mod 4; W=2), and shifted windows (W=8)
+    (1, 131, 128, 16, 4, "bf16"),
+    (2, 260, 64, 8, 2, "bf16"),
+    (2, 300, 128, 8, 8, "bf16"),
 ]
 
 
