@@ -48,6 +48,9 @@ constexpr unsigned kWaitHint = 2000;
 #ifndef DSC_FWD_SETS
 #define DSC_FWD_SETS 2         // epilogue warp sets working on alternating tiles (1 or 2)
 #endif
+#ifndef DSC_FWD_CHPAIR
+#define DSC_FWD_CHPAIR 1       // groups of 4+ channels: fp32x2 FMAs over channel pairs
+#endif
 #ifndef DSC_FWD_F32X2
 #define DSC_FWD_F32X2 2        // pair taps with packed fp32x2 FMAs: 1 always, 0 never, 2 for W <= 4
 #endif
@@ -153,29 +156,47 @@ __device__ __forceinline__ void conv_chunk(const uint32_t *wr, const uint4 (&xu)
     float xv[W][8];
 #pragma unroll
     for (int k = 0; k < W; ++k) unpack8(xu[k], xv[k]);
+    if constexpr (GC >= 4 && DSC_FWD_CHPAIR) {
+        // a group spans at least 4 channels: channel pairs (2m, 2m+1) share its taps, so
+        // packed fp32x2 FMAs take the two channels at once (each tap duplicated once per
+        // group; the same fmaf sequence per channel as the scalar form)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        const int gl = GC <= 8 ? e / GC : 0;
-        const uint32_t *wg = wr + gl * W;
-        // measured: the packed form is faster with 4 taps (lowrank_qkv 0.095 -> 0.091 ms)
-        // and slower with 8 (lowrank_mlp 0.145 -> 0.157 ms)
-        constexpr bool kPair = DSC_FWD_F32X2 == 1 || (DSC_FWD_F32X2 == 2 && W <= 4);
-        if constexpr (kPair && W >= 2) {
-            // taps in pairs with packed fp32x2 FMAs (two partial sums, added at the end)
-            uint64_t acc = f2pack(xv[0][e], 0.f);
+        for (int m = 0; m < 4; ++m) {
+            const int gl = GC <= 8 ? (2 * m) / GC : 0;
+            const uint32_t *wg = wr + gl * W;
+            uint64_t acc = f2pack(xv[0][2 * m], xv[0][2 * m + 1]);
 #pragma unroll
-            for (int k = 0; k + 1 < W; k += 2)
-                acc = f2fma(f2pack(__uint_as_float(wg[k]), __uint_as_float(wg[k + 1])),
-                            f2pack(xv[k][e], xv[k + 1][e]), acc);
-            float a0, a1;
-            f2unpack(acc, a0, a1);
-            if (W & 1) a0 = fmaf(__uint_as_float(wg[W - 1]), xv[W - 1][e], a0);
-            out[e] = a0 + a1;
-        } else {
-            float acc = xv[0][e];
+            for (int k = 0; k < W; ++k) {
+                const float wk = __uint_as_float(wg[k]);
+                acc = f2fma(f2pack(wk, wk), f2pack(xv[k][2 * m], xv[k][2 * m + 1]), acc);
+            }
+            f2unpack(acc, out[2 * m], out[2 * m + 1]);
+        }
+    } else {
 #pragma unroll
-            for (int k = 0; k < W; ++k) acc = fmaf(__uint_as_float(wg[k]), xv[k][e], acc);
-            out[e] = acc;
+        for (int e = 0; e < 8; ++e) {
+            const int gl = GC <= 8 ? e / GC : 0;
+            const uint32_t *wg = wr + gl * W;
+            // measured: the packed form is faster with 4 taps (lowrank_qkv 0.095 -> 0.091 ms)
+            // and slower with 8 (lowrank_mlp 0.145 -> 0.157 ms)
+            constexpr bool kPair = DSC_FWD_F32X2 == 1 || (DSC_FWD_F32X2 == 2 && W <= 4);
+            if constexpr (kPair && W >= 2) {
+                // taps in pairs with packed fp32x2 FMAs (two partial sums, added at the end)
+                uint64_t acc = f2pack(xv[0][e], 0.f);
+#pragma unroll
+                for (int k = 0; k + 1 < W; k += 2)
+                    acc = f2fma(f2pack(__uint_as_float(wg[k]), __uint_as_float(wg[k + 1])),
+                                f2pack(xv[k][e], xv[k + 1][e]), acc);
+                float a0, a1;
+                f2unpack(acc, a0, a1);
+                if (W & 1) a0 = fmaf(__uint_as_float(wg[W - 1]), xv[W - 1][e], a0);
+                out[e] = a0 + a1;
+            } else {
+                float acc = xv[0][e];
+#pragma unroll
+                for (int k = 0; k < W; ++k) acc = fmaf(__uint_as_float(wg[k]), xv[k][e], acc);
+                out[e] = acc;
+            }
         }
     }
 }
