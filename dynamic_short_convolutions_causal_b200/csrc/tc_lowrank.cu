@@ -392,6 +392,23 @@ __device__ __forceinline__ void fwd_tiles(const CUtensorMap &tm_x, const CUtenso
         const int dslice = step % p.n_slices, dtl = step / p.n_slices;
         for (; i < p.n_tiles; i += step) {
             const int t0 = tt * kTt;
+            // RoPE (when on): channel pairs (2i, 2i+1) of the first n_rot channels rotated by
+            // the angle of pair i = (c mod dh) / 2 at this row's position in its sequence.
+            // A chunk's 4 (cos, sin) pairs are read one chunk ahead (the first before the
+            // waits); the table is pair-major, so a warp's 32 rows read 256 contiguous bytes.
+            const int c_warp = slice * kDt + ES::CPW * h;
+            const bool rot_row = ROPE && t0 + row < p.T;
+            float2 csn[4];
+            auto load_cs = [&](int cq) {
+                const int c8 = c_warp + 8 * cq;
+                if (rot_row && c8 < p.n_rot) {
+                    const float2 *src = reinterpret_cast<const float2 *>(p.cs) +
+                                        (size_t)((c8 % p.dh) / 2) * p.T + (t0 + row);
+#pragma unroll
+                    for (int m2 = 0; m2 < 4; ++m2) csn[m2] = __ldg(src + (size_t)m2 * p.T);
+                }
+            };
+            if (ROPE) load_cs(0);
             if (!warp_wait<kWaitHint>(bar.full(s), n & 1, abort, 32u, &g_fault, p.wt.wait_ns)) break;
             if (!warp_wait<kWaitHint>(bar.accf(a), m & 1, abort, 64u, &g_fault, p.wt.wait_ns)) break;
             tc_fence_after();
@@ -416,24 +433,17 @@ __device__ __forceinline__ void fwd_tiles(const CUtensorMap &tm_x, const CUtenso
                 }
             };
             issue_taps(0, wr[0]);
-            // RoPE (when on): channel pairs (2i, 2i+1) of the first n_rot channels rotated by
-            // the angle of pair i = (c mod dh) / 2 at this row's position in its sequence
-            const int c_warp = slice * kDt + ES::CPW * h;
-            const bool rot_row = ROPE && t0 + row < p.T;
 #pragma unroll
             for (int cq = 0; cq < ES::CHUNKS; ++cq) {
                 uint4 xu[W];
 #pragma unroll
                 for (int k = 0; k < W; ++k) xu[k] = lds128(xs + (xrow[k] ^ ((uint32_t)cq << 4)));
                 float2 csv[4];
-                const int c8 = c_warp + 8 * cq;
-                const bool rot = rot_row && c8 < p.n_rot;
-                if (rot) {      // the chunk's 4 pairs, read ahead of the math; the table is
-                                // pair-major, so a warp's 32 rows read 256 contiguous bytes
-                    const float2 *src = reinterpret_cast<const float2 *>(p.cs) +
-                                        (size_t)((c8 % p.dh) / 2) * p.T + (t0 + row);
+                const bool rot = rot_row && c_warp + 8 * cq < p.n_rot;
+                if (ROPE) {
 #pragma unroll
-                    for (int m2 = 0; m2 < 4; ++m2) csv[m2] = __ldg(src + (size_t)m2 * p.T);
+                    for (int m2 = 0; m2 < 4; ++m2) csv[m2] = csn[m2];
+                    if (cq + 1 < ES::CHUNKS) load_cs(cq + 1);
                 }
                 tmem_wait_ld_regs(wr[cq & 1]);
                 if (cq + 1 < ES::CHUNKS) issue_taps(cq + 1, wr[(cq + 1) & 1]);   // overlaps the math below
