@@ -38,6 +38,8 @@ CASES = [
     (2, 200, 384, 2, 4, 32, 128, 256),      # two thirds, as in a stacked QKV
     (1, 77, 128, 16, 2, 32, 16, 64),        # grouped filters, small heads
     (2, 150, 128, 1, 4, 32, 64, 0),         # nothing rotated: the plain op
+    (1, 140, 128, 1, 6, 16, 32, 128),       # 6 taps: products stored as computed
+    (2, 100, 256, 32, 4, 32, 64, 128),      # one filter per 32 channels (virtual groups)
 ]
 
 
