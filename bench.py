@@ -412,7 +412,8 @@ def measure_comparators(dsc, dev, peak, args):
     """Other paths timed in the same run, each on its own workload: the in-repo static
     depthwise causal convolution (the primitive the method generalises) on the MLP-width
     shape, the fused low-rank step on the MLP-width shape, the stacked-QKV step with RoPE
-    fused, the explicit-filter forward on the stacked-QKV shape, and the decode step.
+    fused, the explicit-filter forward and backward on the stacked-QKV shape, and the decode
+    steps (low-rank and explicit filters).
     Inputs exceed L2; times are CUDA events per call."""
     stream = torch.cuda.current_stream(dev)
     steps = max(3, min(args.steps, 10))
@@ -539,6 +540,23 @@ def measure_comparators(dsc, dev, peak, args):
                     "sequence (w = z U by tcgen05, window moved by TMA stores), below it a "
                     "CUDA-core kernel"}
         del U, x, z, st, y
+        # explicit-filter decode step (tied filters of the tied_qkv shape: w_t [B, D/G, W])
+        wle = di.WORKLOADS["tied_qkv"]
+        Ge, We = wle.G, wle.W
+        dec = {}
+        for B in (1, 8, 64, 256, 512):
+            x = torch.randn((B, D), generator=gen, device=dev).to(torch.bfloat16)
+            w = (torch.randn((B, D // Ge, We), generator=gen, device=dev) * 0.5).to(torch.bfloat16)
+            st = torch.randn((B, We - 1, D), generator=gen, device=dev).to(torch.bfloat16)
+            y = torch.empty_like(x)
+            ms = _time_graph(lambda: dsc.dsc_decode_step(x, w, st, y, Ge), dev, 100)
+            nb = B * (D * 2 + (D // Ge) * We * 2 + 2 * (We - 1) * D * 2 + D * 2)
+            dec["B=%d" % B] = {"us": ms * 1e3, "algorithmic_bytes": nb, "gbs": nb / (ms * 1e-3) / 1e9,
+                               "frac_of_hbm_peak": nb / (ms * 1e-3) / 1e9 / peak, "tokens_per_s": B / (ms * 1e-3)}
+        out["decode_explicit_" + wle.name.split("_", 1)[1]] = {
+            "shape": {"D": D, "G": Ge, "W": We}, "per_batch": dec,
+            "note": "as decode_lowrank_qkv, with the step's filters given (CUDA cores)"}
+        del x, w, st, y
         torch.cuda.empty_cache()
     return out
 
