@@ -147,6 +147,64 @@ k_decode_lowrank(const T *__restrict__ x_t, const T *__restrict__ z_t, const T *
     }
 }
 
+// Low-rank decode for a few sequences (B <= kSmB): a block owns 64 channels; each thread
+// forms 4 filter columns of them for every sequence straight from U in global memory
+// (its R row loads are independent and issued together: one memory round trip, no U
+// staging and no padded sequence rows), then the block applies the convolution, one
+// thread per (sequence, 4 channels).  Needs the block's first column and N to be
+// multiples of 4 (checked on the host).
+constexpr int kSmCh = 64;          // channels per block
+constexpr int kSmB = 4;            // largest batch
+constexpr int kSmThreads = 128;
+
+template <typename T, int W>
+__global__ void __launch_bounds__(kSmThreads)
+k_decode_lowrank_small(const T *__restrict__ x_t, const T *__restrict__ z_t, const T *__restrict__ U,
+                       T *__restrict__ state, T *__restrict__ y_t, int B, int D, int G, int R) {
+    extern __shared__ float dsm[];
+    const int N = (D / G) * W;
+    const int cb = blockIdx.x * kSmCh;
+    const int ce = min(cb + kSmCh, D);
+    const int g0 = cb / G, g1 = (ce - 1) / G;
+    const int ncol = (g1 - g0 + 1) * W;                // this block's filter columns
+    const int col0 = g0 * W;
+    float *zs = dsm;                                   // [B][R]
+    float *ws = zs + kSmB * R;                         // [B][ncol]
+    const int tid = threadIdx.x;
+    for (int e = tid; e < B * R; e += kSmThreads) zs[e] = to_f(z_t[e]);
+    __syncthreads();
+    for (int q = tid; 4 * q < ncol; q += kSmThreads) {
+        float acc[kSmB][4] = {};
+        const T *up = U + col0 + 4 * q;
+#pragma unroll 16
+        for (int r = 0; r < R; ++r) {
+            float u[4];
+            ld4(up + (size_t)r * N, u);
+            float zb[kSmB];
+#pragma unroll
+            for (int b = 0; b < kSmB; ++b) zb[b] = b < B ? zs[b * R + r] : 0.f;
+#pragma unroll
+            for (int b = 0; b < kSmB; ++b)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[b][i] = fmaf(zb[b], u[i], acc[b][i]);
+        }
+#pragma unroll
+        for (int b = 0; b < kSmB; ++b)
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+                if (b < B && 4 * q + i < ncol) ws[b * ncol + 4 * q + i] = acc[b][i];
+    }
+    __syncthreads();
+    const int nv = (ce - cb) / 4;
+    for (int task = tid; task < B * nv; task += kSmThreads) {
+        const int b = task / nv, v = task - b * nv;
+        const int c0 = cb + 4 * v;
+        const float *wb = ws + b * ncol;
+        decode_conv<T, W>(x_t, state, y_t, (size_t)b, c0, D,
+                          [&](int e, int k) { return wb[((c0 + e) / G - g0) * W + k]; });
+    }
+}
+
 // Explicit-filter decode: w_t [B, D/G, W]; one thread per (sequence, 4 channels).
 template <typename T, int W>
 __global__ void __launch_bounds__(256)
@@ -171,9 +229,33 @@ size_t decode_smem(int D, int G, int W, int R) {
     return sizeof(float) * ((size_t)R * kDcSeq + (size_t)R * 4 * nq + (size_t)kDcSeq * 4 * nq);
 }
 
+// The small-batch kernel's conditions: at most kSmB sequences, a rank of at most 32 (a
+// thread's R loads of U in flight at once; with R = 64 and 8 taps it measured slower,
+// 5.49 -> 5.89 us at B = 1), whole 4-channel vectors per block, and filter columns that
+// start every block (and every row of U) on a multiple of 4.  D=6144, R=32, W=4: B = 1
+// 4.76 -> 3.79 us, B = 4 5.06 -> 3.83 us.
+bool decode_small_ok(int B, int D, int G, int W, int R) {
+    return B <= kSmB && R <= 32 && D % 4 == 0 && G <= kSmCh && kSmCh % G == 0 && ((kSmCh / G) * W) % 4 == 0 &&
+           ((D / G) * W) % 4 == 0;
+}
+size_t decode_small_smem(int G, int W, int R) {
+    return sizeof(float) * ((size_t)kSmB * R + (size_t)kSmB * (kSmCh / G + 1) * W);
+}
+
 template <typename T, int W>
 cudaError_t launch_dl(const void *x, const void *z, const void *U, void *st, void *y, int B, int D, int G, int R,
                       cudaStream_t s) {
+    if (decode_small_ok(B, D, G, W, R)) {
+        const size_t smem = decode_small_smem(G, W, R);
+        auto kern = k_decode_lowrank_small<T, W>;
+        if (smem > 48 * 1024) {
+            const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+            if (e != cudaSuccess) return e;
+        }
+        kern<<<cdiv(D, kSmCh), kSmThreads, smem, s>>>((const T *)x, (const T *)z, (const T *)U, (T *)st, (T *)y,
+                                                      B, D, G, R);
+        return cudaGetLastError();
+    }
     const size_t smem = decode_smem(D, G, W, R);
     auto kern = k_decode_lowrank<T, W>;
     if (smem > 48 * 1024) {

@@ -37,6 +37,10 @@ DECODE = [
     (3, 40, 8, 3, 16, "f32"),          # D not a multiple of the 32-channel block
     (5, 64, 1, 1, 4, "bf16"),          # W = 1: no window
     (2, 128, 64, 2, 48, "bf16"),
+    # up to 4 sequences with rank <= 32: U read straight from global memory
+    (4, 256, 4, 2, 8, "f32"),
+    (2, 512, 16, 4, 16, "bf16"),
+    (2, 96, 1, 4, 8, "bf16"),          # a last block of 32 channels
     # tensor-core decode (the forward kernel with one row per sequence)
     (256, 6144, 1, 4, 32, "bf16"),     # two full 128-sequence tiles
     (130, 128, 2, 8, 16, "bf16"),      # a ragged second tile, W = 8
