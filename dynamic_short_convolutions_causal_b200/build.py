@@ -5,7 +5,8 @@
 (run as a script: importing the package itself needs the built library)
 
 Each .cu under csrc/ is compiled to an object in csrc/_build/ (rebuilt when it or any
-header is newer), then linked into libdsc.so next to this file.
+header is newer; the files compile in parallel), then linked into libdsc.so next to
+this file.
 """
 from __future__ import annotations
 
@@ -36,17 +37,23 @@ def build(force: bool = False, verbose: bool = False, ptxas_verbose: bool = Fals
     os.makedirs(OBJ, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     hdr_time = max(os.path.getmtime(h) for h in _headers())
-    objs = []
+    objs, cmds = [], []
     for src in srcs:
         obj = os.path.join(OBJ, os.path.basename(src)[:-3] + ".o")
         objs.append(obj)
         if (not force and os.path.exists(obj) and os.path.getmtime(obj) >= os.path.getmtime(src)
                 and os.path.getmtime(obj) >= hdr_time):
             continue
-        cmd = [NVCC] + ARCH + FLAGS + (["-Xptxas", "-v"] if ptxas_verbose else []) + ["-c", src, "-o", obj]
-        if verbose:
+        cmds.append([NVCC] + ARCH + FLAGS + (["-Xptxas", "-v"] if ptxas_verbose else []) + ["-c", src, "-o", obj])
+    # compile in parallel (the tensor-core backward alone takes most of the time)
+    if verbose:
+        for cmd in cmds:
             print(" ".join(cmd), flush=True)
-        subprocess.run(cmd, check=True)
+    if cmds:
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(max_workers=max(1, min(len(cmds), os.cpu_count() or 1))) as ex:
+            for f in [ex.submit(subprocess.run, cmd, check=True) for cmd in cmds]:
+                f.result()          # re-raises a failed compile
     if force or not os.path.exists(LIB) or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
         tmp = LIB + ".tmp.%d" % os.getpid()
         cmd = [NVCC] + ARCH + ["-shared", "-o", tmp] + objs + ["-lcudart"]
