@@ -41,6 +41,9 @@ DECODE = [
     (4, 256, 4, 2, 8, "f32"),
     (2, 512, 16, 4, 16, "bf16"),
     (2, 96, 1, 4, 8, "bf16"),          # a last block of 32 channels
+    (3, 104, 1, 4, 24, "bf16"),        # a last block of 40 channels
+    (4, 128, 2, 8, 32, "f32"),         # 8 taps, fp32
+    (2, 64, 1, 1, 16, "bf16"),         # W = 1: no window
     # tensor-core decode (the forward kernel with one row per sequence)
     (256, 6144, 1, 4, 32, "bf16"),     # two full 128-sequence tiles
     (130, 128, 2, 8, 16, "bf16"),      # a ragged second tile, W = 8
